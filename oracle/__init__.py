@@ -1,0 +1,152 @@
+"""CPU oracle for weight-only group-64 symmetric int4/int8 quantized products.
+
+TEST INFRASTRUCTURE ONLY.  The product library never imports, links or calls
+anything in this package; only the test suite, the smoke check and the
+benchmark's CPU-baseline leg may.  It shares no code, header, table or helper
+with the CUDA path; the only thing both sides see is the seeded input
+generator module, which holds none of the method's arithmetic.
+
+The arithmetic lives in ``rqo.c`` (plain scalar C, fp32 quantizer exactly as
+defined, fp64 products); this module builds it with gcc and wraps it with
+ctypes.  What it follows, and every reading taken where the pages are silent,
+is written at the top of ``rqo.c``:
+
+  * "Hakureirm/rwkv7-sglang-w4gptq-1.5b" model card, opening summary and
+    "Format & loading (important)": GROUP = 64, symmetric int4, packed codes
+    plus per-group scales, calibration-free round-to-nearest; the kernel output
+    equals the product with the offline-dequantised weight.
+  * same card, "Accuracy warning": the int8 w8g64 tier.
+
+Parity status: the quantizer is pinned bit-exactly (hand-worked examples,
+exact-reconstruction and tie-break cases, an independent numpy restatement,
+invariants); the fp16 converter is pinned against numpy's conversion; the
+products are pinned against an independent numpy fp64 dequantise-then-matmul
+and hand-worked values.  No function is left unpinned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rqo.c")
+_LIB_PATH = os.path.join(_HERE, "_build", "librqo.so")
+_lib = None
+
+GROUP = 64
+QMAX = {4: 7, 8: 127}
+STATUS_OK, STATUS_NONFINITE, STATUS_RANGE = 0, 5, 6
+
+
+def build(force: bool = False) -> str:
+    """Compile rqo.c into oracle/_build/librqo.so (gcc, no fast-math)."""
+    os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+           "-ffp-contract=off", "-fno-fast-math", "-fno-finite-math-only",
+           _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    i64, vp = ctypes.c_int64, ctypes.c_void_p
+    lib.rqo_f32_to_f16.argtypes = [ctypes.c_float]
+    lib.rqo_f32_to_f16.restype = ctypes.c_uint16
+    lib.rqo_f16_to_f64.argtypes = [ctypes.c_uint16]
+    lib.rqo_f16_to_f64.restype = ctypes.c_double
+    lib.rqo_quantize_g64.argtypes = [vp, i64, i64, ctypes.c_int, vp, vp]
+    lib.rqo_quantize_g64.restype = ctypes.c_int
+    lib.rqo_matmul.argtypes = [vp, i64, i64, vp, vp, i64, ctypes.c_int, vp, vp]
+    lib.rqo_matmul.restype = None
+    lib.rqo_matmul_sampled.argtypes = [vp, i64, i64, vp, vp, i64, ctypes.c_int,
+                                       i64, vp, vp, vp, vp]
+    lib.rqo_matmul_sampled.restype = None
+    lib.rqo_get_code.argtypes = [vp, i64, ctypes.c_int, i64, i64]
+    lib.rqo_get_code.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def f32_to_f16_bits(v: float) -> int:
+    """Round-to-nearest-even fp32 -> fp16 bit pattern (the oracle's own)."""
+    return int(_load().rqo_f32_to_f16(ctypes.c_float(v)))
+
+
+def f16_bits_to_f64(h: int) -> float:
+    return float(_load().rqo_f16_to_f64(ctypes.c_uint16(h)))
+
+
+def codes_bytes(N: int, K: int, bits: int) -> int:
+    return N * K * bits // 8
+
+
+def quantize_g64(W: np.ndarray, bits: int):
+    """RTN group-64 quantization of fp32 W[N, K].
+
+    Returns (codes uint8 [N, K*bits/8], scales uint16 fp16-bits [N, K/64],
+    status int)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    if bits not in (4, 8) or K % GROUP:
+        raise ValueError("bits must be 4 or 8 and K a multiple of 64")
+    codes = np.zeros((N, K * bits // 8), dtype=np.uint8)
+    scales = np.zeros((N, K // GROUP), dtype=np.uint16)
+    st = _load().rqo_quantize_g64(_ptr(W), N, K, bits, _ptr(codes), _ptr(scales))
+    return codes, scales, int(st)
+
+
+def matmul(x_f16: np.ndarray, codes: np.ndarray, scales: np.ndarray, bits: int,
+           with_bound: bool = True):
+    """y[M, N] = x @ (c * s16)^T in fp64, plus the budget sum |x||c*s16|.
+
+    x_f16 is float16 (or uint16 fp16 bit patterns) [M, K]."""
+    x = np.ascontiguousarray(x_f16).view(np.uint16)
+    M, K = x.shape
+    N = scales.shape[0]
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales).view(np.uint16)
+    y = np.zeros((M, N), dtype=np.float64)
+    b = np.zeros((M, N), dtype=np.float64) if with_bound else None
+    _load().rqo_matmul(_ptr(x), M, K, _ptr(codes), _ptr(scales), N, bits, _ptr(y),
+                       _ptr(b) if b is not None else None)
+    return (y, b) if with_bound else y
+
+
+def matmul_sampled(x_f16: np.ndarray, codes: np.ndarray, scales: np.ndarray,
+                   bits: int, ms, ns):
+    """y and budget at the sampled outputs (ms[p], ns[p])."""
+    x = np.ascontiguousarray(x_f16).view(np.uint16)
+    M, K = x.shape
+    N = scales.shape[0]
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales).view(np.uint16)
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    P = ms.shape[0]
+    y = np.zeros(P, dtype=np.float64)
+    b = np.zeros(P, dtype=np.float64)
+    _load().rqo_matmul_sampled(_ptr(x), M, K, _ptr(codes), _ptr(scales), N, bits, P,
+                               _ptr(ms), _ptr(ns), _ptr(y), _ptr(b))
+    return y, b
+
+
+def get_code(codes: np.ndarray, K: int, bits: int, n: int, k: int) -> int:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    return int(_load().rqo_get_code(_ptr(codes), K, bits, n, k))

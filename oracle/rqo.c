@@ -1,0 +1,272 @@
+/*
+ * rqo.c -- the ORACLE for weight-only, group-64, symmetric int4/int8
+ * quantized projections.  Plain, slow, scalar C.  Test infrastructure only:
+ * nothing in the product library links, includes or calls this file.  Only
+ * the test suite, the smoke check and the CPU-baseline leg of the benchmark
+ * may load it.
+ *
+ * What it follows:
+ *   - "Hakureirm/rwkv7-sglang-w4gptq-1.5b" model card, opening summary and
+ *     "Format & loading (important)": weights are stored group-wise with
+ *     GROUP = 64, symmetric (no zero point), as packed int4 codes (.qweight)
+ *     plus one scale per group (.scale); the calibration-free variant is plain
+ *     round-to-nearest (RTN); the kernel's output equals a product with the
+ *     offline-dequantised weight.
+ *   - same card, "Accuracy warning": the int8 "w8g64" tier uses the same
+ *     group of 64 with 8-bit codes.
+ *   - "RWKV-7 Quantization Toolkit" (rwkv-quant-nv 1.2.1), "Key Design":
+ *     products are taken directly on the quantized weights; no dequantised
+ *     weight matrix exists on the inference path.  The oracle is the
+ *     definition, so it may dequantise.
+ *
+ * Readings where the pages are silent (each one is listed in the design notes):
+ *   - the group runs along the reduction axis K: 64 consecutive k of one
+ *     output row n of W[N, K];
+ *   - scale: s32 = amax / qmax as one IEEE fp32 division, then s16 =
+ *     round-to-nearest-even of s32 to fp16; the stored scale is s16;
+ *   - codes are computed against the stored scale: c = clamp(rint(w / s16),
+ *     -qmax, qmax) with w / s16 one IEEE fp32 division and rint rounding half
+ *     to even;  qmax = 7 (int4) or 127 (int8);
+ *   - a group whose s16 is zero (all-zero group or an underflowing amax) gets
+ *     codes 0;
+ *   - a group holding a non-finite weight gets scale 0x7E00 (fp16 NaN) and
+ *     codes 0, status NONFINITE;  a group whose s16 overflows to +inf keeps
+ *     scale 0x7C00 and codes 0, status RANGE;
+ *   - int4 packing: byte j of a row holds k = 2j in its low nibble and
+ *     k = 2j + 1 in its high nibble, 4-bit two's complement; int8 codes are
+ *     plain signed bytes; scales are row-major [N, K/64].
+ *   - products: y[m, n] = sum_k x[m, k] * c[n, k] * s16[n, k/64] in fp64, with
+ *     x given as fp16 bit patterns; the per-output error budget is
+ *     B[m, n] = sum_k |x[m, k]| * |c[n, k] * s16[n, k/64]|.
+ *
+ * Build: gcc -O2 -fPIC -shared -fopenmp -ffp-contract=off -fno-fast-math.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define RQO_GROUP 64
+
+/* status values: the same numbering as the library's public header, written
+ * out here on purpose (the oracle includes no header of the product). */
+enum { RQO_OK = 0, RQO_ERR_NONFINITE = 5, RQO_ERR_RANGE = 6 };
+
+/* ---------------------------------------------------------------- fp16 --- */
+
+/* fp32 -> IEEE binary16, round to nearest, ties to even.  Written from the
+ * IEEE 754 binary16 definition: 1 sign bit, 5 exponent bits (bias 15),
+ * 10 fraction bits; subnormals below 2^-14; overflow to infinity. */
+uint16_t rqo_f32_to_f16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+    uint32_t exp = (u >> 23) & 0xFFu;
+    uint32_t man = u & 0x7FFFFFu;
+
+    if (exp == 0xFFu) {                      /* inf or NaN */
+        if (man == 0) return (uint16_t)(sign | 0x7C00u);
+        return (uint16_t)(sign | 0x7E00u);   /* quiet NaN */
+    }
+    int e = (int)exp - 127;                  /* unbiased exponent */
+    if (exp == 0) return sign;               /* fp32 zero/subnormal: < 2^-126, rounds to 0 */
+
+    uint32_t m = man | 0x800000u;            /* 24-bit significand, value m * 2^(e-23) */
+    if (e > 15) return (uint16_t)(sign | 0x7C00u);
+
+    int shift;                               /* right shift applied to m */
+    uint32_t hexp;                           /* biased fp16 exponent before rounding */
+    if (e >= -14) {                          /* normal range: keep 11 bits */
+        shift = 13;
+        hexp = (uint32_t)(e + 15);
+    } else {                                 /* subnormal: value = q * 2^-24 */
+        shift = 13 + (-14 - e);
+        hexp = 0;
+        if (shift > 24) return sign;         /* below half the smallest subnormal */
+    }
+    uint32_t q = m >> shift;
+    uint32_t rem = m & ((1u << shift) - 1u);
+    uint32_t half = 1u << (shift - 1);
+    if (rem > half || (rem == half && (q & 1u))) q += 1u;
+
+    if (hexp == 0) {
+        /* q counts units of 2^-24; q == 0x400 is the smallest normal, which
+         * the bit pattern below encodes correctly by itself */
+        return (uint16_t)(sign | q);
+    }
+    /* q holds 1.fraction in 11 bits, possibly carried to 0x800 */
+    if (q == 0x800u) { q = 0x400u; hexp += 1; }
+    if (hexp >= 31) return (uint16_t)(sign | 0x7C00u);
+    return (uint16_t)(sign | (hexp << 10) | (q & 0x3FFu));
+}
+
+/* IEEE binary16 -> double, exact. */
+double rqo_f16_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int exp = (h >> 10) & 0x1F;
+    int man = h & 0x3FF;
+    double v;
+    if (exp == 0x1F) v = man ? NAN : INFINITY;
+    else if (exp == 0) v = ldexp((double)man, -24);
+    else v = ldexp((double)(man | 0x400), exp - 25);
+    return sign ? -v : v;
+}
+
+/* ------------------------------------------------------------ quantize --- */
+
+static int qmax_of(int bits) { return bits == 4 ? 7 : 127; }
+
+/* Store code c (|c| <= qmax) for element (n, k) in the packed layout. */
+static void put_code(uint8_t *codes, int64_t K, int bits, int64_t n, int64_t k, int c)
+{
+    if (bits == 8) {
+        codes[n * K + k] = (uint8_t)(int8_t)c;
+    } else {
+        uint8_t *b = &codes[n * (K / 2) + k / 2];
+        uint8_t nib = (uint8_t)(c & 0xF);
+        if (k % 2 == 0) *b = (uint8_t)((*b & 0xF0u) | nib);
+        else            *b = (uint8_t)((*b & 0x0Fu) | (nib << 4));
+    }
+}
+
+/* Read back code (n, k) from the packed layout. */
+int rqo_get_code(const uint8_t *codes, int64_t K, int bits, int64_t n, int64_t k)
+{
+    if (bits == 8) return (int)(int8_t)codes[n * K + k];
+    uint8_t b = codes[n * (K / 2) + k / 2];
+    int nib = (k % 2 == 0) ? (b & 0xF) : (b >> 4);
+    return nib >= 8 ? nib - 16 : nib;
+}
+
+/* RTN quantization of one group of 64 weights; returns a status. */
+static int quantize_group(const float *w, int bits, uint16_t *scale_out, int *c_out)
+{
+    const int qmax = qmax_of(bits);
+    int i;
+    for (i = 0; i < RQO_GROUP; i++) {
+        if (!isfinite(w[i])) {
+            *scale_out = 0x7E00u;
+            for (i = 0; i < RQO_GROUP; i++) c_out[i] = 0;
+            return RQO_ERR_NONFINITE;
+        }
+    }
+    /* step 1: amax = max |w| (exact in fp32) */
+    float amax = 0.0f;
+    for (i = 0; i < RQO_GROUP; i++) {
+        float a = fabsf(w[i]);
+        if (a > amax) amax = a;
+    }
+    /* step 2: s32 = amax / qmax, one IEEE fp32 division */
+    volatile float s32 = amax / (float)qmax;
+    /* step 3: s16 = fp16(s32), round to nearest even */
+    uint16_t s16 = rqo_f32_to_f16(s32);
+    *scale_out = s16;
+    /* step 4: codes against the stored scale */
+    float sf = (float)rqo_f16_to_f64(s16);
+    if (s16 == 0x7C00u) {
+        for (i = 0; i < RQO_GROUP; i++) c_out[i] = 0;
+        return RQO_ERR_RANGE;
+    }
+    if (sf == 0.0f) {
+        for (i = 0; i < RQO_GROUP; i++) c_out[i] = 0;
+        return RQO_OK;
+    }
+    for (i = 0; i < RQO_GROUP; i++) {
+        volatile float t = w[i] / sf;        /* IEEE fp32 division */
+        float r = rintf(t);                  /* half to even (default mode) */
+        if (r > (float)qmax) r = (float)qmax;
+        if (r < (float)-qmax) r = (float)-qmax;
+        c_out[i] = (int)r;
+    }
+    return RQO_OK;
+}
+
+/* Quantize W[N, K] (fp32, row-major).  Writes codes (N*K*bits/8 bytes) and
+ * scales (N*(K/64) fp16 bit patterns).  Returns the highest-priority status
+ * seen: NONFINITE over RANGE over OK.  K must be a multiple of 64 and bits
+ * 4 or 8; the caller checks. */
+int rqo_quantize_g64(const float *W, int64_t N, int64_t K, int bits,
+                     uint8_t *codes, uint16_t *scales)
+{
+    const int64_t G = K / RQO_GROUP;
+    int status = RQO_OK;
+    int64_t n;
+#pragma omp parallel for schedule(static) reduction(max : status)
+    for (n = 0; n < N; n++) {
+        int c[RQO_GROUP];
+        int64_t g;
+        for (g = 0; g < G; g++) {
+            int st = quantize_group(&W[n * K + g * RQO_GROUP], bits, &scales[n * G + g], c);
+            int64_t i;
+            for (i = 0; i < RQO_GROUP; i++) put_code(codes, K, bits, n, g * RQO_GROUP + i, c[i]);
+            if (st > status) status = st;
+        }
+    }
+    /* NONFINITE (5) must win over RANGE (6) */
+    if (status != RQO_OK) {
+        int64_t i, total = N * G;
+        for (i = 0; i < total; i++) if (scales[i] == 0x7E00u) return RQO_ERR_NONFINITE;
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------ products --- */
+
+/* Dequantised weight (n, k) = c * s16, exact in fp64. */
+double rqo_weight(const uint8_t *codes, const uint16_t *scales, int64_t K, int bits,
+                  int64_t n, int64_t k)
+{
+    return (double)rqo_get_code(codes, K, bits, n, k) *
+           rqo_f16_to_f64(scales[n * (K / RQO_GROUP) + k / RQO_GROUP]);
+}
+
+/* One output: y[m, n] and its error budget B[m, n] (either pointer may be
+ * null).  x is fp16 bit patterns, row-major [M, K]. */
+static void one_output(const uint16_t *x, int64_t K, const uint8_t *codes,
+                       const uint16_t *scales, int bits, int64_t m, int64_t n,
+                       double *y, double *bound)
+{
+    double acc = 0.0, b = 0.0;
+    int64_t k;
+    for (k = 0; k < K; k++) {
+        double xv = rqo_f16_to_f64(x[m * K + k]);
+        double wv = rqo_weight(codes, scales, K, bits, n, k);
+        acc += xv * wv;
+        b += fabs(xv) * fabs(wv);
+    }
+    if (y) *y = acc;
+    if (bound) *bound = b;
+}
+
+/* Full product y[M, N] (row-major, fp64) and budget B[M, N] (nullable). */
+void rqo_matmul(const uint16_t *x, int64_t M, int64_t K, const uint8_t *codes,
+                const uint16_t *scales, int64_t N, int bits, double *y, double *bound)
+{
+    int64_t idx;
+#pragma omp parallel for schedule(static)
+    for (idx = 0; idx < M * N; idx++) {
+        int64_t m = idx / N, n = idx % N;
+        one_output(x, K, codes, scales, bits, m, n, &y[idx], bound ? &bound[idx] : 0);
+    }
+}
+
+/* Sampled outputs: for each of the P pairs (ms[p], ns[p]) compute y and B. */
+void rqo_matmul_sampled(const uint16_t *x, int64_t M, int64_t K, const uint8_t *codes,
+                        const uint16_t *scales, int64_t N, int bits, int64_t P,
+                        const int64_t *ms, const int64_t *ns, double *y, double *bound)
+{
+    int64_t p;
+    (void)M; (void)N;
+#pragma omp parallel for schedule(static)
+    for (p = 0; p < P; p++)
+        one_output(x, K, codes, scales, bits, ms[p], ns[p], &y[p], bound ? &bound[p] : 0);
+}
+
+/* Quantize one row-block of W (rows [n0, n0 + rows)) -- lets a caller check
+ * sampled rows of a matrix too large to quantize whole on the host. */
+int rqo_quantize_rows(const float *Wrows, int64_t rows, int64_t K, int bits,
+                      uint8_t *codes, uint16_t *scales)
+{
+    return rqo_quantize_g64(Wrows, rows, K, bits, codes, scales);
+}

@@ -1,0 +1,98 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of the oracle's C source (on the CPU,
+in a temporary directory), builds it, swaps it in for the real oracle, and
+checks that at least one pin in test_oracle_pins.py fails.  The real oracle is
+restored afterwards.
+"""
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "rqo.c")
+
+MUTANTS = {
+    # rounding half away from zero instead of half to even
+    "round_half_away": ("float r = rintf(t);", "float r = roundf(t);"),
+    # codes against the fp32 scale instead of the stored fp16 scale
+    "divide_by_s32": ("volatile float t = w[i] / sf;", "volatile float t = w[i] / s32;"),
+    # even k in the high nibble
+    "nibble_order": ("if (k % 2 == 0) *b = (uint8_t)((*b & 0xF0u) | nib);",
+                     "if (k % 2 == 1) *b = (uint8_t)((*b & 0xF0u) | nib);"),
+    # fp16 conversion truncates instead of rounding to nearest
+    "fp16_truncate": ("if (rem > half || (rem == half && (q & 1u))) q += 1u;", ";"),
+    # fp16 ties away from zero
+    "fp16_ties_away": ("if (rem > half || (rem == half && (q & 1u))) q += 1u;",
+                       "if (rem >= half) q += 1u;"),
+    # amax taken over signed values
+    "amax_signed": ("float a = fabsf(w[i]);", "float a = w[i];"),
+    # wrong group index for the scale in products
+    "scale_index": ("scales[n * (K / RQO_GROUP) + k / RQO_GROUP]",
+                    "scales[n * (K / RQO_GROUP) + (k / RQO_GROUP + 1) % (K / RQO_GROUP)]"),
+    # transposed x index in products
+    "x_transposed": ("double xv = rqo_f16_to_f64(x[m * K + k]);",
+                     "double xv = rqo_f16_to_f64(x[k * (K > 0 ? 1 : 0) + m * 0 + (k % K)]);"),
+    # qmax of int8 taken as 128
+    "qmax_int8": ("return bits == 4 ? 7 : 127;", "return bits == 4 ? 7 : 128;"),
+    # scale from amax / (qmax + 1)
+    "qmax_plus_one": ("volatile float s32 = amax / (float)qmax;",
+                      "volatile float s32 = amax / (float)(qmax + 1);"),
+}
+
+PIN_TESTS = [
+    lambda: pins.test_hand_examples(4),
+    lambda: pins.test_hand_examples(8),
+    pins.test_hand_int4_exact_reconstruction_row,
+    pins.test_fp16_conversion_edges,
+    lambda: pins.test_quantizer_matches_numpy_restatement(4, (37, 192), 0.02),
+    lambda: pins.test_quantizer_matches_numpy_restatement(8, (5, 768), 1.0),
+    lambda: pins.test_quantizer_invariants(8),
+    lambda: pins.test_exact_reconstruction_on_grid(8),
+    lambda: pins.test_products_match_numpy_fp64(4),
+    pins.test_unit_vector_picks_column,
+]
+
+
+def _build_mutant(name, old, new, tmp):
+    src = open(SRC).read()
+    assert old in src, f"mutation site for {name} not found"
+    path_c = os.path.join(tmp, f"{name}.c")
+    with open(path_c, "w") as f:
+        f.write(src.replace(old, new))
+    path_so = os.path.join(tmp, f"{name}.so")
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+                    "-ffp-contract=off", path_c, "-o", path_so, "-lm"], check=True)
+    return path_so
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name):
+    real = oracle._load()
+    old, new = MUTANTS[name]
+    with tempfile.TemporaryDirectory() as tmp:
+        so = _build_mutant(name, old, new, tmp)
+        lib = ctypes.CDLL(so)
+        for fn in ("rqo_f32_to_f16", "rqo_f16_to_f64", "rqo_quantize_g64", "rqo_matmul",
+                   "rqo_matmul_sampled", "rqo_get_code"):
+            getattr(lib, fn).argtypes = getattr(real, fn).argtypes
+            getattr(lib, fn).restype = getattr(real, fn).restype
+        caught = False
+        oracle._lib = lib
+        try:
+            for t in PIN_TESTS:
+                try:
+                    with np.errstate(all="ignore"):
+                        t()
+                except AssertionError:
+                    caught = True
+                    break
+        finally:
+            oracle._lib = real
+    assert caught, f"no pin fails for mutant {name}"
