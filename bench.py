@@ -1,0 +1,497 @@
+#!/usr/bin/env python3
+"""Benchmark: decode weight GB/s (and prefill TFLOP/s) of group-64 quantized
+RWKV-7 projections on B200, through librq's C ABI.
+
+Default workload: the RWKV-7 1.5B-shaped int4 g64 decode layer (D = 2048:
+fused R/K/V 3 x 2048^2, O 2048^2, channel-mix key 2048->8192 and value
+8192->2048), over the model's 24 layers, at every batch M in {1, 4, 8, 16, 32}.
+One step = one decode pass through the 24-layer projection stack at each M
+(5 x 24 x 4 kernel launches), replayed from CUDA graphs.  The weights
+(642 MB) are larger than L2, so every step streams them from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank decodes its
+own batch through its own copy of the stack (independent replicas, no
+collective on the data path: weak scaling); value = bytes all ranks streamed
+/ the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from weight_only_quantized_g64_b200 import build as rq_build  # noqa: E402
+from weight_only_quantized_g64_b200 import rq, synth  # noqa: E402
+
+METRIC = "decode w4g64 GEMV weight GB/s (% of B200 HBM peak); prefill TFLOP/s; 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(
+            d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------ distributed --
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [t.strip() for t in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [s for s, p in zip(sm, power) if p > 200] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------ the stack --
+
+def flush_l2(buf):
+    buf.add_(1)   # write a buffer larger than L2
+
+
+class DecodeStack:
+    """Quantized projection weights of every layer of a workload."""
+
+    def __init__(self, wl, rank):
+        self.wl = wl
+        self.layers = []
+        D = wl.projs[0].N
+        self.D = D
+        for layer in range(wl.layers):
+            q = {}
+            for pi, pj in enumerate(wl.projs):
+                W = synth.weights(pj.N, pj.K, seed=synth.seed_for(wl.index, layer, pi) + 7919 * rank,
+                                  device="cuda")
+                q[pj.name] = (rq.quantize_g64(W, wl.bits), pj)
+                del W
+            self.layers.append(q)
+        torch.cuda.synchronize()
+        self.bytes_per_pass = wl.layers * sum(
+            synth.algorithmic_weight_bytes(p.N, p.K, wl.bits) for p in wl.projs)
+        self.launches_per_pass = wl.layers * 4
+
+    def buffers(self, M):
+        wl = self.wl
+        D = self.D
+        F = wl.projs[4].N
+        xs = {"xD": synth.activations(M, D, seed=100 + M, device="cuda",
+                                      massive_channel=wl.massive_channel),
+              "xF": synth.activations(M, F, seed=200 + M, device="cuda",
+                                      massive_channel=wl.massive_channel)}
+        ys = {n: torch.empty((M, p.N), dtype=torch.float32, device="cuda") for n, p in
+              ((p.name, p) for p in wl.projs)}
+        return xs, ys
+
+    def run_pass(self, xs, ys):
+        bits = self.wl.bits
+        D = self.D
+        for q in self.layers:
+            (wr, _), (wk, _), (wv, _) = q["r"], q["k"], q["v"]
+            rq.rkv_fused(xs["xD"], wr, wk, wv, D, bits, ys=(ys["r"], ys["k"], ys["v"]))
+            (wo, po) = q["o"]
+            rq.gemv_wq(xs["xD"], wo[0], wo[1], po.N, bits, y=ys["o"])
+            (wkey, pkey) = q["ffn_key"]
+            rq.gemv_wq(xs["xD"], wkey[0], wkey[1], pkey.N, bits, y=ys["ffn_key"])
+            (wval, pval) = q["ffn_value"]
+            rq.gemv_wq(xs["xF"], wval[0], wval[1], pval.N, bits, y=ys["ffn_value"])
+
+
+def capture(fn):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()           # warm (sets kernel attributes outside capture)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+# ---------------------------------------------------------- CPU baseline --
+
+def cpu_oracle_rate(wl, budget_s=12.0, layer_rows=16):
+    """The oracle, as it stands, on a bounded sample of the decode workload:
+    `layer_rows` rows of every projection of layer 0 at every M, repeated
+    until `budget_s` of wall time; returns (weight GB/s, cores, sample)."""
+    import oracle
+    cores = os.cpu_count() or 1
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    oracle.build()
+    jobs = []
+    for pi, pj in enumerate(wl.projs):
+        W = synth.weights(layer_rows, pj.K, seed=synth.seed_for(wl.index, 0, pi))
+        c, s, _ = oracle.quantize_g64(W.numpy(), wl.bits)
+        for M in wl.Ms:
+            x = synth.activations(M, pj.K, seed=M, massive_channel=wl.massive_channel).numpy()
+            jobs.append((x, c, s, synth.algorithmic_weight_bytes(layer_rows, pj.K, wl.bits)))
+    done_bytes, t0, reps = 0, time.perf_counter(), 0
+    while True:
+        for x, c, s, b in jobs:
+            oracle.matmul(x, c, s, wl.bits, with_bound=False)
+            done_bytes += b
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    sample = (f"oracle fp64 products of {layer_rows} rows of each of the {len(wl.projs)} "
+              f"projections of one layer at M in {list(wl.Ms)}, {reps} repetitions "
+              f"({dt:.1f} s)")
+    return done_bytes / dt / 1e9, cores, sample
+
+
+def reference_arm(args, wl, rank, world):
+    """`--impl reference`: the oracle timed on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    cores = os.cpu_count() or 1
+    rows = 4
+    jobs = []
+    for pi, pj in enumerate(wl.projs):
+        W = synth.weights(rows, pj.K, seed=synth.seed_for(wl.index, 0, pi))
+        c, s, _ = oracle.quantize_g64(W.numpy(), wl.bits)
+        for M in wl.Ms:
+            x = synth.activations(M, pj.K, seed=M, massive_channel=wl.massive_channel).numpy()
+            jobs.append((x, c, s, synth.algorithmic_weight_bytes(rows, pj.K, wl.bits)))
+    step_bytes = sum(j[3] for j in jobs)
+
+    def step():
+        for x, c, s, _ in jobs:
+            oracle.matmul(x, c, s, wl.bits, with_bound=False)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = step_bytes * args.steps / dt / 1e9
+    sample = (f"each step: oracle fp64 products of {rows} rows of each projection of one "
+              f"layer at M in {list(wl.Ms)}")
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": wl.name, "bits": wl.bits, "M": list(wl.Ms)},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------ prefill, quantizer --
+
+def bench_prefill(hbm_peak, tf_peak, reps=5):
+    wl = synth.WORKLOADS[4]
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")  # 256 MB
+    weights = []
+    for pi, pj in enumerate(wl.projs):
+        W = synth.weights(pj.N, pj.K, seed=synth.seed_for(4, 0, pi), device="cuda")
+        weights.append((rq.quantize_g64(W, 4), pj))
+        del W
+    per_layer = {"d_x_d": 4, "ffn_key": 1, "ffn_value": 1}
+    out = {}
+    s = torch.cuda.current_stream()
+    for M in wl.Ms:
+        tot_flops, tot_ms = 0.0, 0.0
+        shapes = {}
+        for (cw, pj) in weights:
+            x = synth.activations(M, pj.K, seed=M, device="cuda")
+            y = torch.empty((M, pj.N), dtype=torch.float32, device="cuda")
+            rq.gemm_wq(x, cw[0], cw[1], pj.N, 4, y=y)   # warm
+            times = []
+            for _ in range(reps):
+                flush_l2(flush)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(s)
+                rq.gemm_wq(x, cw[0], cw[1], pj.N, 4, y=y)
+                e1.record(s)
+                e1.synchronize()
+                times.append(e0.elapsed_time(e1))
+            ms = statistics.median(times)
+            fl = 2.0 * M * pj.N * pj.K
+            shapes[pj.name] = {"ms": ms, "tflops": fl / ms / 1e9}
+            tot_flops += fl * per_layer[pj.name]
+            tot_ms += ms * per_layer[pj.name]
+        tf = tot_flops / tot_ms / 1e9
+        out[str(M)] = {"tflops_layer": tf, "frac": tf / tf_peak, "shapes": shapes}
+    return out
+
+
+def bench_quantizer(hbm_peak, reps=5):
+    N, K = 16384, 4096
+    W = synth.weights(N, K, seed=5, device="cuda")
+    codes, scales = rq.empty_weights(N, K, 4)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    rq.quantize_g64(W, 4, codes=codes, scales=scales)
+    s = torch.cuda.current_stream()
+    times = []
+    for _ in range(reps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        rq.quantize_g64(W, 4, codes=codes, scales=scales)
+        e1.record(s)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    byts = N * K * 4 + synth.algorithmic_weight_bytes(N, K, 4)
+    return {"shape": [N, K], "bits": 4, "ms": ms, "gbs": byts / ms / 1e6,
+            "frac": byts / ms / 1e6 / hbm_peak}
+
+
+# ------------------------------------------------------------------ main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
+    ap.add_argument("--no-pdl", action="store_true")
+    ap.add_argument("--skip-extras", action="store_true",
+                    help="decode only (no prefill/quantizer/cpu baseline/e2e)")
+    args = ap.parse_args()
+    wl = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        reference_arm(args, wl, rank, world)
+        return
+
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    rq_build.build()
+    rank, world, local = dist_setup(args.gpus)
+    rq.lib()
+    rq.set_pdl(not args.no_pdl)
+    hbm_peak, tf_peak, tf_sust, peak_kind = peaks()
+
+    stack = DecodeStack(wl, rank)
+    graphs, bufs = {}, {}
+    for M in wl.Ms:
+        xs, ys = stack.buffers(M)
+        bufs[M] = (xs, ys)
+        graphs[M] = capture(lambda xs=xs, ys=ys: stack.run_pass(xs, ys))
+
+    s = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        for M in wl.Ms:
+            graphs[M].replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, each = one pass per M -----------------
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(s)
+    for _ in range(args.steps):
+        for M in wl.Ms:
+            graphs[M].replay()
+    t_end.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+
+    # per-M split of the same passes (events between replays, no host sync)
+    n_split = max(20, args.steps // 10)
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(len(wl.Ms) + 1)]
+             for _ in range(n_split)]
+    for st in range(n_split):
+        marks[st][0].record(s)
+        for i, M in enumerate(wl.Ms):
+            graphs[M].replay()
+            marks[st][i + 1].record(s)
+    torch.cuda.synchronize()
+    per_m_ms = {M: sum(marks[st][i].elapsed_time(marks[st][i + 1]) for st in range(n_split))
+                for i, M in enumerate(wl.Ms)}
+
+    bytes_per_step = stack.bytes_per_pass * len(wl.Ms)
+    launches_per_step = stack.launches_per_pass * len(wl.Ms)
+    ms_per_step = elapsed_ms / args.steps
+    value = world * bytes_per_step * args.steps / (elapsed_ms / 1e3) / 1e9
+    per_rank_gbs = bytes_per_step / (ms_per_step / 1e3) / 1e9
+    per_m = {str(M): {"us_per_pass": per_m_ms[M] / n_split * 1e3,
+                      "gbs": stack.bytes_per_pass / (per_m_ms[M] / n_split / 1e3) / 1e9,
+                      "frac": stack.bytes_per_pass / (per_m_ms[M] / n_split / 1e3) / 1e9 / hbm_peak}
+             for M in wl.Ms}
+
+    # ---- e2e: host inputs in, host results out, through the same calls --
+    e2e = None
+    if not args.skip_extras:
+        host_x = {M: {k: v.cpu().pin_memory() for k, v in bufs[M][0].items()} for M in wl.Ms}
+        host_y = {M: {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                      for k, v in bufs[M][1].items()} for M in wl.Ms}
+        h2d = sum(t.numel() * t.element_size() for M in wl.Ms for t in host_x[M].values())
+        d2h = sum(t.numel() * t.element_size() for M in wl.Ms for t in host_y[M].values())
+        e2e_steps = max(10, args.steps // 10)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(e2e_steps):
+            for M in wl.Ms:
+                xs, ys = bufs[M]
+                for k in xs:
+                    xs[k].copy_(host_x[M][k], non_blocking=True)
+                graphs[M].replay()
+                for k in ys:
+                    host_y[M][k].copy_(ys[k], non_blocking=True)
+        e1.record(s)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": world * bytes_per_step * e2e_steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / e2e_steps,
+               "how": "pinned host x -> device, replay of the captured rq_* calls, "
+                      "every output -> pinned host, per step"}
+
+    prefill = quant = cpu = None
+    if not args.skip_extras:
+        prefill = bench_prefill(hbm_peak, tf_peak)
+        quant = bench_quantizer(hbm_peak)
+        if rank == 0 and world == 1:
+            g, cores, sample = cpu_oracle_rate(wl)
+            cpu = {"value": g, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        achieved = per_rank_gbs
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16xint4->f32" if wl.bits == 4 else "f16xint8->f32",
+            "data": "synthetic (seeded N(0,0.02^2) weights quantized on device, N(0,1) fp16 x)",
+            "config": {"workload": wl.name, "bits": wl.bits, "layers": wl.layers,
+                       "M": list(wl.Ms), "bytes_per_pass": stack.bytes_per_pass,
+                       "l2": "weights (%.0f MB per pass) larger than L2; no flush needed"
+                             % (stack.bytes_per_pass / 1e6),
+                       "pdl": not args.no_pdl, "graphs": True, "parallelism": f"replicas{world}"},
+            "hbm_frac": value / world / hbm_peak,
+            "per_M": per_m,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None,
+                         "kernel": "tc_wq_kernel (decode: fused RKV + O + key + value)",
+                         "bytes_per_launch": bytes_per_step / launches_per_step,
+                         "us_per_launch": ms_per_step * 1e3 / launches_per_step,
+                         "peak_kind": peak_kind + " copy bandwidth"},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+            "prefill": prefill,
+            "prefill_peak": {"tflops": tf_peak, "kind": peak_kind + " bf16 (fp16 same nominal rate)"},
+            "quantizer": quant,
+        }
+        print(json.dumps(line), flush=True)
+
+    for g in graphs.values():
+        del g
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * rq.h -- C ABI of librq: weight-only, group-64, symmetric int4/int8
+ * quantized projections on NVIDIA B200 (sm_100a).
+ *
+ * The operation: a projection weight W[N, K] (N output features, K input
+ * features, row-major) is stored group-wise with GROUP = 64 consecutive k of
+ * one row sharing one fp16 scale, symmetric (no zero point), as packed signed
+ * codes plus scales -- the ".qweight + .scale" format of the
+ * "Hakureirm/rwkv7-sglang-w4gptq-1.5b" model card ("Format & loading
+ * (important)"), in its int4 form and the int8 "w8g64" tier of its
+ * "Accuracy warning" section.  Products are taken directly on those codes
+ * ("RWKV-7 Quantization Toolkit", rwkv-quant-nv 1.2.1, "Key Design": no
+ * dequantised weight matrix is materialised), in three kernel families named
+ * by the model card's opening summary: a GEMV for decode, a small-M product
+ * and a tensor-core GEMM for prefill.  The fused R/K/V call follows the same
+ * "Key Design" list (three projections in one kernel launch).
+ *
+ * Layouts (all row-major, all device memory owned by the caller):
+ *   W       fp32 [N, K]
+ *   codes   int4: uint8 [N, K/2]; byte j of row n holds k = 2j in its low
+ *           nibble and k = 2j+1 in its high nibble, 4-bit two's complement,
+ *           values in [-7, 7].  int8: int8 [N, K], values in [-127, 127].
+ *   scales  fp16 bit patterns [N, K/64]; scales[n, g] covers k in [64g, 64g+64).
+ *   x       fp16 [M, K]            y  fp32 [M, N]
+ *   Dequantised weight: w_hat[n, k] = code[n, k] * scales[n, k/64].
+ *   y[m, n] = sum_k x[m, k] * w_hat[n, k], accumulated in fp32; the result is
+ *   within 2e-3 * sum_k |x[m, k]| * |w_hat[n, k]| of the exact value.
+ *
+ * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ * stream).  Argument errors are found before any launch and returned
+ * synchronously; nothing is launched then.  The library allocates no device
+ * memory per call; pointers must stay valid until the stream reaches the
+ * call.  Inputs and outputs must not overlap.  All pointers must be 16-byte
+ * aligned.  A call that fails to launch returns RQ_ERR_CUDA (the CUDA error
+ * string is available from rq_last_cuda_error()).
+ */
+#ifndef RQ_H_
+#define RQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *rq_stream_t;
+
+typedef enum {
+    RQ_OK = 0,
+    RQ_ERR_NULL = 1,       /* a required pointer is NULL */
+    RQ_ERR_BITS = 2,       /* bits is not 4 or 8 */
+    RQ_ERR_SHAPE = 3,      /* K % 64 != 0, N < 1, K < 64, M out of range, or sizes too large */
+    RQ_ERR_ALIGN = 4,      /* a pointer is not 16-byte aligned */
+    RQ_ERR_NONFINITE = 5,  /* (device status) a weight is NaN or +-inf */
+    RQ_ERR_RANGE = 6,      /* (device status) a group scale overflows fp16 */
+    RQ_ERR_TIMEOUT = 7,    /* (device status) a bounded on-chip wait gave up */
+    RQ_ERR_CUDA = 8        /* a CUDA call or kernel launch failed */
+} rq_status;
+
+#define RQ_GROUP 64
+#define RQ_MAX_DECODE_M 32
+
+/* Bytes of packed codes for an N x K matrix: N*K*bits/8. 0 on bad arguments. */
+size_t rq_codes_bytes(int64_t N, int64_t K, int bits);
+
+/* Bytes of fp16 scales for an N x K matrix: N*(K/64)*2. 0 on bad arguments. */
+size_t rq_scales_bytes(int64_t N, int64_t K);
+
+/*
+ * rq_quantize_g64 -- round-to-nearest group-64 symmetric quantization (the
+ * "calibration-free RTN" of the model card's accuracy bullet).
+ *
+ * For every row n and group g, with qmax = 7 (bits 4) or 127 (bits 8):
+ *   amax = max |W[n, k]| over the group          (fp32, exact)
+ *   s32  = amax / qmax                           (IEEE fp32 division)
+ *   s16  = fp16(s32), round to nearest even     -> scales[n, g]
+ *   code = clamp(rint(W[n, k] / float(s16)), -qmax, qmax)
+ *          (IEEE fp32 division by the STORED scale, rint = half to even);
+ *          code = 0 for every k when s16 == 0.
+ * W: fp32 [N, K] device.  codes: rq_codes_bytes(N, K, bits) bytes device.
+ * scales: N*(K/64) fp16 device.  dev_status: optional device int; when given,
+ * the kernel raises it (atomicMax) to RQ_ERR_RANGE if a scale overflows fp16
+ * (that group gets scale +inf, codes 0) and to RQ_ERR_NONFINITE if a weight
+ * is NaN/inf (that group gets scale 0x7E00, codes 0); the caller zeroes it
+ * beforehand.  Bandwidth-bound: reads 4 B and writes 0.53 / 1.03 B per weight.
+ * Requires K % 64 == 0, N >= 1.
+ */
+rq_status rq_quantize_g64(const float *W, int64_t N, int64_t K, int bits,
+                          void *codes, uint16_t *scales, int *dev_status,
+                          rq_stream_t stream);
+
+/*
+ * rq_gemv_wq -- decode product y[M, N] = x[M, K] * w_hat^T for 1 <= M <= 32.
+ * Streams each code and scale byte from HBM once.
+ * x: fp16 [M, K] device.  codes/scales: as produced by rq_quantize_g64.
+ * y: fp32 [M, N] device, fully overwritten.  Requires K % 64 == 0, N >= 1.
+ */
+rq_status rq_gemv_wq(const uint16_t *x, int64_t M, int64_t K, const void *codes,
+                     const uint16_t *scales, int64_t N, int bits, float *y,
+                     rq_stream_t stream);
+
+/*
+ * rq_rkv_fused -- the three receptance/key/value projections of one RWKV-7
+ * time-mix block, sharing one input x, in ONE kernel launch:
+ *   yR = x * w_hat_R^T,  yK = x * w_hat_K^T,  yV = x * w_hat_V^T.
+ * All three weights are N x K with the same bits.  Same rules as rq_gemv_wq
+ * (1 <= M <= 32).
+ */
+rq_status rq_rkv_fused(const uint16_t *x, int64_t M, int64_t K, int64_t N, int bits,
+                       const void *codes_r, const uint16_t *scales_r,
+                       const void *codes_k, const uint16_t *scales_k,
+                       const void *codes_v, const uint16_t *scales_v,
+                       float *y_r, float *y_k, float *y_v, rq_stream_t stream);
+
+/*
+ * rq_gemm_wq -- prefill product y[M, N] = x[M, K] * w_hat^T on the tcgen05
+ * tensor cores (fp16 operands, fp32 accumulation in tensor memory).  Tuned
+ * for M >= 64; accepts any M >= 1.  Same layouts and rules as rq_gemv_wq.
+ */
+rq_status rq_gemm_wq(const uint16_t *x, int64_t M, int64_t K, const void *codes,
+                     const uint16_t *scales, int64_t N, int bits, float *y,
+                     rq_stream_t stream);
+
+/*
+ * rq_set_pdl -- opt in (enable != 0) or out of programmatic dependent launch
+ * for the product kernels launched afterwards by this process.  With it on, a
+ * product kernel may start while the previous kernel of the stream is still
+ * running: it fetches its codes and scales early and waits for the previous
+ * kernel's completion only before it reads x or writes y.  So with it on, the
+ * kernel launched immediately before a product call must not write that
+ * call's codes or scales.  Off by default.  Not thread-safe.
+ */
+rq_status rq_set_pdl(int enable);
+
+/*
+ * rq_set_wait_limit_ns -- time limit of every bounded on-chip wait of the
+ * library's kernels (default 1 s).  A kernel whose wait exceeds it stops its
+ * work, sets the device status word to RQ_ERR_TIMEOUT and exits; its outputs
+ * are then undefined.  0 is rejected with RQ_ERR_RANGE.
+ */
+rq_status rq_set_wait_limit_ns(uint64_t limit_ns);
+
+/*
+ * rq_read_device_status -- copy the library's device status word of the
+ * current device to *out (RQ_OK or RQ_ERR_TIMEOUT), synchronously (it waits
+ * for the device), and reset it to RQ_OK when reset != 0.
+ */
+rq_status rq_read_device_status(int *out, int reset);
+
+/*
+ * rq_selftest_bounded_wait -- launch a one-warp kernel that waits on an
+ * mbarrier nothing ever completes.  Its bounded wait must give up after
+ * limit_ns and set the device status word to RQ_ERR_TIMEOUT; the kernel then
+ * exits normally.  Diagnostic for the timeout path; faults nothing.
+ */
+rq_status rq_selftest_bounded_wait(uint64_t limit_ns, rq_stream_t stream);
+
+/* Static description of a status code. */
+const char *rq_status_string(rq_status s);
+
+/* Message of the last CUDA error a call of this thread returned RQ_ERR_CUDA for. */
+const char *rq_last_cuda_error(void);
+
+/* Library version, e.g. "0.1.0". */
+const char *rq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RQ_H_ */

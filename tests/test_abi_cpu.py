@@ -1,0 +1,102 @@
+"""librq's C ABI on a machine without a GPU: it loads, exports every function
+include/rq.h declares, sizes come out right, and argument errors are returned
+synchronously before any CUDA call (so these tests launch nothing)."""
+import ctypes
+import subprocess
+
+import pytest
+
+from weight_only_quantized_g64_b200 import build as rq_build
+from weight_only_quantized_g64_b200 import rq
+
+
+@pytest.fixture(scope="module")
+def L():
+    rq_build.build()
+    return rq.lib()
+
+
+def test_exports_every_header_function(L):
+    names = rq.header_functions()
+    assert len(names) >= 13
+    out = subprocess.run(["nm", "-D", "--defined-only", rq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, n
+        assert getattr(L, n) is not None
+
+
+def test_sizes(L):
+    assert L.rq_codes_bytes(768, 768, 4) == 768 * 384
+    assert L.rq_codes_bytes(2560, 10240, 8) == 2560 * 10240
+    assert L.rq_scales_bytes(4096, 16384) == 4096 * 256 * 2
+    assert L.rq_codes_bytes(10, 100, 4) == 0       # K % 64 != 0
+    assert L.rq_codes_bytes(10, 128, 3) == 0       # bad bits
+    assert L.rq_codes_bytes(0, 128, 4) == 0
+
+
+FAKE = 1 << 20          # aligned, non-null; never dereferenced because validation fails first
+
+
+@pytest.mark.parametrize("fn", ["rq_gemv_wq", "rq_gemm_wq"])
+def test_product_argument_errors(L, fn):
+    f = getattr(L, fn)
+    assert f(FAKE, 1, 768, FAKE, FAKE, 768, 3, FAKE, None) == rq.ERR_BITS
+    assert f(FAKE, 1, 100, FAKE, FAKE, 768, 4, FAKE, None) == rq.ERR_SHAPE
+    assert f(FAKE, 1, 0, FAKE, FAKE, 768, 4, FAKE, None) == rq.ERR_SHAPE
+    assert f(FAKE, 1, 768, FAKE, FAKE, 0, 4, FAKE, None) == rq.ERR_SHAPE
+    assert f(FAKE, 0, 768, FAKE, FAKE, 768, 4, FAKE, None) == rq.ERR_SHAPE
+    assert f(None, 1, 768, FAKE, FAKE, 768, 4, FAKE, None) == rq.ERR_NULL
+    assert f(FAKE, 1, 768, None, FAKE, 768, 4, FAKE, None) == rq.ERR_NULL
+    assert f(FAKE, 1, 768, FAKE, None, 768, 4, FAKE, None) == rq.ERR_NULL
+    assert f(FAKE, 1, 768, FAKE, FAKE, 768, 4, None, None) == rq.ERR_NULL
+    assert f(FAKE + 2, 1, 768, FAKE, FAKE, 768, 4, FAKE, None) == rq.ERR_ALIGN
+    assert f(FAKE, 1, 768, FAKE + 8, FAKE, 768, 4, FAKE, None) == rq.ERR_ALIGN
+    assert f(FAKE, 1, 768, FAKE, FAKE + 2, 768, 4, FAKE, None) == rq.ERR_ALIGN
+    assert f(FAKE, 1, 768, FAKE, FAKE, 768, 4, FAKE + 4, None) == rq.ERR_ALIGN
+
+
+def test_gemv_m_range(L):
+    assert L.rq_gemv_wq(FAKE, 33, 768, FAKE, FAKE, 768, 4, FAKE, None) == rq.ERR_SHAPE
+    assert L.rq_gemv_wq(FAKE, -1, 768, FAKE, FAKE, 768, 4, FAKE, None) == rq.ERR_SHAPE
+
+
+def test_fused_argument_errors(L):
+    ok = [FAKE] * 9
+    assert L.rq_rkv_fused(FAKE, 1, 768, 768, 5, *ok, None) == rq.ERR_BITS
+    assert L.rq_rkv_fused(FAKE, 40, 768, 768, 4, *ok, None) == rq.ERR_SHAPE
+    for i in range(9):
+        bad = list(ok)
+        bad[i] = None
+        assert L.rq_rkv_fused(FAKE, 1, 768, 768, 4, *bad, None) == rq.ERR_NULL, i
+        bad[i] = FAKE + 4
+        assert L.rq_rkv_fused(FAKE, 1, 768, 768, 4, *bad, None) == rq.ERR_ALIGN, i
+
+
+def test_quantize_argument_errors(L):
+    q = L.rq_quantize_g64
+    assert q(FAKE, 16, 768, 6, FAKE, FAKE, None, None) == rq.ERR_BITS
+    assert q(FAKE, 16, 65, 4, FAKE, FAKE, None, None) == rq.ERR_SHAPE
+    assert q(None, 16, 768, 4, FAKE, FAKE, None, None) == rq.ERR_NULL
+    assert q(FAKE, 16, 768, 4, None, FAKE, None, None) == rq.ERR_NULL
+    assert q(FAKE + 4, 16, 768, 4, FAKE, FAKE, None, None) == rq.ERR_ALIGN
+    assert q(FAKE, 16, 768, 4, FAKE, FAKE, FAKE + 2, None) == rq.ERR_ALIGN
+
+
+def test_control_calls(L):
+    assert L.rq_set_wait_limit_ns(0) == rq.ERR_RANGE
+    assert L.rq_set_wait_limit_ns(10**9) == rq.OK
+    assert L.rq_set_pdl(0) == rq.OK
+    assert L.rq_selftest_bounded_wait(0, None) == rq.ERR_RANGE
+    assert L.rq_read_device_status(None, 0) == rq.ERR_NULL
+    for s in range(9):
+        assert L.rq_status_string(s)
+    assert L.rq_version() == b"0.1.0"
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(rq, "_lib", None)
+    monkeypatch.setattr(rq, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        rq.lib()

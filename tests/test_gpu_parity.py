@@ -1,0 +1,303 @@
+"""GPU parity: librq's sm_100a kernels against the CPU oracle, through the C ABI.
+
+Quantizer: codes and scales bit-exact (and the device status).  Products:
+|y_gpu - y_ref| <= 2e-3 * sum_k |x||w_hat| per output, the tolerance the
+format's accuracy claim is held to here (fp16 rounding of code*scale, at most
+2^-11 relative, plus fp32 accumulation).  Product tests feed the ORACLE's
+codes to the GPU so they do not depend on the GPU quantizer.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from weight_only_quantized_g64_b200 import build as rq_build
+from weight_only_quantized_g64_b200 import rq, synth
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    rq_build.build()
+    rq.lib()
+    rq.set_pdl(False)
+    yield
+    assert rq.read_device_status(reset=True) == rq.OK
+
+
+def to_host(t):
+    return t.detach().cpu().numpy()
+
+
+def oracle_weights(W_dev, bits):
+    codes, scales, st = oracle.quantize_g64(to_host(W_dev), bits)
+    assert st == 0
+    return codes, scales
+
+
+def upload(codes, scales):
+    return (torch.from_numpy(codes).cuda(), torch.from_numpy(scales.view(np.int16)).cuda())
+
+
+def check_close(y_gpu, y_ref, bound, what):
+    diff = np.abs(y_gpu.astype(np.float64) - y_ref)
+    lim = TOL * bound
+    bad = diff > lim
+    assert not bad.any(), (f"{what}: {int(bad.sum())} outputs out of tolerance; worst "
+                           f"diff {diff.max():.3e} vs limit {lim[np.unravel_index(diff.argmax(), diff.shape)]:.3e}")
+
+
+# ------------------------------------------------------------- quantizer ---
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("N,K", [(1, 64), (3, 128), (300, 640), (768, 768), (129, 4096)])
+def test_quantizer_bit_exact(bits, N, K):
+    W = synth.weights(N, K, seed=synth.seed_for(0, N, K % 7), device="cuda")
+    codes, scales = rq.quantize_g64(W, bits)
+    c_ref, s_ref, st = oracle.quantize_g64(to_host(W), bits)
+    assert st == 0
+    torch.cuda.synchronize()
+    assert np.array_equal(to_host(scales).view(np.uint16), s_ref)
+    assert np.array_equal(to_host(codes), c_ref)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_quantizer_special_values(bits):
+    N, K = 8, 256
+    W = synth.weights(N, K, seed=77, device="cpu")
+    W[0, :64] = 0.0                                            # all-zero group
+    W[1, :64] = 0.125 * (torch.arange(64) % 15 - 7).float()    # on grid, with ties below
+    W[1, 1], W[1, 2], W[1, 3] = 0.3125, 0.4375, -0.3125
+    W[2, 64:128] = 1e-9                                        # scale underflows to fp16 subnormal/0
+    W[3, 5] = 1e6                                              # fp16 scale overflow -> RANGE
+    W[4, 70] = float("nan")                                    # NONFINITE
+    W[5, 200] = -float("inf")                                  # NONFINITE
+    W[6, 128:192] = torch.linspace(-3e-5, 3e-5, 64)            # subnormal fp16 scales
+    Wd = W.cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    codes, scales = rq.quantize_g64(Wd, bits, dev_status=status)
+    c_ref, s_ref, st = oracle.quantize_g64(W.numpy(), bits)
+    torch.cuda.synchronize()
+    assert int(status.item()) == st == oracle.STATUS_NONFINITE
+    assert np.array_equal(to_host(scales).view(np.uint16), s_ref)
+    assert np.array_equal(to_host(codes), c_ref)
+    # RANGE alone
+    W2 = synth.weights(4, 128, seed=78)
+    W2[2, 100] = 3e6
+    status.zero_()
+    codes2, scales2 = rq.quantize_g64(W2.cuda(), bits, dev_status=status)
+    c2, s2, st2 = oracle.quantize_g64(W2.numpy(), bits)
+    torch.cuda.synchronize()
+    assert int(status.item()) == st2 == oracle.STATUS_RANGE
+    assert np.array_equal(to_host(scales2).view(np.uint16), s2)
+    assert np.array_equal(to_host(codes2), c2)
+
+
+# -------------------------------------------------------------- products ---
+
+def product_case(N, K, bits, M, seed, massive=None):
+    W = synth.weights(N, K, seed=seed, device="cuda")
+    x = synth.activations(M, K, seed=seed, device="cuda", massive_channel=massive)
+    codes, scales = oracle_weights(W, bits)
+    return x, codes, scales
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 16, 17, 31, 32])
+@pytest.mark.parametrize("N,K", [(300, 640), (1, 64), (129, 128), (256, 2048)])
+def test_gemv_parity(bits, M, N, K):
+    x, codes, scales = product_case(N, K, bits, M, seed=1000 + M + N + K)
+    cd, sd = upload(codes, scales)
+    y = rq.gemv_wq(x, cd, sd, N, bits)
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.matmul(to_host(x), codes, scales, bits)
+    check_close(to_host(y), y_ref, bound, f"gemv bits={bits} M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M", [1, 8, 32])
+def test_rkv_fused_parity(bits, M):
+    N, K = 200, 512
+    cases = [product_case(N, K, bits, M, seed=2000 + i) for i in range(3)]
+    x = cases[0][0]
+    ws = [upload(c[1], c[2]) for c in cases]
+    ys = rq.rkv_fused(x, ws[0], ws[1], ws[2], N, bits)
+    torch.cuda.synchronize()
+    for i in range(3):
+        y_ref, bound = oracle.matmul(to_host(x), cases[i][1], cases[i][2], bits)
+        check_close(to_host(ys[i]), y_ref, bound, f"rkv[{i}] bits={bits} M={M}")
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M", [1, 64, 100, 256, 300])
+def test_gemm_parity(bits, M):
+    N, K = 384, 512
+    x, codes, scales = product_case(N, K, bits, M, seed=3000 + M)
+    cd, sd = upload(codes, scales)
+    y = rq.gemm_wq(x, cd, sd, N, bits)
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.matmul(to_host(x), codes, scales, bits)
+    check_close(to_host(y), y_ref, bound, f"gemm bits={bits} M={M}")
+
+
+def test_unit_vectors_pick_columns():
+    """x = e_j returns column j of the dequantised weight (exact up to fp32)."""
+    N, K, bits = 130, 192, 4
+    W = synth.weights(N, K, seed=9, device="cuda")
+    codes, scales = oracle_weights(W, bits)
+    cd, sd = upload(codes, scales)
+    js = [0, 1, 63, 64, 127, 191]
+    x = torch.zeros((len(js), K), dtype=torch.float16, device="cuda")
+    for i, j in enumerate(js):
+        x[i, j] = 1.0
+    y = to_host(rq.gemv_wq(x, cd, sd, N, bits))
+    s = scales.view(np.float16).astype(np.float64)
+    for i, j in enumerate(js):
+        col = np.array([oracle.get_code(codes, K, bits, n, j) for n in range(N)]) * s[:, j // 64]
+        # fp16(code*s) is what the tensor core sees: within 2^-11 relative of code*s
+        assert np.all(np.abs(y[i] - col) <= np.abs(col) * 2.0 ** -11 + 1e-12)
+
+
+def test_quantize_then_product_chain():
+    """GPU quantizer feeding GPU products on the same stream."""
+    N, K, bits, M = 512, 1024, 4, 5
+    W = synth.weights(N, K, seed=11, device="cuda")
+    x = synth.activations(M, K, seed=11, device="cuda")
+    codes, scales = rq.quantize_g64(W, bits)
+    y = rq.gemv_wq(x, codes, scales, N, bits)
+    torch.cuda.synchronize()
+    c_ref, s_ref, _ = oracle.quantize_g64(to_host(W), bits)
+    y_ref, bound = oracle.matmul(to_host(x), c_ref, s_ref, bits)
+    check_close(to_host(y), y_ref, bound, "quantize->gemv")
+
+
+# ------------------------------------------ configuration shapes, sampled ---
+
+def sampled_check(y, x, codes_dev, scales_dev, N, K, bits, n_samples=512, seed=0, rows=None):
+    """Compare sampled outputs; rows of the weight are pulled to the host only
+    for the sampled n."""
+    M = x.shape[0]
+    rng = np.random.default_rng(seed)
+    ns = rng.integers(0, N, size=n_samples)
+    ns[:4] = [0, N - 1, N // 2, 127 % N]
+    ms = rng.integers(0, M, size=n_samples)
+    ms[:2] = [0, M - 1]
+    uniq = np.unique(ns)
+    sub_c = to_host(codes_dev[torch.from_numpy(uniq).cuda()])
+    sub_s = to_host(scales_dev[torch.from_numpy(uniq).cuda()]).view(np.uint16)
+    remap = {int(n): i for i, n in enumerate(uniq)}
+    ns_local = np.array([remap[int(n)] for n in ns])
+    y_ref, bound = oracle.matmul_sampled(to_host(x), sub_c, sub_s, bits, ms, ns_local)
+    yg = to_host(y)[ms, ns]
+    check_close(yg, y_ref, bound, f"sampled N={N} K={K} bits={bits} M={M}")
+
+
+def quantize_checked(W, bits, sample_rows=64, seed=0):
+    """GPU quantizer, with a bit-exact oracle check on sampled rows."""
+    codes, scales = rq.quantize_g64(W, bits)
+    N = W.shape[0]
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, N - 1], rng.integers(0, N, size=sample_rows)]))
+    Wr = to_host(W[torch.from_numpy(rows).cuda()])
+    c_ref, s_ref, st = oracle.quantize_g64(Wr, bits)
+    assert st == 0
+    idx = torch.from_numpy(rows).cuda()
+    assert np.array_equal(to_host(codes[idx]), c_ref)
+    assert np.array_equal(to_host(scales[idx]).view(np.uint16), s_ref)
+    return codes, scales
+
+
+@pytest.mark.parametrize("wl", [1, 2, 3, 5])
+def test_decode_workload_shapes(wl):
+    w = synth.WORKLOADS[wl]
+    for pi, pj in enumerate(w.projs):
+        W = synth.weights(pj.N, pj.K, seed=synth.seed_for(wl, 0, pi), device="cuda")
+        codes, scales = quantize_checked(W, w.bits, seed=pi)
+        del W
+        for M in w.Ms:
+            x = synth.activations(M, pj.K, seed=synth.seed_for(wl, 0, pi) + M, device="cuda",
+                                  massive_channel=w.massive_channel)
+            y = rq.gemv_wq(x, codes, scales, pj.N, w.bits)
+            torch.cuda.synchronize()
+            sampled_check(y, x, codes, scales, pj.N, pj.K, w.bits, seed=M)
+
+
+def test_decode_workload_rkv_fused():
+    for wl in (2, 3, 5):
+        w = synth.WORKLOADS[wl]
+        D = w.projs[0].N
+        ws = []
+        for pi in range(3):
+            W = synth.weights(D, D, seed=synth.seed_for(wl, 1, pi), device="cuda")
+            ws.append(rq.quantize_g64(W, w.bits))
+            del W
+        for M in (w.Ms[0], w.Ms[-1]):
+            x = synth.activations(M, D, seed=M, device="cuda", massive_channel=w.massive_channel)
+            ys = rq.rkv_fused(x, ws[0], ws[1], ws[2], D, w.bits)
+            torch.cuda.synchronize()
+            for i in range(3):
+                sampled_check(ys[i], x, ws[i][0], ws[i][1], D, D, w.bits, n_samples=256, seed=i)
+
+
+def test_prefill_workload_shapes():
+    w = synth.WORKLOADS[4]
+    for pi, pj in enumerate(w.projs):
+        W = synth.weights(pj.N, pj.K, seed=synth.seed_for(4, 0, pi), device="cuda")
+        codes, scales = quantize_checked(W, w.bits, seed=pi)
+        del W
+        for M in w.Ms:
+            x = synth.activations(M, pj.K, seed=M + pi, device="cuda")
+            y = rq.gemm_wq(x, codes, scales, pj.N, w.bits)
+            torch.cuda.synchronize()
+            sampled_check(y, x, codes, scales, pj.N, pj.K, w.bits, n_samples=384, seed=M)
+
+
+# ------------------------------------------------------------ robustness ---
+
+def test_bounded_wait_times_out_cleanly():
+    """A wait nothing completes gives up, reports RQ_ERR_TIMEOUT, and the
+    context stays usable."""
+    assert rq.read_device_status(reset=True) == rq.OK
+    rq.selftest_bounded_wait(50_000_000)        # 50 ms
+    torch.cuda.synchronize()
+    assert rq.read_device_status(reset=True) == rq.ERR_TIMEOUT
+    # the context still works
+    x, codes, scales = product_case(128, 128, 4, 1, seed=5)
+    cd, sd = upload(codes, scales)
+    y = rq.gemv_wq(x, cd, sd, 128, 4)
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.matmul(to_host(x), codes, scales, 4)
+    check_close(to_host(y), y_ref, bound, "after timeout")
+    assert rq.read_device_status() == rq.OK
+
+
+def test_pdl_chain_matches():
+    """With programmatic dependent launch on, a chain of dependent products
+    (each reading the previous output as its input) still matches."""
+    N = K = 512
+    bits = 4
+    M = 4
+    W = [synth.weights(N, K, seed=40 + i, device="cuda") for i in range(3)]
+    qs = [rq.quantize_g64(w, bits) for w in W]
+    torch.cuda.synchronize()
+    x0 = synth.activations(M, K, seed=40, device="cuda")
+    rq.set_pdl(True)
+    try:
+        x = x0
+        outs = []
+        for c, s in qs:
+            y = rq.gemv_wq(x, c, s, N, bits)
+            x = (y * 0.05).to(torch.float16)   # torch op between: still ordered
+            outs.append(y)
+        torch.cuda.synchronize()
+    finally:
+        rq.set_pdl(False)
+    xh = to_host(x0)
+    for i, (c, s) in enumerate(qs):
+        ch, sh = to_host(c), to_host(s).view(np.uint16)
+        y_ref, bound = oracle.matmul(xh, ch, sh, bits)
+        check_close(to_host(outs[i]), y_ref, bound, f"pdl chain {i}")
+        xh = (to_host(outs[i]) * 0.05).astype(np.float16)

@@ -1,0 +1,218 @@
+// rq_api.cu -- the C ABI of include/rq.h: argument validation, dispatch to
+// the kernels, TMA descriptor creation, status strings.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "rq_internal.h"
+
+namespace rq {
+
+// Library-wide device status word (one per device that loads the module):
+// bounded waits raise RQ_ERR_TIMEOUT here.
+__device__ int g_device_status = 0;
+
+static constexpr int kMaxDevices = 64;
+static int* g_status_ptr[kMaxDevices] = {};
+static std::mutex g_mu;
+static bool g_pdl = false;
+static uint64_t g_wait_limit_ns = 1000000000ull;  // 1 s
+
+int* device_status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (g_status_ptr[dev] == nullptr) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_status_ptr[dev] == nullptr) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+            g_status_ptr[dev] = static_cast<int*>(p);
+        }
+    }
+    return g_status_ptr[dev];
+}
+
+uint64_t wait_limit_ns() { return g_wait_limit_ns; }
+bool pdl_enabled() { return g_pdl; }
+
+// ------------------------------------------------------------ tensor maps --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                  uint64_t inner_elems, uint64_t rows, uint64_t row_stride_bytes,
+                  uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {inner_elems, rows};
+    cuuint64_t strides[1] = {row_stride_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace rq
+
+using namespace rq;
+
+static thread_local std::string t_last_cuda_error;
+
+static rq_status cuda_fail(cudaError_t e) {
+    t_last_cuda_error = cudaGetErrorString(e);
+    return RQ_ERR_CUDA;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static rq_status check_weight_shape(int64_t N, int64_t K, int bits) {
+    if (bits != 4 && bits != 8) return RQ_ERR_BITS;
+    if (N < 1 || K < kGroup || K % kGroup != 0) return RQ_ERR_SHAPE;
+    if (N > (int64_t{1} << 31) - 1 || K > (int64_t{1} << 30)) return RQ_ERR_SHAPE;
+    return RQ_OK;
+}
+
+static rq_status check_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
+                               int64_t max_m) {
+    rq_status st = check_weight_shape(N, K, bits);
+    if (st != RQ_OK) return st;
+    if (M < 1 || M > max_m) return RQ_ERR_SHAPE;
+    if (x == nullptr) return RQ_ERR_NULL;
+    if (!aligned16(x)) return RQ_ERR_ALIGN;
+    return RQ_OK;
+}
+
+static rq_status check_operand(const void* codes, const uint16_t* scales, const float* y) {
+    if (codes == nullptr || scales == nullptr || y == nullptr) return RQ_ERR_NULL;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(y)) return RQ_ERR_ALIGN;
+    return RQ_OK;
+}
+
+extern "C" {
+
+size_t rq_codes_bytes(int64_t N, int64_t K, int bits) {
+    if (check_weight_shape(N, K, bits) != RQ_OK) return 0;
+    return static_cast<size_t>(N) * static_cast<size_t>(K) * static_cast<size_t>(bits) / 8;
+}
+
+size_t rq_scales_bytes(int64_t N, int64_t K) {
+    if (check_weight_shape(N, K, 4) != RQ_OK) return 0;
+    return static_cast<size_t>(N) * static_cast<size_t>(K / kGroup) * 2;
+}
+
+rq_status rq_quantize_g64(const float* W, int64_t N, int64_t K, int bits, void* codes,
+                          uint16_t* scales, int* dev_status, rq_stream_t stream) {
+    rq_status st = check_weight_shape(N, K, bits);
+    if (st != RQ_OK) return st;
+    if (W == nullptr || codes == nullptr || scales == nullptr) return RQ_ERR_NULL;
+    if (!aligned16(W) || !aligned16(codes) || !aligned16(scales)) return RQ_ERR_ALIGN;
+    if (dev_status != nullptr && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return RQ_ERR_ALIGN;
+    cudaError_t e = launch_quantize(W, N * (K / kGroup), bits, codes, scales, dev_status,
+                                    reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+rq_status rq_gemv_wq(const uint16_t* x, int64_t M, int64_t K, const void* codes,
+                     const uint16_t* scales, int64_t N, int bits, float* y, rq_stream_t stream) {
+    rq_status st = check_product(x, M, K, N, bits, RQ_MAX_DECODE_M);
+    if (st != RQ_OK) return st;
+    if ((st = check_operand(codes, scales, y)) != RQ_OK) return st;
+    WOperand w = {codes, scales, y};
+    cudaError_t e = launch_tc_product(x, M, K, N, bits, &w, 1, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+rq_status rq_rkv_fused(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
+                       const void* codes_r, const uint16_t* scales_r, const void* codes_k,
+                       const uint16_t* scales_k, const void* codes_v, const uint16_t* scales_v,
+                       float* y_r, float* y_k, float* y_v, rq_stream_t stream) {
+    rq_status st = check_product(x, M, K, N, bits, RQ_MAX_DECODE_M);
+    if (st != RQ_OK) return st;
+    if ((st = check_operand(codes_r, scales_r, y_r)) != RQ_OK) return st;
+    if ((st = check_operand(codes_k, scales_k, y_k)) != RQ_OK) return st;
+    if ((st = check_operand(codes_v, scales_v, y_v)) != RQ_OK) return st;
+    WOperand w[3] = {{codes_r, scales_r, y_r}, {codes_k, scales_k, y_k}, {codes_v, scales_v, y_v}};
+    cudaError_t e = launch_tc_product(x, M, K, N, bits, w, 3, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+rq_status rq_gemm_wq(const uint16_t* x, int64_t M, int64_t K, const void* codes,
+                     const uint16_t* scales, int64_t N, int bits, float* y, rq_stream_t stream) {
+    rq_status st = check_product(x, M, K, N, bits, (int64_t{1} << 31) - 1);
+    if (st != RQ_OK) return st;
+    if ((st = check_operand(codes, scales, y)) != RQ_OK) return st;
+    if (M * K > (int64_t{1} << 40)) return RQ_ERR_SHAPE;
+    WOperand w = {codes, scales, y};
+    cudaError_t e = launch_tc_product(x, M, K, N, bits, &w, 1, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+rq_status rq_set_pdl(int enable) {
+    g_pdl = enable != 0;
+    return RQ_OK;
+}
+
+rq_status rq_set_wait_limit_ns(uint64_t limit_ns) {
+    if (limit_ns == 0) return RQ_ERR_RANGE;
+    g_wait_limit_ns = limit_ns;
+    return RQ_OK;
+}
+
+rq_status rq_read_device_status(int* out, int reset) {
+    if (out == nullptr) return RQ_ERR_NULL;
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_device_status, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (reset) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return RQ_OK;
+}
+
+rq_status rq_selftest_bounded_wait(uint64_t limit_ns, rq_stream_t stream) {
+    if (limit_ns == 0) return RQ_ERR_RANGE;
+    cudaError_t e = launch_wait_selftest(limit_ns, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+const char* rq_status_string(rq_status s) {
+    switch (s) {
+        case RQ_OK: return "ok";
+        case RQ_ERR_NULL: return "a required pointer is NULL";
+        case RQ_ERR_BITS: return "bits must be 4 or 8";
+        case RQ_ERR_SHAPE: return "bad shape (K % 64 != 0, N < 1, M out of range, or too large)";
+        case RQ_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case RQ_ERR_NONFINITE: return "a weight is NaN or infinite";
+        case RQ_ERR_RANGE: return "a value is out of range (fp16 scale overflow or bad limit)";
+        case RQ_ERR_TIMEOUT: return "a bounded on-chip wait timed out";
+        case RQ_ERR_CUDA: return "a CUDA call failed";
+    }
+    return "unknown status";
+}
+
+const char* rq_last_cuda_error(void) { return t_last_cuda_error.c_str(); }
+
+const char* rq_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,49 @@
+// rq_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/rq.h"
+
+namespace rq {
+
+// Group size of the format (64 consecutive k of one row share a scale).
+constexpr int kGroup = 64;
+
+// Quantizer: flat over all N*K/64 groups (groups are contiguous in W, codes
+// and scales when all three are row-major).
+cudaError_t launch_quantize(const float* W, int64_t n_groups, int bits, void* codes,
+                            uint16_t* scales, int* dev_status, cudaStream_t s);
+
+// One weight operand of a product: its TMA descriptor (codes), scales, output.
+struct WOperand {
+    const void* codes;
+    const uint16_t* scales;
+    float* y;
+};
+
+// Tensor-core product (dequantise into TMEM, tcgen05.mma with fp32
+// accumulation).  nmat = 1 (single projection) or 3 (fused R/K/V).
+cudaError_t launch_tc_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
+                              const WOperand* w, int nmat, cudaStream_t s);
+
+// Bounded-wait self test: a kernel waits on an mbarrier nothing completes.
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s);
+
+// Tensor map creation (driver entry point fetched once through the runtime).
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                  uint64_t inner_elems, uint64_t rows, uint64_t row_stride_bytes,
+                  uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz);
+
+// Whether programmatic dependent launch is requested for kernel launches.
+bool pdl_enabled();
+
+// Device address of the library status word on the current device.
+int* device_status_ptr();
+
+// Time limit of every bounded on-chip wait, in nanoseconds.
+uint64_t wait_limit_ns();
+
+}  // namespace rq

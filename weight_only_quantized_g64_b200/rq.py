@@ -1,0 +1,172 @@
+"""Thin Python binding of librq (include/rq.h): argument marshalling only.
+
+Every step of every call runs in librq's sm_100a kernels; torch is used for
+device memory, streams and output allocation.  There is no fallback: if
+librq.so is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librq.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "rq.h")
+
+GROUP = 64
+MAX_DECODE_M = 32
+
+STATUS = {0: "RQ_OK", 1: "RQ_ERR_NULL", 2: "RQ_ERR_BITS", 3: "RQ_ERR_SHAPE", 4: "RQ_ERR_ALIGN",
+          5: "RQ_ERR_NONFINITE", 6: "RQ_ERR_RANGE", 7: "RQ_ERR_TIMEOUT", 8: "RQ_ERR_CUDA"}
+OK, ERR_NULL, ERR_BITS, ERR_SHAPE, ERR_ALIGN, ERR_NONFINITE, ERR_RANGE, ERR_TIMEOUT, ERR_CUDA = range(9)
+
+_lib = None
+
+
+class RQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = f"{what}: {STATUS.get(status, status)}"
+        if status == ERR_CUDA and _lib is not None:
+            msg += f" ({_lib.rq_last_cuda_error().decode()})"
+        super().__init__(msg)
+
+
+def lib():
+    """Load librq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"librq.so not built at {LIB_PATH}: run "
+                           "`python -m weight_only_quantized_g64_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    i64, vp, i32, u64 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64
+    L.rq_codes_bytes.argtypes = [i64, i64, i32]
+    L.rq_codes_bytes.restype = ctypes.c_size_t
+    L.rq_scales_bytes.argtypes = [i64, i64]
+    L.rq_scales_bytes.restype = ctypes.c_size_t
+    L.rq_quantize_g64.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
+    L.rq_quantize_g64.restype = i32
+    L.rq_gemv_wq.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, vp]
+    L.rq_gemv_wq.restype = i32
+    L.rq_gemm_wq.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, vp]
+    L.rq_gemm_wq.restype = i32
+    L.rq_rkv_fused.argtypes = [vp, i64, i64, i64, i32] + [vp] * 9 + [vp]
+    L.rq_rkv_fused.restype = i32
+    L.rq_set_pdl.argtypes = [i32]
+    L.rq_set_pdl.restype = i32
+    L.rq_set_wait_limit_ns.argtypes = [u64]
+    L.rq_set_wait_limit_ns.restype = i32
+    L.rq_read_device_status.argtypes = [ctypes.POINTER(ctypes.c_int), i32]
+    L.rq_read_device_status.restype = i32
+    L.rq_selftest_bounded_wait.argtypes = [u64, vp]
+    L.rq_selftest_bounded_wait.restype = i32
+    L.rq_status_string.argtypes = [i32]
+    L.rq_status_string.restype = ctypes.c_char_p
+    L.rq_last_cuda_error.argtypes = []
+    L.rq_last_cuda_error.restype = ctypes.c_char_p
+    L.rq_version.argtypes = []
+    L.rq_version.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def header_functions() -> list[str]:
+    """Names of every function include/rq.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_]+\s*\*?\s*(rq_[a-z0-9_]+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _p(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check(st: int, what: str):
+    if st != OK:
+        raise RQError(st, what)
+
+
+def codes_bytes(N: int, K: int, bits: int) -> int:
+    return int(lib().rq_codes_bytes(N, K, bits))
+
+
+def scales_bytes(N: int, K: int) -> int:
+    return int(lib().rq_scales_bytes(N, K))
+
+
+def empty_weights(N: int, K: int, bits: int, device="cuda"):
+    """Allocate (codes uint8 [N, K*bits/8], scales int16 [N, K/64]) for N x K."""
+    codes = torch.empty((N, K * bits // 8), dtype=torch.uint8, device=device)
+    scales = torch.empty((N, K // GROUP), dtype=torch.int16, device=device)
+    return codes, scales
+
+
+def quantize_g64(W: torch.Tensor, bits: int, codes=None, scales=None, dev_status=None,
+                 stream=None):
+    """RTN group-64 quantization of fp32 W[N, K] on the GPU -> (codes, scales)."""
+    N, K = W.shape
+    if codes is None:
+        codes, scales = empty_weights(N, K, bits, W.device)
+    _check(lib().rq_quantize_g64(_p(W), N, K, bits, _p(codes), _p(scales), _p(dev_status),
+                                 _stream(stream)), "rq_quantize_g64")
+    return codes, scales
+
+
+def gemv_wq(x: torch.Tensor, codes, scales, N: int, bits: int, y=None, stream=None):
+    """Decode product y[M, N] = x[M, K] @ w_hat^T, 1 <= M <= 32."""
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _check(lib().rq_gemv_wq(_p(x), M, K, _p(codes), _p(scales), N, bits, _p(y), _stream(stream)),
+           "rq_gemv_wq")
+    return y
+
+
+def gemm_wq(x: torch.Tensor, codes, scales, N: int, bits: int, y=None, stream=None):
+    """Prefill product y[M, N] = x[M, K] @ w_hat^T on the tcgen05 tensor cores."""
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _check(lib().rq_gemm_wq(_p(x), M, K, _p(codes), _p(scales), N, bits, _p(y), _stream(stream)),
+           "rq_gemm_wq")
+    return y
+
+
+def rkv_fused(x: torch.Tensor, wr, wk, wv, N: int, bits: int, ys=None, stream=None):
+    """Three projections of one shared x in one launch; w* = (codes, scales)."""
+    M, K = x.shape
+    if ys is None:
+        ys = tuple(torch.empty((M, N), dtype=torch.float32, device=x.device) for _ in range(3))
+    _check(lib().rq_rkv_fused(_p(x), M, K, N, bits, _p(wr[0]), _p(wr[1]), _p(wk[0]), _p(wk[1]),
+                              _p(wv[0]), _p(wv[1]), _p(ys[0]), _p(ys[1]), _p(ys[2]),
+                              _stream(stream)), "rq_rkv_fused")
+    return ys
+
+
+def set_pdl(enable: bool):
+    _check(lib().rq_set_pdl(1 if enable else 0), "rq_set_pdl")
+
+
+def set_wait_limit_ns(ns: int):
+    _check(lib().rq_set_wait_limit_ns(ns), "rq_set_wait_limit_ns")
+
+
+def read_device_status(reset: bool = False) -> int:
+    out = ctypes.c_int(-1)
+    _check(lib().rq_read_device_status(ctypes.byref(out), 1 if reset else 0),
+           "rq_read_device_status")
+    return out.value
+
+
+def selftest_bounded_wait(limit_ns: int, stream=None):
+    _check(lib().rq_selftest_bounded_wait(limit_ns, _stream(stream)), "rq_selftest_bounded_wait")
