@@ -80,11 +80,11 @@ size_t rq_scales_bytes(int64_t N, int64_t K);
  *          (IEEE fp32 division by the STORED scale, rint = half to even);
  *          code = 0 for every k when s16 == 0.
  * W: fp32 [N, K] device.  codes: rq_codes_bytes(N, K, bits) bytes device.
- * scales: N*(K/64) fp16 device.  dev_status: optional device int; when given,
- * the kernel raises it (atomicMax) to RQ_ERR_RANGE if a scale overflows fp16
- * (that group gets scale +inf, codes 0) and to RQ_ERR_NONFINITE if a weight
- * is NaN/inf (that group gets scale 0x7E00, codes 0); the caller zeroes it
- * beforehand.  Bandwidth-bound: reads 4 B and writes 0.53 / 1.03 B per weight.
+ * scales: N*(K/64) fp16 device.  dev_status: optional device int that the
+ * caller zeroes beforehand; the kernel sets it to RQ_ERR_NONFINITE if any
+ * weight is NaN/inf (that group gets scale 0x7E00, codes 0), otherwise to
+ * RQ_ERR_RANGE if any group scale overflows fp16 (that group gets scale +inf,
+ * codes 0); it stays RQ_OK otherwise.  Bandwidth-bound: reads 4 B and writes 0.53 / 1.03 B per weight.
  * Requires K % 64 == 0, N >= 1.
  */
 rq_status rq_quantize_g64(const float *W, int64_t N, int64_t K, int bits,

@@ -71,7 +71,11 @@ __global__ void __launch_bounds__(256) quantize_g64_kernel(const float4* __restr
         }
         if (lane16 == 0) {
             scales[gid] = s_bits;
-            if (status != 0 && dev_status != nullptr) atomicMax(dev_status, status);
+            // NONFINITE overrides everything; RANGE only replaces OK.
+            if (dev_status != nullptr) {
+                if (status == 5) atomicExch(dev_status, 5);
+                else if (status == 6) atomicCAS(dev_status, 0, 6);
+            }
         }
     }
 }
