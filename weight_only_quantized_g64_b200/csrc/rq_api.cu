@@ -138,7 +138,7 @@ rq_status rq_gemv_wq(const uint16_t* x, int64_t M, int64_t K, const void* codes,
     if (st != RQ_OK) return st;
     if ((st = check_operand(codes, scales, y)) != RQ_OK) return st;
     WOperand w = {codes, scales, y};
-    cudaError_t e = launch_tc_product(x, M, K, N, bits, &w, 1, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_gemv_product(x, M, K, N, bits, &w, 1, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? RQ_OK : cuda_fail(e);
 }
 
@@ -152,7 +152,7 @@ rq_status rq_rkv_fused(const uint16_t* x, int64_t M, int64_t K, int64_t N, int b
     if ((st = check_operand(codes_k, scales_k, y_k)) != RQ_OK) return st;
     if ((st = check_operand(codes_v, scales_v, y_v)) != RQ_OK) return st;
     WOperand w[3] = {{codes_r, scales_r, y_r}, {codes_k, scales_k, y_k}, {codes_v, scales_v, y_v}};
-    cudaError_t e = launch_tc_product(x, M, K, N, bits, w, 3, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_gemv_product(x, M, K, N, bits, w, 3, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? RQ_OK : cuda_fail(e);
 }
 

@@ -29,6 +29,11 @@ struct WOperand {
 cudaError_t launch_tc_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
                               const WOperand* w, int nmat, cudaStream_t s);
 
+// Decode product (M <= 32): TMA-staged codes, in-register dequantisation,
+// warp-level tensor-core MMA (mma.sync), split-K over a cluster.
+cudaError_t launch_gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
+                                const WOperand* w, int nmat, cudaStream_t s);
+
 // Bounded-wait self test: a kernel waits on an mbarrier nothing completes.
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s);
 
