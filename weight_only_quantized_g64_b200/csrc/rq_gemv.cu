@@ -26,11 +26,13 @@
 // owns, per group of 64 k, the 16 k [16t, 16t+16) of rows g and g+8 of each
 // of its m-tiles: MMA k-slot sigma of step j maps to one of those k, the same
 // map on the A (weights) and B (x) side, so the sum over k is unchanged and
-// every thread's codes and x are contiguous in memory.  Codes become fp16
-// exactly (the biased code is placed in the mantissa of 1024 + u and the bias
-// is removed with one fp16 operation: Kim et al., arXiv:2211.10017); the MMA
-// sums x * code for one group in fp32 registers; the group's scale is applied
-// in fp32 (acc = fma(partial, s, acc)).  Nothing dequantised is stored.
+// every thread's codes and x are contiguous in memory.  Codes enter the MMA
+// as exact biased fp16 values (code + bias placed in the mantissa of an fp16
+// in [1024, 2048): Kim et al., arXiv:2211.10017); each group's fp32
+// accumulation is seeded with -bias * sum_k x (an MMA against a constant
+// operand), so the MMA yields sum_k x * code for the group; the group's scale
+// is applied in fp32 (acc = fma(partial, s, acc)).  Nothing dequantised is
+// stored.
 //
 // Split-K: CTAs of one cluster share a row tile and take disjoint k-stage
 // ranges; partials are summed in a fixed order through distributed shared
@@ -57,11 +59,10 @@ constexpr int kGvConsumers = 8;
 constexpr int kGvThreads = (kGvConsumers + 1) * 32;
 
 // BITS: 4 or 8.  NT: 8-token n-tiles (M <= 8 NT).  MT: 16-row m-tiles per
-// consumer warp.  PERM (int4 only): k-order of the fp16 pairs, see below.
-// SSC: scales staged in shared memory by the producer warp (needs the
+// consumer warp.  SSC: scales staged in shared memory by the producer warp (needs the
 // stage's groups to be all valid or all past the end: G % groups-per-stage
 // == 0); otherwise consumers load them from global memory.
-template <int BITS, int NT, int MT, bool PERM, bool SSC>
+template <int BITS, int NT, int MT, bool SSC>
 struct GvCfg {
     static constexpr int kRows = kGvConsumers * 16 * MT;      // weight rows per CTA
     static constexpr int kKPS = BITS == 4 ? 256 : 128;        // k per stage (128 code bytes)
@@ -71,7 +72,7 @@ struct GvCfg {
     static constexpr int kXStage = kGPS * kTok * 128;
     static constexpr int kSStage = SSC ? ((kRows * kGPS * 2 + 1023) / 1024) * 1024 : 0;
     static constexpr int kStage = kWStage + kXStage + kSStage;
-    static constexpr int kBudget = (NT == 1 ? 100 : 196) * 1024;   // two CTAs per SM when NT == 1
+    static constexpr int kBudget = (NT == 1 && MT == 1 ? 100 : 196) * 1024;   // two CTAs per SM when NT == MT == 1
     static constexpr int kSS = kBudget / kStage > 8 ? 8 : (kBudget / kStage < 2 ? 2 : kBudget / kStage);
     static constexpr int kRing = kSS * kStage;
     static constexpr int kRed = kTok * kRows * 4;
@@ -91,39 +92,34 @@ __device__ __forceinline__ uint32_t lop3_bmux(uint32_t a, uint32_t b, uint32_t c
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-// int4, permuted order: one 32-bit code word (slice positions 0..7 of one row)
-// -> four fp16 pairs holding the exact codes (p0,p4), (p1,p5), (p2,p6), (p3,p7).
-// 9 instructions per 8 codes; the x side is permuted to match.
-__device__ __forceinline__ void i4_word_to_pairs_perm(uint32_t w, uint32_t (&P)[4]) {
-    const __half2 bias_lo = u32_as_h2(0x64086408u);                      // 1032, 1032
-    const __half2 inv16 = u32_as_h2(0x2C002C00u);                        // 1/16
-    const __half2 bias_hi = u32_as_h2(0xD480D480u);                      // -72
-    const uint32_t w8 = w >> 8;
-    // low nibbles of bytes 0 and 2 -> 1024 + (nibble ^ 8); high nibbles -> 1024 + 16*(nibble ^ 8)
-    P[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_bmux(w, 0x000F000Fu, 0x64086408u)), bias_lo));
-    P[1] = h2_as_u32(__hfma2(u32_as_h2(lop3_bmux(w, 0x00F000F0u, 0x64806480u)), inv16, bias_hi));
-    P[2] = h2_as_u32(__hsub2(u32_as_h2(lop3_bmux(w8, 0x000F000Fu, 0x64086408u)), bias_lo));
-    P[3] = h2_as_u32(__hfma2(u32_as_h2(lop3_bmux(w8, 0x00F000F0u, 0x64806480u)), inv16, bias_hi));
-}
+// Code unpacking.  Each fp16 pair holds BIASED codes: the code plus a bias
+// placed in the mantissa of an fp16 in [1024, 2048), exact, with no
+// arithmetic (the bit placement of Kim et al., arXiv:2211.10017).  The bias is
+// removed inside the MMA: every group's accumulation starts from
+// -bias * sum_k x[k], itself computed by an MMA with a constant A operand.
+//   int4: 1024 + (nibble ^ 8) = code + 1032
+//   int8: 1024 + (byte ^ 0x80) = code + 1152
+constexpr uint32_t kBiasI4 = 0xE408E408u;   // fp16 pair (-1032, -1032)
+constexpr uint32_t kBiasI8 = 0xE480E480u;   // fp16 pair (-1152, -1152)
 
-// int4, natural order: one code word -> pairs (p0,p1), (p2,p3), (p4,p5), (p6,p7)
-// (the two nibbles of each byte), 13 instructions per 8 codes; x is used as is.
-__device__ __forceinline__ void i4_word_to_pairs_nat(uint32_t w, uint32_t (&P)[4]) {
-    const __half2 bias = u32_as_h2(0x64086408u);                         // 1032, 1032
+// int4: one 32-bit code word (positions 0..7 of one row, position 2i in the
+// low nibble of byte i) -> pairs (p0,p1), (p2,p3), (p4,p5), (p6,p7).
+// 9 instructions per 8 codes.
+__device__ __forceinline__ void i4_word_to_pairs(uint32_t w, uint32_t (&P)[4]) {
     const uint32_t w4 = w >> 4;   // byte b of w4 holds the high nibble of byte b of w in its low bits
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
         const uint32_t v = __byte_perm(w, w4, static_cast<uint32_t>(b) | ((4u + b) << 8));
-        P[b] = h2_as_u32(__hsub2(u32_as_h2(lop3_bmux(v, 0x000F000Fu, 0x64086408u)), bias));
+        P[b] = lop3_bmux(v, 0x000F000Fu, 0x64086408u);   // (nibble ^ 8) under exponent 0x64
     }
 }
 
-// int8: one 32-bit word (positions 0..3) -> fp16 pairs (p0, p1), (p2, p3).
+// int8: one 32-bit word (positions 0..3) -> pairs (p0, p1), (p2, p3).
+// 3 instructions per 4 codes.
 __device__ __forceinline__ void i8_word_to_pairs(uint32_t w, uint32_t (&Q)[2]) {
-    const __half2 bias = u32_as_h2(0x64806480u);                         // 1152 = 1024 + 128
     w ^= 0x80808080u;
-    Q[0] = h2_as_u32(__hsub2(u32_as_h2(__byte_perm(w, 0x64646464u, 0x5140u)), bias));
-    Q[1] = h2_as_u32(__hsub2(u32_as_h2(__byte_perm(w, 0x64646464u, 0x5342u)), bias));
+    Q[0] = __byte_perm(w, 0x64646464u, 0x5140u);
+    Q[1] = __byte_perm(w, 0x64646464u, 0x5342u);
 }
 
 // Not volatile: a pure function of its operands, so the compiler may
@@ -154,10 +150,10 @@ __device__ __forceinline__ int phys_row(int g) {
     else return (g >> 1) + 4 * (g & 1);
 }
 
-template <int BITS, int NT, int MT, bool PERM, bool SSC>
-__global__ void __launch_bounds__(kGvThreads, NT == 1 ? 2 : 1)
+template <int BITS, int NT, int MT, bool SSC>
+__global__ void __launch_bounds__(kGvThreads, (NT == 1 && MT == 1) ? 2 : 1)
     gemv_wq_kernel(const __grid_constant__ GvParams p) {
-    using Cfg = GvCfg<BITS, NT, MT, PERM, SSC>;
+    using Cfg = GvCfg<BITS, NT, MT, SSC>;
     constexpr int SS = Cfg::kSS;
     constexpr int ROWS = Cfg::kRows;
     constexpr int GPS = Cfg::kGPS;
@@ -331,6 +327,8 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 2 : 1)
 #pragma unroll
             for (int q = 0; q < GPS; ++q) {
                 // ---- x fragments of this group: B registers per n-tile and step
+                // (thread (g, t): token g of the n-tile, positions 16t .. 16t+15
+                // of the group; step j covers positions 4j .. 4j+3)
                 uint32_t b[NT][4][2];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
@@ -339,23 +337,22 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 2 : 1)
                     const int sw = tok & 7;
                     const uint4 x0 = *reinterpret_cast<const uint4*>(xrow + (((2 * t) ^ sw) << 4));
                     const uint4 x1 = *reinterpret_cast<const uint4*>(xrow + (((2 * t + 1) ^ sw) << 4));
-                    const uint32_t X[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                    if constexpr (BITS == 4 && PERM) {
-                        // step j pairs (p0,p4),(p1,p5) / (p2,p6),(p3,p7) of word group j/2
+                    b[nt][0][0] = x0.x; b[nt][0][1] = x0.y;
+                    b[nt][1][0] = x0.z; b[nt][1][1] = x0.w;
+                    b[nt][2][0] = x1.x; b[nt][2][1] = x1.y;
+                    b[nt][3][0] = x1.z; b[nt][3][1] = x1.w;
+                }
+                // ---- bias term of the group: -bias * sum_k x[tok, k], the same
+                // for every row; it seeds each m-tile's accumulation
+                float corr[NT][4];
+                {
+                    const uint32_t cb = BITS == 4 ? kBiasI4 : kBiasI8;
+                    const uint32_t Ac[4] = {cb, cb, cb, cb};
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int hb = (j >> 1) * 4;
-                            const int lo = (j & 1);
-                            b[nt][j][0] = __byte_perm(X[hb + lo], X[hb + lo + 2], 0x5410);
-                            b[nt][j][1] = __byte_perm(X[hb + lo], X[hb + lo + 2], 0x7632);
-                        }
-                    } else {
+                    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            b[nt][j][0] = X[2 * j];
-                            b[nt][j][1] = X[2 * j + 1];
-                        }
-                    }
+                        for (int j = 0; j < 4; ++j)
+                            mma16816(corr[nt], Ac, b[nt][j][0], b[nt][j][1], j == 0);
                 }
                 // ---- per m-tile: codes -> A registers, 4 MMA steps, scale
 #pragma unroll
@@ -371,14 +368,10 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 2 : 1)
                             const uint2 cw = *reinterpret_cast<const uint2*>(
                                 crow + (((2 * q + (t >> 1)) ^ sw) << 4) + ((t & 1) << 3));
                             uint32_t P0[4], P1[4];
-                            if constexpr (PERM) {
-                                i4_word_to_pairs_perm(cw.x, P0);
-                                i4_word_to_pairs_perm(cw.y, P1);
-                            } else {
-                                i4_word_to_pairs_nat(cw.x, P0);
-                                i4_word_to_pairs_nat(cw.y, P1);
-                            }
-                            // step j: a0a1 (h = 0) / a2a3 (h = 1) and a4a5 / a6a7
+                            i4_word_to_pairs(cw.x, P0);
+                            i4_word_to_pairs(cw.y, P1);
+                            // step j: a0a1 (h = 0) / a2a3 (h = 1) = positions 4j, 4j+1;
+                            //         a4a5 / a6a7 = positions 4j+2, 4j+3
                             A[0][h] = P0[0]; A[0][h + 2] = P0[1];
                             A[1][h] = P0[2]; A[1][h + 2] = P0[3];
                             A[2][h] = P1[0]; A[2][h + 2] = P1[1];
@@ -399,13 +392,15 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 2 : 1)
                     }
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
+                        // the bias chain runs beside this one (no dependency); it is
+                        // added to the group's partial before scaling
                         float part[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) mma16816(part, A[j], b[nt][j][0], b[nt][j][1], j == 0);
-                        acc[mi][nt][0] = fmaf(part[0], sv[mi][0][q], acc[mi][nt][0]);
-                        acc[mi][nt][1] = fmaf(part[1], sv[mi][0][q], acc[mi][nt][1]);
-                        acc[mi][nt][2] = fmaf(part[2], sv[mi][1][q], acc[mi][nt][2]);
-                        acc[mi][nt][3] = fmaf(part[3], sv[mi][1][q], acc[mi][nt][3]);
+                        acc[mi][nt][0] = fmaf(part[0] + corr[nt][0], sv[mi][0][q], acc[mi][nt][0]);
+                        acc[mi][nt][1] = fmaf(part[1] + corr[nt][1], sv[mi][0][q], acc[mi][nt][1]);
+                        acc[mi][nt][2] = fmaf(part[2] + corr[nt][2], sv[mi][1][q], acc[mi][nt][2]);
+                        acc[mi][nt][3] = fmaf(part[3] + corr[nt][3], sv[mi][1][q], acc[mi][nt][3]);
                     }
                 }
             }
@@ -478,11 +473,11 @@ static int gv_num_sms() {
     return sms;
 }
 
-template <int BITS, int NT, int MT, bool PERM, bool SSC>
+template <int BITS, int NT, int MT, bool SSC>
 static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* codes, int nmat,
                              cudaStream_t s) {
-    using Cfg = GvCfg<BITS, NT, MT, PERM, SSC>;
-    auto kern = gemv_wq_kernel<BITS, NT, MT, PERM, SSC>;
+    using Cfg = GvCfg<BITS, NT, MT, SSC>;
+    auto kern = gemv_wq_kernel<BITS, NT, MT, SSC>;
     static int resident[64] = {};   // CTAs per SM, per device (0 = not yet set up)
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -543,21 +538,23 @@ static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* co
 template <int BITS, bool SSC>
 static cudaError_t gv_dispatch_ssc(GvParams& prm, const void* x, const void* const* codes, int nmat,
                                    cudaStream_t s) {
-    // 8 tokens per n-tile.  int4 with one n-tile permutes x (cheaper code
-    // unpacking); with more n-tiles the natural pair order avoids touching x.
-    // Two m-tiles per warp halve the x traffic when N leaves enough tiles.
+    // 8 tokens per n-tile; two m-tiles per warp (x fragments and the bias
+    // term reused twice) when N leaves enough row tiles for the SMs.
     const bool wide = static_cast<int64_t>(nmat) * prm.N >= 8192;
-    if (prm.M <= 8) return gv_launch<BITS, 1, 1, true, SSC>(prm, x, codes, nmat, s);
+    if (prm.M <= 8) {
+        if (wide) return gv_launch<BITS, 1, 2, SSC>(prm, x, codes, nmat, s);
+        return gv_launch<BITS, 1, 1, SSC>(prm, x, codes, nmat, s);
+    }
     if (prm.M <= 16) {
-        if (wide) return gv_launch<BITS, 2, 2, false, SSC>(prm, x, codes, nmat, s);
-        return gv_launch<BITS, 2, 1, false, SSC>(prm, x, codes, nmat, s);
+        if (wide) return gv_launch<BITS, 2, 2, SSC>(prm, x, codes, nmat, s);
+        return gv_launch<BITS, 2, 1, SSC>(prm, x, codes, nmat, s);
     }
     if (prm.M <= 24) {
-        if (wide) return gv_launch<BITS, 3, 2, false, SSC>(prm, x, codes, nmat, s);
-        return gv_launch<BITS, 3, 1, false, SSC>(prm, x, codes, nmat, s);
+        if (wide) return gv_launch<BITS, 3, 2, SSC>(prm, x, codes, nmat, s);
+        return gv_launch<BITS, 3, 1, SSC>(prm, x, codes, nmat, s);
     }
-    if (wide) return gv_launch<BITS, 4, 2, false, SSC>(prm, x, codes, nmat, s);
-    return gv_launch<BITS, 4, 1, false, SSC>(prm, x, codes, nmat, s);
+    if (wide) return gv_launch<BITS, 4, 2, SSC>(prm, x, codes, nmat, s);
+    return gv_launch<BITS, 4, 1, SSC>(prm, x, codes, nmat, s);
 }
 
 template <int BITS>
