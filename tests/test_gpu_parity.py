@@ -301,3 +301,26 @@ def test_pdl_chain_matches():
         y_ref, bound = oracle.matmul(xh, ch, sh, bits)
         check_close(to_host(outs[i]), y_ref, bound, f"pdl chain {i}")
         xh = (to_host(outs[i]) * 0.05).astype(np.float16)
+
+
+# ------------------------------------------------------------ repeatability ---
+
+@pytest.mark.parametrize("path", ["gemv", "gemm"])
+def test_repeat_runs_bit_identical(path):
+    """Both kernels sum in a fixed order, so repeated runs must agree bit for
+    bit; a pipeline race (a stage read before or after its data) shows up here
+    even when it stays within tolerance."""
+    if path == "gemv":
+        N, K, M, bits = 4096, 4096, 5, 4
+    else:
+        N, K, M, bits = 1024, 8192, 512, 4
+    W = synth.weights(N, K, seed=31, device="cuda")
+    codes, scales = rq.quantize_g64(W, bits)
+    x = synth.activations(M, K, seed=31, device="cuda")
+    fn = rq.gemv_wq if path == "gemv" else rq.gemm_wq
+    ref = fn(x, codes, scales, N, bits)
+    torch.cuda.synchronize()
+    for _ in range(20):
+        y = fn(x, codes, scales, N, bits)
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref)

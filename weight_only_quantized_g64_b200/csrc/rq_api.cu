@@ -37,6 +37,72 @@ int* device_status_ptr() {
 uint64_t wait_limit_ns() { return g_wait_limit_ns; }
 bool pdl_enabled() { return g_pdl; }
 
+// ------------------------------------------------------------- workspace --
+struct Workspace {
+    float* ws = nullptr;
+    size_t ws_bytes = 0;
+    int* cnt = nullptr;
+    size_t n_cnt = 0;
+};
+static Workspace g_ws[kMaxDevices];
+
+cudaError_t workspace_get(size_t ws_bytes, size_t n_counters, float** ws, int** cnt) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace& w = g_ws[dev];
+    if (w.ws_bytes < ws_bytes) {
+        const size_t want = ws_bytes > (size_t{32} << 20) ? ws_bytes : (size_t{32} << 20);
+        void* p = nullptr;
+        if (w.ws != nullptr) {
+            e = cudaFree(w.ws);
+            if (e != cudaSuccess) return e;
+            w.ws = nullptr;
+            w.ws_bytes = 0;
+        }
+        e = cudaMalloc(&p, want);
+        if (e != cudaSuccess) return e;
+        w.ws = static_cast<float*>(p);
+        w.ws_bytes = want;
+    }
+    if (w.n_cnt < n_counters) {
+        const size_t want = n_counters > (size_t{1} << 18) ? n_counters : (size_t{1} << 18);
+        void* p = nullptr;
+        if (w.cnt != nullptr) {
+            e = cudaFree(w.cnt);
+            if (e != cudaSuccess) return e;
+            w.cnt = nullptr;
+            w.n_cnt = 0;
+        }
+        e = cudaMalloc(&p, want * sizeof(int));
+        if (e != cudaSuccess) return e;
+        e = cudaMemset(p, 0, want * sizeof(int));
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) return e;
+        w.cnt = static_cast<int*>(p);
+        w.n_cnt = want;
+    }
+    *ws = w.ws;
+    *cnt = w.cnt;
+    return cudaSuccess;
+}
+
+cudaError_t workspace_reset_counters() {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace& w = g_ws[dev];
+    if (w.cnt == nullptr) return cudaSuccess;
+    e = cudaMemset(w.cnt, 0, w.n_cnt * sizeof(int));
+    if (e != cudaSuccess) return e;
+    return cudaDeviceSynchronize();
+}
+
 // ------------------------------------------------------------ tensor maps --
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -185,6 +251,8 @@ rq_status rq_read_device_status(int* out, int reset) {
     if (reset) {
         const int zero = 0;
         e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = workspace_reset_counters();
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return RQ_OK;

@@ -26,17 +26,19 @@
 // owns, per group of 64 k, the 16 k [16t, 16t+16) of rows g and g+8 of each
 // of its m-tiles: MMA k-slot sigma of step j maps to one of those k, the same
 // map on the A (weights) and B (x) side, so the sum over k is unchanged and
-// every thread's codes and x are contiguous in memory.  Codes enter the MMA
-// as exact biased fp16 values (code + bias placed in the mantissa of an fp16
-// in [1024, 2048): Kim et al., arXiv:2211.10017); each group's fp32
-// accumulation is seeded with -bias * sum_k x (an MMA against a constant
-// operand), so the MMA yields sum_k x * code for the group; the group's scale
-// is applied in fp32 (acc = fma(partial, s, acc)).  Nothing dequantised is
-// stored.
+// every thread's codes and x are contiguous in memory.  Codes become exact
+// fp16 values in registers (bit placement plus one exact fp16 operation:
+// Kim et al., arXiv:2211.10017); the MMA sums x * code for one group in fp32
+// registers; the group's scale is applied in fp32 (acc = fma(partial, s,
+// acc)).  Nothing dequantised is stored.
 //
-// Split-K: CTAs of one cluster share a row tile and take disjoint k-stage
-// ranges; partials are summed in a fixed order through distributed shared
-// memory (deterministic, no atomics, no global workspace).
+// Work split (stream-K): the work is a list of units (one 128-row tile x one
+// k-stage, tile-major) cut into equal contiguous runs, one per resident CTA,
+// so every SM streams the same number of bytes whatever the shape.  A CTA
+// stores a tile it covers whole directly; a tile shared by several CTAs is
+// stored as pieces in a global workspace and summed, in a fixed CTA order, by
+// whichever contributor arrives last (an atomic counter per tile), so results
+// are deterministic.
 #include "rq_internal.h"
 #include "rq_ptx.cuh"
 
@@ -49,8 +51,13 @@ struct GvParams {
     float* y[3];
     int M, N, K;
     int n_tiles;          // row tiles per matrix
-    int kstages;          // k stages per row (ceil(K / k-per-stage))
+    int kstages;          // k stages per row tile (ceil(K / k-per-stage))
     int groups;           // K / 64
+    int units;            // work units: nmat * n_tiles * kstages (one tile x one stage each)
+    int uq, ur;           // units / gridDim.x and units % gridDim.x: CTA c owns
+                          // [c*uq + min(c, ur), (c+1)*uq + min(c+1, ur))
+    float* ws;            // partial-tile slots: [2 * gridDim.x][8*NT tokens * ROWS rows] fp32
+    int* cnt;             // per-tile arrival counters, zero between launches
     int* status;
     uint64_t timeout_ns;
 };
@@ -92,34 +99,44 @@ __device__ __forceinline__ uint32_t lop3_bmux(uint32_t a, uint32_t b, uint32_t c
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-// Code unpacking.  Each fp16 pair holds BIASED codes: the code plus a bias
-// placed in the mantissa of an fp16 in [1024, 2048), exact, with no
-// arithmetic (the bit placement of Kim et al., arXiv:2211.10017).  The bias is
-// removed inside the MMA: every group's accumulation starts from
-// -bias * sum_k x[k], itself computed by an MMA with a constant A operand.
-//   int4: 1024 + (nibble ^ 8) = code + 1032
-//   int8: 1024 + (byte ^ 0x80) = code + 1152
-constexpr uint32_t kBiasI4 = 0xE408E408u;   // fp16 pair (-1032, -1032)
-constexpr uint32_t kBiasI8 = 0xE480E480u;   // fp16 pair (-1152, -1152)
+// Code unpacking to EXACT fp16 codes, without integer->float conversions:
+// the biased code is placed in the mantissa of an fp16 in [1024, 2048) and
+// the bias is removed with one exact fp16 operation (the bit placement of
+// Kim et al., "Who Says Elephants Can't Run?", arXiv:2211.10017).
 
-// int4: one 32-bit code word (positions 0..7 of one row, position 2i in the
-// low nibble of byte i) -> pairs (p0,p1), (p2,p3), (p4,p5), (p6,p7).
-// 9 instructions per 8 codes.
-__device__ __forceinline__ void i4_word_to_pairs(uint32_t w, uint32_t (&P)[4]) {
+// int4, permuted order: one code word (positions 0..7 of a row, position 2i
+// in the low nibble of byte i) -> pairs (p0,p4), (p1,p5), (p2,p6), (p3,p7).
+// 9 instructions per 8 codes; x is permuted to the same order.
+__device__ __forceinline__ void i4_word_to_pairs_perm(uint32_t w, uint32_t (&P)[4]) {
+    const __half2 bias_lo = u32_as_h2(0x64086408u);                      // 1032, 1032
+    const __half2 inv16 = u32_as_h2(0x2C002C00u);                        // 1/16
+    const __half2 bias_hi = u32_as_h2(0xD480D480u);                      // -72
+    const uint32_t w8 = w >> 8;
+    // low nibbles of bytes 0 and 2 -> 1024 + (nibble ^ 8); high nibbles -> 1024 + 16*(nibble ^ 8)
+    P[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_bmux(w, 0x000F000Fu, 0x64086408u)), bias_lo));
+    P[1] = h2_as_u32(__hfma2(u32_as_h2(lop3_bmux(w, 0x00F000F0u, 0x64806480u)), inv16, bias_hi));
+    P[2] = h2_as_u32(__hsub2(u32_as_h2(lop3_bmux(w8, 0x000F000Fu, 0x64086408u)), bias_lo));
+    P[3] = h2_as_u32(__hfma2(u32_as_h2(lop3_bmux(w8, 0x00F000F0u, 0x64806480u)), inv16, bias_hi));
+}
+
+// int4, natural order: one code word -> pairs (p0,p1), (p2,p3), (p4,p5), (p6,p7)
+// (the two nibbles of each byte).  13 instructions per 8 codes; x is used as is.
+__device__ __forceinline__ void i4_word_to_pairs_nat(uint32_t w, uint32_t (&P)[4]) {
+    const __half2 bias = u32_as_h2(0x64086408u);                         // 1032, 1032
     const uint32_t w4 = w >> 4;   // byte b of w4 holds the high nibble of byte b of w in its low bits
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
         const uint32_t v = __byte_perm(w, w4, static_cast<uint32_t>(b) | ((4u + b) << 8));
-        P[b] = lop3_bmux(v, 0x000F000Fu, 0x64086408u);   // (nibble ^ 8) under exponent 0x64
+        P[b] = h2_as_u32(__hsub2(u32_as_h2(lop3_bmux(v, 0x000F000Fu, 0x64086408u)), bias));
     }
 }
 
-// int8: one 32-bit word (positions 0..3) -> pairs (p0, p1), (p2, p3).
-// 3 instructions per 4 codes.
+// int8: one 32-bit word (positions 0..3) -> exact pairs (p0, p1), (p2, p3).
 __device__ __forceinline__ void i8_word_to_pairs(uint32_t w, uint32_t (&Q)[2]) {
+    const __half2 bias = u32_as_h2(0x64806480u);                         // 1152 = 1024 + 128
     w ^= 0x80808080u;
-    Q[0] = __byte_perm(w, 0x64646464u, 0x5140u);
-    Q[1] = __byte_perm(w, 0x64646464u, 0x5342u);
+    Q[0] = h2_as_u32(__hsub2(u32_as_h2(__byte_perm(w, 0x64646464u, 0x5140u)), bias));
+    Q[1] = h2_as_u32(__hsub2(u32_as_h2(__byte_perm(w, 0x64646464u, 0x5342u)), bias));
 }
 
 // Not volatile: a pure function of its operands, so the compiler may
@@ -150,6 +167,22 @@ __device__ __forceinline__ int phys_row(int g) {
     else return (g >> 1) + 4 * (g & 1);
 }
 
+// First work unit of CTA c: the first ur CTAs take uq + 1 units, the rest uq.
+__device__ __forceinline__ int range_begin(int c, int uq, int ur) {
+    return c * uq + (c < ur ? c : ur);
+}
+
+// The CTA whose unit range holds unit u.
+__device__ __forceinline__ int range_owner(int u, int uq, int ur) {
+    const int big = ur * (uq + 1);
+    return u < big ? u / (uq + 1) : ur + (u - big) / uq;
+}
+
+// Named barrier over the eight consumer warps (the producer warp is not in it).
+__device__ __forceinline__ void consumers_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kGvConsumers * 32) : "memory");
+}
+
 template <int BITS, int NT, int MT, bool SSC>
 __global__ void __launch_bounds__(kGvThreads, (NT == 1 && MT == 1) ? 2 : 1)
     gemv_wq_kernel(const __grid_constant__ GvParams p) {
@@ -165,16 +198,18 @@ __global__ void __launch_bounds__(kGvThreads, (NT == 1 && MT == 1) ? 2 : 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kData);
     uint64_t* empty = full + SS;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + SS);
+    volatile int* last_flag = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int ksplit = gridDim.x;
-    const int kq = blockIdx.x;
-    const int mat = blockIdx.y / p.n_tiles;
-    const int n0 = (blockIdx.y - mat * p.n_tiles) * ROWS;
-    const int st0 = static_cast<int>((static_cast<int64_t>(kq) * p.kstages) / ksplit);
-    const int st1 = static_cast<int>((static_cast<int64_t>(kq + 1) * p.kstages) / ksplit);
-    const int nst = st1 - st0;
+    const int G = static_cast<int>(gridDim.x);
+    const int cta = static_cast<int>(blockIdx.x);
+    const int S = p.kstages;
+    const int u0 = range_begin(cta, p.uq, p.ur);
+    const int nu = p.uq + (cta < p.ur ? 1 : 0);
+    // position of the first unit: tile (matrix, row tile) and k-stage
+    const int tile0 = u0 / S;
+    const int st0 = u0 - tile0 * S;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SS; ++s) {
@@ -182,11 +217,13 @@ __global__ void __launch_bounds__(kGvThreads, (NT == 1 && MT == 1) ? 2 : 1)
             mbar_init(&empty[s], kGvConsumers);
         }
         *abort_flag = 0;
+        *last_flag = 0;
         fence_mbar_init();
     }
     if (warp == kGvConsumers && lane == 0) {
         tma_prefetch_desc(&p.tm_x);
-        tma_prefetch_desc(&p.tm_w[mat]);
+        for (int m = 0; m < 3; ++m)
+            if (p.y[m] != nullptr) tma_prefetch_desc(&p.tm_w[m]);
     }
     __syncthreads();
     pdl_launch_dependents();
@@ -194,17 +231,25 @@ __global__ void __launch_bounds__(kGvThreads, (NT == 1 && MT == 1) ? 2 : 1)
     if (warp == kGvConsumers) {
         // ---------------------------------------------- producer warp --
         // lane 0 issues the TMA copies; with SSC every lane also copies the
-        // stage's scales (rows lane, lane+32, ...) with cp.async completing
-        // on the same barrier.
+        // unit's scales (rows lane, lane+32, ...) with cp.async completing on
+        // the same barrier.
         const bool leader = lane == 0;
         const uint64_t pol_w = l2_policy_evict_first();
         const uint64_t pol_x = l2_policy_evict_last();
-        const CUtensorMap* tmw = &p.tm_w[mat];
-        const uint16_t* sbase = p.scales[mat];
-        auto stage_scales = [&](int i, int s) {
+        // position of the next unit to issue, advanced one unit at a time
+        int c_st = st0, c_tm = tile0 % p.n_tiles, c_mat = tile0 / p.n_tiles;
+        auto unit_codes = [&](int s) {
+            const int st = c_st;
+            const int mat = c_mat;
+            const int n0 = c_tm * ROWS;
+            if (leader) {
+                mbar_arrive_expect_tx(&full[s], Cfg::kWStage + Cfg::kXStage);
+                tma_load_2d(ring + s * Cfg::kStage, &p.tm_w[mat], &full[s], st * 128, n0, pol_w);
+            }
             if constexpr (SSC) {
                 uint8_t* dst = ring + s * Cfg::kStage + Cfg::kWStage + Cfg::kXStage;
-                const int grp = (st0 + i) * GPS;
+                const int grp = st * GPS;
+                const uint16_t* sbase = p.scales[mat];
 #pragma unroll
                 for (int rr = lane; rr < ROWS; rr += 32) {
                     const int n = n0 + rr;
@@ -216,37 +261,45 @@ __global__ void __launch_bounds__(kGvThreads, (NT == 1 && MT == 1) ? 2 : 1)
                 cp_async_arrive_noinc(&full[s]);
             }
         };
-        const int pre = nst < SS ? nst : SS;
-        for (int i = 0; i < pre; ++i) {
-            if (leader) {
-                mbar_arrive_expect_tx(&full[i], Cfg::kWStage + Cfg::kXStage);
-                tma_load_2d(ring + i * Cfg::kStage, tmw, &full[i], (st0 + i) * 128, n0, pol_w);
+        auto advance = [&]() {
+            if (++c_st == S) {
+                c_st = 0;
+                if (++c_tm == p.n_tiles) {
+                    c_tm = 0;
+                    ++c_mat;
+                }
             }
-            stage_scales(i, i);
+        };
+        auto unit_x = [&](int st, int s) {
+#pragma unroll
+            for (int q = 0; q < GPS; ++q)
+                tma_load_2d(ring + s * Cfg::kStage + Cfg::kWStage + q * TOK * 128, &p.tm_x,
+                            &full[s], st * Cfg::kKPS + q * 64, 0, pol_x);
+        };
+        const int pre = nu < SS ? nu : SS;
+        // Weights do not depend on the previous kernel: fetch them first.
+        for (int i = 0; i < pre; ++i) {
+            unit_codes(i);
+            advance();
         }
         if (leader) {
             pdl_wait();   // x may be produced by the previous kernel
-            for (int i = 0; i < pre; ++i)
-#pragma unroll
-                for (int q = 0; q < GPS; ++q)
-                    tma_load_2d(ring + i * Cfg::kStage + Cfg::kWStage + q * TOK * 128, &p.tm_x,
-                                &full[i], (st0 + i) * Cfg::kKPS + q * 64, 0, pol_x);
+            int st = st0;
+            for (int i = 0; i < pre; ++i) {
+                unit_x(st, i);
+                if (++st == S) st = 0;
+            }
         }
         int issued = pre;
-        for (int i = SS; i < nst; ++i) {
+        for (int i = SS; i < nu; ++i) {
             const int s = i % SS;
             if (!mbar_wait(&empty[s], static_cast<uint32_t>(i / SS - 1) & 1, abort_flag,
                            p.timeout_ns, p.status))
                 break;
-            if (leader) {
-                mbar_arrive_expect_tx(&full[s], Cfg::kWStage + Cfg::kXStage);
-                tma_load_2d(ring + s * Cfg::kStage, tmw, &full[s], (st0 + i) * 128, n0, pol_w);
-#pragma unroll
-                for (int q = 0; q < GPS; ++q)
-                    tma_load_2d(ring + s * Cfg::kStage + Cfg::kWStage + q * TOK * 128, &p.tm_x,
-                                &full[s], (st0 + i) * Cfg::kKPS + q * 64, 0, pol_x);
-            }
-            stage_scales(i, s);
+            const int st = c_st;
+            unit_codes(s);
+            if (leader) unit_x(st, s);
+            advance();
             issued = i + 1;
         }
         // Wait (bounded, regardless of abort) until every copy this warp
@@ -257,57 +310,86 @@ __global__ void __launch_bounds__(kGvThreads, (NT == 1 && MT == 1) ? 2 : 1)
             mbar_wait(&full[i % SS], static_cast<uint32_t>(i / SS) & 1, &dummy_abort,
                       p.timeout_ns, p.status);
         __syncwarp();
-    }
-
-    float acc[MT][NT][4];
-#pragma unroll
-    for (int i = 0; i < MT; ++i)
-#pragma unroll
-        for (int j = 0; j < NT; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.0f;
-
-    const int g = lane >> 2;
-    const int t = lane & 3;
-    const int rbase = warp * 16 * MT;           // this warp's first row in the tile
-    if (warp < kGvConsumers) {
+    } else {
         // ---------------------------------------------------- consumers --
+        const int g = lane >> 2;
+        const int t = lane & 3;
+        const int rbase = warp * 16 * MT;       // this warp's first row in a tile
         int rloc[MT][2];                        // physical rows (within the tile)
 #pragma unroll
         for (int i = 0; i < MT; ++i)
 #pragma unroll
             for (int h = 0; h < 2; ++h) rloc[i][h] = rbase + 16 * i + phys_row<BITS>(g) + 8 * h;
-        // global scale pointers, only for the path without shared-memory scales
-        const uint16_t* srow[MT][2];
-        bool rok[MT][2];
-#pragma unroll
-        for (int i = 0; i < MT; ++i)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int n = n0 + rloc[i][h];
-                rok[i][h] = n < p.N;
-                srow[i][h] = p.scales[mat] + static_cast<int64_t>(rok[i][h] ? n : 0) * p.groups;
-            }
 
-        for (int i = 0; i < nst; ++i) {
+        float acc[MT][NT][4];
+        int seg_first_i = 0;                    // unit index where the current segment began
+        // After a timeout a warp keeps walking the units without working, so
+        // every consumer warp reaches the same named barriers: none can wait
+        // at one that another warp has left.
+        bool dead = false;
+        int st = st0, tile = tile0, tm = tile0 % p.n_tiles, mat = tile0 / p.n_tiles;
+        for (int i = 0; i < nu; ++i) {
+            if (i > 0 && ++st == S) {     // next unit: next stage, or next row tile
+                st = 0;
+                ++tile;
+                if (++tm == p.n_tiles) {
+                    tm = 0;
+                    ++mat;
+                }
+            }
+            const int n0 = tm * ROWS;
+            if (i == 0 || st == 0) {
+                seg_first_i = i;
+#pragma unroll
+                for (int a = 0; a < MT; ++a)
+#pragma unroll
+                    for (int j = 0; j < NT; ++j)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[a][j][e] = 0.0f;
+            }
             const int s = i % SS;
-            if (!mbar_wait(&full[s], static_cast<uint32_t>(i / SS) & 1, abort_flag, p.timeout_ns,
-                           p.status))
-                break;
+            if (!dead && !mbar_wait(&full[s], static_cast<uint32_t>(i / SS) & 1, abort_flag,
+                                    p.timeout_ns, p.status))
+                dead = true;
+            if (!dead) {
             const uint8_t* wt = ring + s * Cfg::kStage;
             const uint8_t* xt = wt + Cfg::kWStage;
-            // scales of this stage for the thread's rows: [m-tile][half][group]
-            float sv[MT][2][GPS];
+            // int4 with one n-tile uses the permuted pair order (cheapest
+            // unpacking; x permuted once per group and n-tile)
+            constexpr bool PERM = BITS == 4 && NT == 1;
+            constexpr int CW = BITS == 4 ? 2 : 4;            // code words per row and group
+            // ---- the unit's shared-memory operands, all loaded up front
+            float sv[MT][2][GPS];                             // scales [m-tile][half][group]
+            uint32_t cw[GPS][MT][2][CW];                      // code words
 #pragma unroll
             for (int a = 0; a < MT; ++a)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
+                    const int r = rloc[a][h];
+                    const uint8_t* crow = wt + r * 128;
+                    const int sw = r & 7;
+#pragma unroll
+                    for (int q = 0; q < GPS; ++q) {
+                        if constexpr (BITS == 4) {
+                            // bytes [32q + 8t, +8): chunk 2q + t/2, offset (t&1)*8
+                            const uint2 v = *reinterpret_cast<const uint2*>(
+                                crow + (((2 * q + (t >> 1)) ^ sw) << 4) + ((t & 1) << 3));
+                            cw[q][a][h][0] = v.x;
+                            cw[q][a][h][1] = v.y;
+                        } else {
+                            // bytes [64q + 16t, +16): chunk 4q + t
+                            const uint4 v = *reinterpret_cast<const uint4*>(
+                                crow + (((4 * q + t) ^ sw) << 4));
+                            cw[q][a][h][0] = v.x; cw[q][a][h][1] = v.y;
+                            cw[q][a][h][2] = v.z; cw[q][a][h][3] = v.w;
+                        }
+                    }
                     if constexpr (SSC) {
-                        const uint8_t* sp = xt + Cfg::kXStage + rloc[a][h] * GPS * 2;
+                        const uint8_t* sp = xt + Cfg::kXStage + r * GPS * 2;
                         if constexpr (GPS == 4) {
-                            const uint2 u = *reinterpret_cast<const uint2*>(sp);
-                            const float2 f0 = __half22float2(u32_as_h2(u.x));
-                            const float2 f1 = __half22float2(u32_as_h2(u.y));
+                            const uint2 uu = *reinterpret_cast<const uint2*>(sp);
+                            const float2 f0 = __half22float2(u32_as_h2(uu.x));
+                            const float2 f1 = __half22float2(u32_as_h2(uu.y));
                             sv[a][h][0] = f0.x; sv[a][h][1] = f0.y;
                             sv[a][h][2] = f1.x; sv[a][h][3] = f1.y;
                         } else {
@@ -315,11 +397,13 @@ __global__ void __launch_bounds__(kGvThreads, (NT == 1 && MT == 1) ? 2 : 1)
                             sv[a][h][0] = f0.x; sv[a][h][1] = f0.y;
                         }
                     } else {
+                        const int n = n0 + r;
+                        const uint16_t* srow = p.scales[mat] + static_cast<int64_t>(n < p.N ? n : 0) * p.groups;
 #pragma unroll
                         for (int q = 0; q < GPS; ++q) {
-                            const int grp = (st0 + i) * GPS + q;
-                            sv[a][h][q] = (rok[a][h] && grp < p.groups)
-                                              ? __half2float(__ushort_as_half(__ldg(srow[a][h] + grp)))
+                            const int grp = st * GPS + q;
+                            sv[a][h][q] = (n < p.N && grp < p.groups)
+                                              ? __half2float(__ushort_as_half(__ldg(srow + grp)))
                                               : 0.0f;
                         }
                     }
@@ -337,54 +421,46 @@ __global__ void __launch_bounds__(kGvThreads, (NT == 1 && MT == 1) ? 2 : 1)
                     const int sw = tok & 7;
                     const uint4 x0 = *reinterpret_cast<const uint4*>(xrow + (((2 * t) ^ sw) << 4));
                     const uint4 x1 = *reinterpret_cast<const uint4*>(xrow + (((2 * t + 1) ^ sw) << 4));
-                    b[nt][0][0] = x0.x; b[nt][0][1] = x0.y;
-                    b[nt][1][0] = x0.z; b[nt][1][1] = x0.w;
-                    b[nt][2][0] = x1.x; b[nt][2][1] = x1.y;
-                    b[nt][3][0] = x1.z; b[nt][3][1] = x1.w;
-                }
-                // ---- bias term of the group: -bias * sum_k x[tok, k], the same
-                // for every row; it seeds each m-tile's accumulation
-                float corr[NT][4];
-                {
-                    const uint32_t cb = BITS == 4 ? kBiasI4 : kBiasI8;
-                    const uint32_t Ac[4] = {cb, cb, cb, cb};
+                    const uint32_t X[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            mma16816(corr[nt], Ac, b[nt][j][0], b[nt][j][1], j == 0);
+                    for (int j = 0; j < 4; ++j) {
+                        if constexpr (PERM) {
+                            // step j pairs (p0,p4),(p1,p5) or (p2,p6),(p3,p7) of word j/2
+                            const int wb = (j >> 1) * 4 + (j & 1);
+                            b[nt][j][0] = __byte_perm(X[wb], X[wb + 2], 0x5410);
+                            b[nt][j][1] = __byte_perm(X[wb], X[wb + 2], 0x7632);
+                        } else {
+                            b[nt][j][0] = X[2 * j];
+                            b[nt][j][1] = X[2 * j + 1];
+                        }
+                    }
                 }
-                // ---- per m-tile: codes -> A registers, 4 MMA steps, scale
+                // ---- per m-tile: exact fp16 codes -> A registers, 4 MMA steps,
+                // the group's scale in fp32
 #pragma unroll
                 for (int mi = 0; mi < MT; ++mi) {
                     uint32_t A[4][4];   // [step][a-reg]
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const int r = rloc[mi][h];
-                        const uint8_t* crow = wt + r * 128;
-                        const int sw = r & 7;
                         if constexpr (BITS == 4) {
-                            // bytes [32q + 8t, +8): chunk 2q + t/2, offset (t&1)*8
-                            const uint2 cw = *reinterpret_cast<const uint2*>(
-                                crow + (((2 * q + (t >> 1)) ^ sw) << 4) + ((t & 1) << 3));
                             uint32_t P0[4], P1[4];
-                            i4_word_to_pairs(cw.x, P0);
-                            i4_word_to_pairs(cw.y, P1);
-                            // step j: a0a1 (h = 0) / a2a3 (h = 1) = positions 4j, 4j+1;
-                            //         a4a5 / a6a7 = positions 4j+2, 4j+3
+                            if constexpr (PERM) {
+                                i4_word_to_pairs_perm(cw[q][mi][h][0], P0);
+                                i4_word_to_pairs_perm(cw[q][mi][h][1], P1);
+                            } else {
+                                i4_word_to_pairs_nat(cw[q][mi][h][0], P0);
+                                i4_word_to_pairs_nat(cw[q][mi][h][1], P1);
+                            }
+                            // step j: a0a1 (h = 0) / a2a3 (h = 1), and a4a5 / a6a7
                             A[0][h] = P0[0]; A[0][h + 2] = P0[1];
                             A[1][h] = P0[2]; A[1][h + 2] = P0[3];
                             A[2][h] = P1[0]; A[2][h + 2] = P1[1];
                             A[3][h] = P1[2]; A[3][h + 2] = P1[3];
                         } else {
-                            // bytes [64q + 16t, +16): chunk 4q + t
-                            const uint4 cw = *reinterpret_cast<const uint4*>(
-                                crow + (((4 * q + t) ^ sw) << 4));
-                            const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 uint32_t Q[2];
-                                i8_word_to_pairs(wv[j], Q);
+                                i8_word_to_pairs(cw[q][mi][h][j], Q);
                                 A[j][h] = Q[0];
                                 A[j][h + 2] = Q[1];
                             }
@@ -392,71 +468,103 @@ __global__ void __launch_bounds__(kGvThreads, (NT == 1 && MT == 1) ? 2 : 1)
                     }
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        // the bias chain runs beside this one (no dependency); it is
-                        // added to the group's partial before scaling
                         float part[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) mma16816(part, A[j], b[nt][j][0], b[nt][j][1], j == 0);
-                        acc[mi][nt][0] = fmaf(part[0] + corr[nt][0], sv[mi][0][q], acc[mi][nt][0]);
-                        acc[mi][nt][1] = fmaf(part[1] + corr[nt][1], sv[mi][0][q], acc[mi][nt][1]);
-                        acc[mi][nt][2] = fmaf(part[2] + corr[nt][2], sv[mi][1][q], acc[mi][nt][2]);
-                        acc[mi][nt][3] = fmaf(part[3] + corr[nt][3], sv[mi][1][q], acc[mi][nt][3]);
+                        acc[mi][nt][0] = fmaf(part[0], sv[mi][0][q], acc[mi][nt][0]);
+                        acc[mi][nt][1] = fmaf(part[1], sv[mi][0][q], acc[mi][nt][1]);
+                        acc[mi][nt][2] = fmaf(part[2], sv[mi][1][q], acc[mi][nt][2]);
+                        acc[mi][nt][3] = fmaf(part[3], sv[mi][1][q], acc[mi][nt][3]);
                     }
                 }
             }
+            }   // !dead
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-        }
-    }
+            if (lane == 0 && !dead) mbar_arrive(&empty[s]);
 
-    __syncthreads();   // every stage consumed: the ring is free for the partials
-
-    float* y = p.y[mat];
-    if (warp < kGvConsumers && !*abort_flag) {
-        float* red = reinterpret_cast<float*>(ring);
+            // ---- end of a tile segment: store it, or combine partial tiles
+            if (st == S - 1 || i == nu - 1) {
+                float* y = p.y[mat];
+                const bool whole = (i - seg_first_i) == st && st == S - 1;   // began at stage 0
+                if (whole && !dead) {
 #pragma unroll
-        for (int mi = 0; mi < MT; ++mi)
+                    for (int mi = 0; mi < MT; ++mi)
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+                        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = rbase + 16 * mi + phys_row<BITS>(g) + ((e >> 1) << 3);
-                    const int tok = nt * 8 + 2 * t + (e & 1);
-                    if (ksplit == 1) {
-                        const int n = n0 + r;
-                        if (n < p.N && tok < p.M) y[static_cast<int64_t>(tok) * p.N + n] = acc[mi][nt][e];
-                    } else {
-                        red[tok * ROWS + r] = acc[mi][nt][e];
+                            for (int e = 0; e < 4; ++e) {
+                                const int n = n0 + rloc[mi][e >> 1];
+                                const int tok = nt * 8 + 2 * t + (e & 1);
+                                if (n < p.N && tok < p.M)
+                                    y[static_cast<int64_t>(tok) * p.N + n] = acc[mi][nt][e];
+                            }
+                } else if (!whole) {
+                    // This CTA's piece of a tile that several CTAs share: slot 2c
+                    // for the CTA's first segment, 2c+1 for its last one.
+                    const int slot = 2 * cta + (seg_first_i == 0 ? 0 : 1);
+                    float* wsl = p.ws + static_cast<int64_t>(slot) * (TOK * ROWS);
+                    if (!dead)
+#pragma unroll
+                    for (int mi = 0; mi < MT; ++mi)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                wsl[(nt * 8 + 2 * t + (e & 1)) * ROWS + rloc[mi][e >> 1]] = acc[mi][nt][e];
+                    const int tb = tile * S;
+                    const int c_first = range_owner(tb, p.uq, p.ur);
+                    const int c_last = range_owner(tb + S - 1, p.uq, p.ur);
+                    consumers_sync();
+                    if (threadIdx.x == 0) {
+                        if (*abort_flag) {
+                            *last_flag = 0;
+                        } else {
+                            __threadfence();
+                            const int arrived = atomicAdd(&p.cnt[tile], 1);
+                            *last_flag = arrived == c_last - c_first;
+                        }
                     }
-                }
-    }
-
-    if (ksplit > 1) {
-        __syncthreads();
-        cluster_sync();
-        if (!*abort_flag) {
-            constexpr int E4 = TOK * ROWS / 4;
-            const int e0 = static_cast<int>((static_cast<int64_t>(kq) * E4) / ksplit);
-            const int e1 = static_cast<int>((static_cast<int64_t>(kq + 1) * E4) / ksplit);
-            const uint32_t red_local = smem_u32(ring);
-            for (int e = e0 + static_cast<int>(threadIdx.x); e < e1; e += kGvThreads) {
-                float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int src = 0; src < ksplit; ++src) {
-                    const float4 v = ld_dsmem_f32x4(map_to_rank(red_local + e * 16, src));
-                    sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-                }
-                const int tok = (e * 4) / ROWS;
-                const int r = (e * 4) % ROWS;
-                if (tok < p.M) {
-                    const float out[4] = {sum.x, sum.y, sum.z, sum.w};
-                    float* yrow = y + static_cast<int64_t>(tok) * p.N;
+                    consumers_sync();
+                    if (*last_flag) {
+                        // Last arrival: sum every contributor's piece in CTA
+                        // order (deterministic) and write the tile.
+                        __threadfence();
+                        float sum[MT][NT][4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        if (n0 + r + u < p.N) yrow[n0 + r + u] = out[u];
+                        for (int mi = 0; mi < MT; ++mi)
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) sum[mi][nt][e] = 0.0f;
+                        for (int c = c_first; c <= c_last; ++c) {
+                            const int sl = 2 * c + (range_begin(c, p.uq, p.ur) < tb ? 1 : 0);
+                            const float* src = p.ws + static_cast<int64_t>(sl) * (TOK * ROWS);
+#pragma unroll
+                            for (int mi = 0; mi < MT; ++mi)
+#pragma unroll
+                                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e)
+                                        sum[mi][nt][e] += __ldcg(src + (nt * 8 + 2 * t + (e & 1)) * ROWS +
+                                                                 rloc[mi][e >> 1]);
+                        }
+#pragma unroll
+                        for (int mi = 0; mi < MT; ++mi)
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int n = n0 + rloc[mi][e >> 1];
+                                    const int tok = nt * 8 + 2 * t + (e & 1);
+                                    if (n < p.N && tok < p.M)
+                                        y[static_cast<int64_t>(tok) * p.N + n] = sum[mi][nt][e];
+                                }
+                        if (threadIdx.x == 0) p.cnt[tile] = 0;   // ready for the next launch
+                    }
+                    consumers_sync();
                 }
             }
         }
-        cluster_sync();
     }
 }
 
@@ -486,8 +594,6 @@ static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* co
     if (resident[dev] == 0) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
         int occ = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGvThreads, Cfg::kSmem);
         if (e != cudaSuccess) return e;
@@ -496,9 +602,18 @@ static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* co
     prm.n_tiles = (prm.N + Cfg::kRows - 1) / Cfg::kRows;
     prm.kstages = (prm.K + Cfg::kKPS - 1) / Cfg::kKPS;
     const int64_t tiles = static_cast<int64_t>(nmat) * prm.n_tiles;
+    const int64_t units = tiles * prm.kstages;
+    if (units >= (int64_t{1} << 31)) return cudaErrorInvalidValue;
+    prm.units = static_cast<int>(units);
+    // One wave of resident CTAs, each taking an equal run of units.
     const int64_t slots = static_cast<int64_t>(resident[dev]) * gv_num_sms();
-    int ks = 1;
-    while (ks < 8 && tiles * (ks + 1) <= slots && prm.kstages / (ks + 1) >= 2) ++ks;
+    const int grid = static_cast<int>(units < slots ? units : slots);
+    prm.uq = prm.units / grid;
+    prm.ur = prm.units % grid;
+
+    const size_t ws_bytes = static_cast<size_t>(2) * grid * Cfg::kTok * Cfg::kRows * sizeof(float);
+    e = workspace_get(ws_bytes, static_cast<size_t>(tiles), &prm.ws, &prm.cnt);
+    if (e != cudaSuccess) return e;
 
     // codes tensor maps (box rows = ROWS) and x map (box rows = 8*NT)
     const uint64_t row_bytes = static_cast<uint64_t>(prm.K) * BITS / 8;
@@ -514,17 +629,12 @@ static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* co
         return cudaErrorInvalidValue;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(ks), static_cast<unsigned>(tiles), 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
     cfg.blockDim = dim3(kGvThreads, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::kSmem);
     cfg.stream = s;
-    cudaLaunchAttribute attrs[2];
+    cudaLaunchAttribute attrs[1];
     int na = 0;
-    attrs[na].id = cudaLaunchAttributeClusterDimension;
-    attrs[na].val.clusterDim.x = static_cast<unsigned>(ks);
-    attrs[na].val.clusterDim.y = 1;
-    attrs[na].val.clusterDim.z = 1;
-    ++na;
     if (pdl_enabled()) {
         attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attrs[na].val.programmaticStreamSerializationAllowed = 1;
@@ -538,22 +648,10 @@ static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* co
 template <int BITS, bool SSC>
 static cudaError_t gv_dispatch_ssc(GvParams& prm, const void* x, const void* const* codes, int nmat,
                                    cudaStream_t s) {
-    // 8 tokens per n-tile; two m-tiles per warp (x fragments and the bias
-    // term reused twice) when N leaves enough row tiles for the SMs.
-    const bool wide = static_cast<int64_t>(nmat) * prm.N >= 8192;
-    if (prm.M <= 8) {
-        if (wide) return gv_launch<BITS, 1, 2, SSC>(prm, x, codes, nmat, s);
-        return gv_launch<BITS, 1, 1, SSC>(prm, x, codes, nmat, s);
-    }
-    if (prm.M <= 16) {
-        if (wide) return gv_launch<BITS, 2, 2, SSC>(prm, x, codes, nmat, s);
-        return gv_launch<BITS, 2, 1, SSC>(prm, x, codes, nmat, s);
-    }
-    if (prm.M <= 24) {
-        if (wide) return gv_launch<BITS, 3, 2, SSC>(prm, x, codes, nmat, s);
-        return gv_launch<BITS, 3, 1, SSC>(prm, x, codes, nmat, s);
-    }
-    if (wide) return gv_launch<BITS, 4, 2, SSC>(prm, x, codes, nmat, s);
+    // 8 tokens per n-tile
+    if (prm.M <= 8) return gv_launch<BITS, 1, 1, SSC>(prm, x, codes, nmat, s);
+    if (prm.M <= 16) return gv_launch<BITS, 2, 1, SSC>(prm, x, codes, nmat, s);
+    if (prm.M <= 24) return gv_launch<BITS, 3, 1, SSC>(prm, x, codes, nmat, s);
     return gv_launch<BITS, 4, 1, SSC>(prm, x, codes, nmat, s);
 }
 

@@ -51,4 +51,13 @@ int* device_status_ptr();
 // Time limit of every bounded on-chip wait, in nanoseconds.
 uint64_t wait_limit_ns();
 
+// Per-device scratch of the decode product: partial-tile slots and per-tile
+// arrival counters (zero between launches).  Grows on demand; growing
+// allocates device memory, so the first call at a new size must not be made
+// while a stream is being captured.
+cudaError_t workspace_get(size_t ws_bytes, size_t n_counters, float** ws, int** cnt);
+
+// Zero the current device's arrival counters (after an aborted launch).
+cudaError_t workspace_reset_counters();
+
 }  // namespace rq

@@ -88,6 +88,7 @@ struct TcCfg {
     static constexpr int kChunks = kCodeBytes / 16;               // 16-byte code chunks per row
     static_assert(kColsNeeded <= 512, "TMEM overflow");
     static_assert(kXStage % 1024 == 0 && kWStage % 1024 == 0, "stage alignment");
+    static_assert(SS % G == 0, "each ring stage must belong to one dequantiser group");
 };
 
 // Read one 16-byte chunk `c` of row `r` from a swizzled codes tile.
@@ -385,13 +386,21 @@ __global__ void __launch_bounds__(TcCfg<BITS, BNT, SS, G>::kThreads, 1)
 // ------------------------------------------------------------- launcher --
 
 // Shared-memory ring depth per configuration: as many stages as fit in about
-// 190 KB (one CTA per SM), at most 32.
+// 190 KB (one CTA per SM), at most 32, and a multiple of the dequantiser group
+// count.  The multiple matters for correctness: k-block i uses stage i % SS
+// and group i % G, so with G | SS every stage belongs to one group, which
+// waits on that stage's barrier round after round.  Otherwise a group could
+// wait for round r+1 of a stage while round r is still in flight, and the
+// parity wait would report the earlier phase as complete.
 constexpr int ring_stages(int bits, int bnt) {
-    return (190 * 1024) / (bnt * 128 + kRows * kKB * bits / 8) > 32
-               ? 32
-               : (190 * 1024) / (bnt * 128 + kRows * kKB * bits / 8);
+    return ((190 * 1024) / (bnt * 128 + kRows * kKB * bits / 8) > 32
+                ? 32
+                : (190 * 1024) / (bnt * 128 + kRows * kKB * bits / 8)) /
+           4 * 4;
 }
 constexpr int kGroups = 4;
+static_assert(ring_stages(4, 256) % kGroups == 0 && ring_stages(8, 256) >= kGroups,
+              "ring depth must be a positive multiple of the group count");
 
 struct TcChoice {
     int bnt;      // tokens per tile (MMA N)
