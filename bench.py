@@ -473,7 +473,7 @@ def main():
             "per_M": per_m,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": None,
-                         "kernel": "tc_wq_kernel (decode: fused RKV + O + key + value)",
+                         "kernel": "gemv_wq_kernel (decode: fused RKV + O + key + value, all M)",
                          "bytes_per_launch": bytes_per_step / launches_per_step,
                          "us_per_launch": ms_per_step * 1e3 / launches_per_step,
                          "peak_kind": peak_kind + " copy bandwidth"},
