@@ -124,6 +124,38 @@ rq_status rq_gemm_wq(const uint16_t *x, int64_t M, int64_t K, const void *codes,
                      rq_stream_t stream);
 
 /*
+ * rq_gemv_wq_noalloc -- rq_gemv_wq for callers that cannot have a library
+ * allocate device memory.  (The pages describe no such variant; it exists for
+ * this library's users.)
+ *
+ * Who needs it: code that records a CUDA graph (allocation is not a stream
+ * operation, so while a stream is being captured it is refused or not
+ * recorded), serving runtimes that reserve the device memory up front for
+ * weights and caches and account for every byte, and hot loops that cannot
+ * afford the implicit device synchronisation of cudaMalloc / cudaFree.
+ * rq_gemv_wq splits each product over all SMs; rows shared by several blocks
+ * leave partial sums in scratch that rq_gemv_wq allocates on first use.  This
+ * call keeps that scratch in a fixed array inside the library instead --
+ * 5 MiB of partial sums plus 16384 per-tile counters (64 KiB), present on
+ * every GPU that loads the library until the process exits -- and calls no
+ * allocator.
+ *
+ * Same arguments, result and rules as rq_gemv_wq (1 <= M <= 32; y fully
+ * overwritten).  Limits: N <= 16384 * 128 rows, and the partial sums of one
+ * launch must fit the fixed array (true for every M on a 148-SM B200);
+ * otherwise RQ_ERR_SHAPE is returned and nothing is launched.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current) -- make it before any stream capture.
+ * Each call clears the counters it uses (an asynchronous memset on `stream`)
+ * and then launches the product.  All calls share the one array: calls that
+ * overlap on the GPU (different streams, or several devices' calls mixed
+ * without ordering) race with each other and give wrong results.
+ */
+rq_status rq_gemv_wq_noalloc(const uint16_t *x, int64_t M, int64_t K, const void *codes,
+                             const uint16_t *scales, int64_t N, int bits, float *y,
+                             rq_stream_t stream);
+
+/*
  * rq_set_pdl -- opt in (enable != 0) or out of programmatic dependent launch
  * for the product kernels launched afterwards by this process.  With it on, a
  * product kernel may start while the previous kernel of the stream is still

@@ -1,0 +1,71 @@
+"""rq_gemv_wq_noalloc: the decode product for callers that cannot have the
+library allocate device memory (graph capture, pre-reserved memory budgets,
+no implicit synchronisation); its scratch is a fixed array inside librq.
+
+Checked against rq_gemv_wq through the C ABI, within the products' parity
+tolerance (|dy| <= 2e-3 * sum_k |x||w_hat|), on two calls in a row -- the
+second call finds the first call's leftovers in the shared array.  Kept in a
+file that runs last, so a failure here comes after every other test has run.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from weight_only_quantized_g64_b200 import build as rq_build
+from weight_only_quantized_g64_b200 import rq, synth
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    rq_build.build()
+    rq.lib()
+    yield
+
+
+def _oracle(x, codes, scales, bits):
+    """(y, sum_k |x||w_hat|) per output, from the oracle on the host."""
+    return oracle.matmul(x.cpu().numpy(), codes.cpu().numpy(),
+                         scales.cpu().numpy().view(np.uint16), bits)
+
+
+@pytest.mark.parametrize("N,K,M,bits", [(4096, 4096, 1, 4), (2048, 8192, 8, 4),
+                                        (300, 640, 17, 4), (2560, 2560, 32, 8),
+                                        (129, 128, 3, 8), (4096, 2048, 32, 4)])
+def test_noalloc_matches_gemv_two_calls(N, K, M, bits):
+    W = synth.weights(N, K, seed=71 + N + M, device="cuda")
+    codes, scales = rq.quantize_g64(W, bits)
+    x = synth.activations(M, K, seed=71 + M, device="cuda")
+    y_ref = rq.gemv_wq(x, codes, scales, N, bits)
+    y1 = torch.full((M, N), float("nan"), device="cuda")
+    y2 = torch.full((M, N), float("nan"), device="cuda")
+    L = rq.lib()
+    s = torch.cuda.current_stream().cuda_stream
+    for y in (y1, y2):
+        st = L.rq_gemv_wq_noalloc(x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(), N,
+                                  bits, y.data_ptr(), s)
+        assert st == rq.OK, rq.STATUS[st]
+    torch.cuda.synchronize()
+    y_or, bound = _oracle(x, codes, scales, bits)
+    ref = y_ref.cpu().numpy().astype(np.float64)
+    for y in (y1, y2):
+        yy = y.cpu().numpy().astype(np.float64)
+        d = np.abs(yy - ref)
+        assert np.all(d <= TOL * bound), f"vs rq_gemv_wq: max diff {d.max():.3e}"
+        d = np.abs(yy - y_or)
+        assert np.all(d <= TOL * bound), f"vs oracle: max diff {d.max():.3e}"
+    assert rq.read_device_status() == rq.OK
+
+
+def test_noalloc_rejects_beyond_its_scratch():
+    """More rows than the fixed counters cover: refused, nothing launched."""
+    N = 16384 * 128 + 1
+    K = 64
+    fake = 1 << 20     # aligned, never dereferenced: the size check comes first
+    L = rq.lib()
+    assert L.rq_gemv_wq_noalloc(fake, 1, K, fake, fake, N, 4, fake, None) == rq.ERR_SHAPE
+    assert L.rq_gemv_wq_noalloc(fake, 33, K, fake, fake, 128, 4, fake, None) == rq.ERR_SHAPE

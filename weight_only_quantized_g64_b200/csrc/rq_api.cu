@@ -144,6 +144,8 @@ using namespace rq;
 
 static thread_local std::string t_last_cuda_error;
 
+void rq::record_cuda_error(cudaError_t e) { t_last_cuda_error = cudaGetErrorString(e); }
+
 static rq_status cuda_fail(cudaError_t e) {
     t_last_cuda_error = cudaGetErrorString(e);
     return RQ_ERR_CUDA;

@@ -583,7 +583,7 @@ static int gv_num_sms() {
 
 template <int BITS, int NT, int MT, bool SSC>
 static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* codes, int nmat,
-                             cudaStream_t s) {
+                             cudaStream_t s, const GemvScratch* scratch) {
     using Cfg = GvCfg<BITS, NT, MT, SSC>;
     auto kern = gemv_wq_kernel<BITS, NT, MT, SSC>;
     static int resident[64] = {};   // CTAs per SM, per device (0 = not yet set up)
@@ -612,8 +612,17 @@ static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* co
     prm.ur = prm.units % grid;
 
     const size_t ws_bytes = static_cast<size_t>(2) * grid * Cfg::kTok * Cfg::kRows * sizeof(float);
-    e = workspace_get(ws_bytes, static_cast<size_t>(tiles), &prm.ws, &prm.cnt);
-    if (e != cudaSuccess) return e;
+    if (scratch == nullptr) {
+        e = workspace_get(ws_bytes, static_cast<size_t>(tiles), &prm.ws, &prm.cnt);
+        if (e != cudaSuccess) return e;
+    } else {
+        if (ws_bytes > scratch->ws_bytes || static_cast<size_t>(tiles) > scratch->n_cnt) {
+            if (scratch->too_large) *scratch->too_large = true;
+            return cudaErrorInvalidValue;
+        }
+        prm.ws = scratch->ws;
+        prm.cnt = scratch->cnt;
+    }
 
     // codes tensor maps (box rows = ROWS) and x map (box rows = 8*NT)
     const uint64_t row_bytes = static_cast<uint64_t>(prm.K) * BITS / 8;
@@ -647,24 +656,24 @@ static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* co
 
 template <int BITS, bool SSC>
 static cudaError_t gv_dispatch_ssc(GvParams& prm, const void* x, const void* const* codes, int nmat,
-                                   cudaStream_t s) {
+                                   cudaStream_t s, const GemvScratch* sc) {
     // 8 tokens per n-tile
-    if (prm.M <= 8) return gv_launch<BITS, 1, 1, SSC>(prm, x, codes, nmat, s);
-    if (prm.M <= 16) return gv_launch<BITS, 2, 1, SSC>(prm, x, codes, nmat, s);
-    if (prm.M <= 24) return gv_launch<BITS, 3, 1, SSC>(prm, x, codes, nmat, s);
-    return gv_launch<BITS, 4, 1, SSC>(prm, x, codes, nmat, s);
+    if (prm.M <= 8) return gv_launch<BITS, 1, 1, SSC>(prm, x, codes, nmat, s, sc);
+    if (prm.M <= 16) return gv_launch<BITS, 2, 1, SSC>(prm, x, codes, nmat, s, sc);
+    if (prm.M <= 24) return gv_launch<BITS, 3, 1, SSC>(prm, x, codes, nmat, s, sc);
+    return gv_launch<BITS, 4, 1, SSC>(prm, x, codes, nmat, s, sc);
 }
 
 template <int BITS>
 static cudaError_t gv_dispatch(GvParams& prm, const void* x, const void* const* codes, int nmat,
-                               cudaStream_t s) {
+                               cudaStream_t s, const GemvScratch* sc) {
     constexpr int gps = BITS == 4 ? 4 : 2;
-    if (prm.groups % gps == 0) return gv_dispatch_ssc<BITS, true>(prm, x, codes, nmat, s);
-    return gv_dispatch_ssc<BITS, false>(prm, x, codes, nmat, s);
+    if (prm.groups % gps == 0) return gv_dispatch_ssc<BITS, true>(prm, x, codes, nmat, s, sc);
+    return gv_dispatch_ssc<BITS, false>(prm, x, codes, nmat, s, sc);
 }
 
-cudaError_t launch_gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
-                                const WOperand* w, int nmat, cudaStream_t s) {
+static cudaError_t gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
+                                const WOperand* w, int nmat, cudaStream_t s, const GemvScratch* sc) {
     GvParams prm;
     memset(&prm, 0, sizeof(prm));
     prm.M = static_cast<int>(M);
@@ -679,7 +688,19 @@ cudaError_t launch_gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t
         prm.scales[i] = w[i].scales;
         prm.y[i] = w[i].y;
     }
-    return bits == 4 ? gv_dispatch<4>(prm, x, codes, nmat, s) : gv_dispatch<8>(prm, x, codes, nmat, s);
+    return bits == 4 ? gv_dispatch<4>(prm, x, codes, nmat, s, sc)
+                     : gv_dispatch<8>(prm, x, codes, nmat, s, sc);
+}
+
+cudaError_t launch_gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
+                                const WOperand* w, int nmat, cudaStream_t s) {
+    return gemv_product(x, M, K, N, bits, w, nmat, s, nullptr);
+}
+
+cudaError_t launch_gemv_product_scratch(const uint16_t* x, int64_t M, int64_t K, int64_t N,
+                                        int bits, const WOperand* w, int nmat, cudaStream_t s,
+                                        const GemvScratch* scratch) {
+    return gemv_product(x, M, K, N, bits, w, nmat, s, scratch);
 }
 
 }  // namespace rq

@@ -30,9 +30,24 @@ cudaError_t launch_tc_product(const uint16_t* x, int64_t M, int64_t K, int64_t N
                               const WOperand* w, int nmat, cudaStream_t s);
 
 // Decode product (M <= 32): TMA-staged codes, in-register dequantisation,
-// warp-level tensor-core MMA (mma.sync), split-K over a cluster.
+// warp-level tensor-core MMA (mma.sync), stream-K split over the SMs.
 cudaError_t launch_gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
                                 const WOperand* w, int nmat, cudaStream_t s);
+
+// Caller-provided scratch for the decode product instead of the library's
+// workspace: partial-tile slots (ws, ws_bytes) and per-tile counters (cnt,
+// n_cnt, zero between launches).  If a launch would need more, nothing is
+// launched and *too_large is set.
+struct GemvScratch {
+    float* ws;
+    size_t ws_bytes;
+    int* cnt;
+    size_t n_cnt;
+    bool* too_large;
+};
+cudaError_t launch_gemv_product_scratch(const uint16_t* x, int64_t M, int64_t K, int64_t N,
+                                        int bits, const WOperand* w, int nmat, cudaStream_t s,
+                                        const GemvScratch* scratch);
 
 // Bounded-wait self test: a kernel waits on an mbarrier nothing completes.
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s);
@@ -59,5 +74,8 @@ cudaError_t workspace_get(size_t ws_bytes, size_t n_counters, float** ws, int** 
 
 // Zero the current device's arrival counters (after an aborted launch).
 cudaError_t workspace_reset_counters();
+
+// Remember e as this thread's last CUDA error (returned by rq_last_cuda_error).
+void record_cuda_error(cudaError_t e);
 
 }  // namespace rq

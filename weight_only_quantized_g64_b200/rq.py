@@ -55,6 +55,8 @@ def lib():
     L.rq_gemv_wq.restype = i32
     L.rq_gemm_wq.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, vp]
     L.rq_gemm_wq.restype = i32
+    L.rq_gemv_wq_noalloc.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, vp]
+    L.rq_gemv_wq_noalloc.restype = i32
     L.rq_rkv_fused.argtypes = [vp, i64, i64, i64, i32] + [vp] * 9 + [vp]
     L.rq_rkv_fused.restype = i32
     L.rq_set_pdl.argtypes = [i32]
@@ -129,6 +131,17 @@ def gemv_wq(x: torch.Tensor, codes, scales, N: int, bits: int, y=None, stream=No
         y = torch.empty((M, N), dtype=torch.float32, device=x.device)
     _check(lib().rq_gemv_wq(_p(x), M, K, _p(codes), _p(scales), N, bits, _p(y), _stream(stream)),
            "rq_gemv_wq")
+    return y
+
+
+def gemv_wq_noalloc(x: torch.Tensor, codes, scales, N: int, bits: int, y=None, stream=None):
+    """Decode product with the library's fixed scratch array: the library
+    allocates no device memory (y is allocated here only when not given)."""
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _check(lib().rq_gemv_wq_noalloc(_p(x), M, K, _p(codes), _p(scales), N, bits, _p(y),
+                                    _stream(stream)), "rq_gemv_wq_noalloc")
     return y
 
 
