@@ -141,7 +141,7 @@ rq_status rq_gemm_wq(const uint16_t *x, int64_t M, int64_t K, const void *codes,
  * allocator.
  *
  * Same arguments, result and rules as rq_gemv_wq (1 <= M <= 32; y fully
- * overwritten).  Limits: N <= 16384 * 128 rows, and the partial sums of one
+ * overwritten).  Limits: N <= 16384 * 32 rows, and the partial sums of one
  * launch must fit the fixed array (true for every M on a 148-SM B200);
  * otherwise RQ_ERR_SHAPE is returned and nothing is launched.
  * The first call on a device looks up the array's device address (once per

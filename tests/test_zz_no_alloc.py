@@ -63,7 +63,7 @@ def test_noalloc_matches_gemv_two_calls(N, K, M, bits):
 
 def test_noalloc_rejects_beyond_its_scratch():
     """More rows than the fixed counters cover: refused, nothing launched."""
-    N = 16384 * 128 + 1
+    N = 16384 * 32 + 1
     K = 64
     fake = 1 << 20     # aligned, never dereferenced: the size check comes first
     L = rq.lib()

@@ -16,554 +16,473 @@
 // 128 / 64 / 32 weights per cycle per SM for M <= 8 / 16 / 32.  (Both figures
 // measured on this hardware.)
 //
-// Data path (one CTA = 8 consumer warps + 1 TMA producer warp):
-//   codes   TMA 2D tiles [ROWS rows x 128 B] (int4: 256 k, int8: 128 k per
-//           stage), SWIZZLE_128B, into an SS-deep shared-memory ring;
-//   x       TMA 2D tiles [8*NT tokens x 64 k] per group, SWIZZLE_128B, in the
-//           same stage (rows >= M are zero-filled by the TMA);
-//   scales  per thread with 8-byte loads, one stage ahead.
-// A consumer warp owns 16*MT weight rows.  Thread (g = lane/4, t = lane%4)
-// owns, per group of 64 k, the 16 k [16t, 16t+16) of rows g and g+8 of each
-// of its m-tiles: MMA k-slot sigma of step j maps to one of those k, the same
-// map on the A (weights) and B (x) side, so the sum over k is unchanged and
-// every thread's codes and x are contiguous in memory.  Codes become exact
-// fp16 values in registers (bit placement plus one exact fp16 operation:
-// Kim et al., arXiv:2211.10017); the MMA sums x * code for one group in fp32
-// registers; the group's scale is applied in fp32 (acc = fma(partial, s,
-// acc)).  Nothing dequantised is stored.
+// Work decomposition.  A row tile is RBM = 16*MTM consecutive rows of each of
+// the NMAT matrices (NMAT = 3 for the fused R/K/V call, whose matrices share
+// x), i.e. MT = NMAT*MTM MMA m-tiles of 16 rows.  A unit is one row tile times
+// one 128-byte column stage of codes (int4: 256 k = 4 groups; int8: 128 k = 2
+// groups).  The units, tile-major, are cut into equal contiguous runs, one per
+// CTA (stream-K).  Inside a CTA the units are dealt round-robin to the 8
+// warps (unit j of the CTA to warp j % 8): every warp works on all MT m-tiles
+// of its units, so
+// each x fragment it loads serves MT m-tiles, and the warps' partial sums are
+// added in shared memory when the tile ends.  When the CTAs outnumber the
+// tiles' needs the host picks one tile per CTA, and then nothing is reduced
+// across CTAs; otherwise a tile shared by several CTAs is stored as pieces in
+// a global workspace and summed, in a fixed CTA order, by whichever
+// contributor arrives last (an atomic counter per tile), so results stay
+// deterministic.
 //
-// Work split (stream-K): the work is a list of units (one 128-row tile x one
-// k-stage, tile-major) cut into equal contiguous runs, one per resident CTA,
-// so every SM streams the same number of bytes whatever the shape.  A CTA
-// stores a tile it covers whole directly; a tile shared by several CTAs is
-// stored as pieces in a global workspace and summed, in a fixed CTA order, by
-// whichever contributor arrives last (an atomic counter per tile), so results
-// are deterministic.
+// Data path (one CTA = 8 warps, no dedicated producer):
+//   codes   TMA 2D tiles [RBM rows x 128 B] per matrix, SWIZZLE_128B, into a
+//           ring of SS stages (SS = 8, 16 or 32); the first SS units are
+//           fetched by warp 0 before the kernel waits on the previous grid
+//           (codes and scales do not depend on it);
+//   scales  cp.async into a parallel ring, completing on the same barrier;
+//   x       per warp: cp.async of the M x 256 k (int4; 128 k for int8) slice
+//           of its unit into a buffer of its own, one unit ahead (two
+//           buffers when shared memory allows), after the wait; token rows
+//           >= M are never read (their B fragments are zero).
+// A warp that has read a stage refills that slot itself with the unit SS
+// places ahead, so no slot needs an "empty" barrier and no warp waits to
+// issue; 8 warps leave room for two CTAs per SM at up to 128 registers.
+// Thread (g = lane/4, t = lane%4) owns, per group of 64 k, the 16 k
+// [16t, 16t+16) of rows g and g+8 of each m-tile: MMA k-slot sigma of step j
+// maps to one of those k, the same map on the A (weights) and B (x) side, so
+// the sum over k is unchanged and every thread's codes and x are contiguous in
+// memory.  Codes become exact fp16 values in registers (bit placement plus
+// one exact fp16 operation: Kim et al., arXiv:2211.10017); the MMA sums
+// x * code for one group in fp32 registers; the group's scale is applied in
+// fp32 (acc = fma(partial, s, acc)).  Nothing dequantised is stored.
 #include "rq_internal.h"
 #include "rq_ptx.cuh"
+#include "rq_gemv_unit.cuh"
 
 namespace rq {
 
 struct GvParams {
-    CUtensorMap tm_x;     // x [M, K] fp16: dims {K, M}, box {64, 8*NT}, SWIZZLE_128B
-    CUtensorMap tm_w[3];  // codes [N, K*bits/8] u8: box {128, ROWS}, SWIZZLE_128B
+    CUtensorMap tm_w[3];  // codes [N, K*bits/8] u8; ks == KS: 3D {128 B, N rows, stages}, box
+                          // {128, RBM, KS}; ks == 1: 2D {row bytes, N}, box {128, RBM}; SWIZZLE_128B
+    CUtensorMap tm_s[3];  // scales [N, K/64] fp16: box {SROW groups, RBM}, no swizzle (when ssc)
+    const uint16_t* x;    // [M, K] fp16
     const uint16_t* scales[3];
     float* y[3];
     int M, N, K;
-    int n_tiles;          // row tiles per matrix
-    int kstages;          // k stages per row tile (ceil(K / k-per-stage))
     int groups;           // K / 64
-    int units;            // work units: nmat * n_tiles * kstages (one tile x one stage each)
-    int uq, ur;           // units / gridDim.x and units % gridDim.x: CTA c owns
+    int tiles;            // row tiles (RBM rows of every matrix)
+    int kstages;          // 128-byte code stages per row: ceil(K * bits / 8 / 128)
+    int units;            // tiles * kstages
+    int chunk;            // units are dealt in chunks: kstages (whole tiles) or 1 (stream-K)
+    int uq, ur;           // chunks / gridDim.x and chunks % gridDim.x: CTA c owns chunks
                           // [c*uq + min(c, ur), (c+1)*uq + min(c+1, ur))
-    float* ws;            // partial-tile slots: [2 * gridDim.x][8*NT tokens * ROWS rows] fp32
+    int ks;               // stages per load group (8, 4 when shared memory is short, or 1 when
+                          // rows are not whole stages); warps w < ks compute
+    int sg;               // ring depth in load groups (2..8)
+    int s_ring_off;       // offset of the scale ring (after the code ring)
+    int x_off;            // offset of the per-warp x buffers
+    int x_row;            // bytes per token row of an x buffer
+    int x_nbuf;           // x buffers per warp (1 or 2)
+    int red_off;          // offset of the reduction buffers
+    int red_nbuf;         // reduction buffers (1 or 2)
+    int bar_off;          // offset of the barriers
+    int ssc;              // scales staged by TMA with the codes (rows a multiple of 16 bytes)
+    float* ws;            // partial-tile slots: [2 * gridDim.x][M][RB] fp32
     int* cnt;             // per-tile arrival counters, zero between launches
     int* status;
     uint64_t timeout_ns;
 };
 
-constexpr int kGvConsumers = 8;
-constexpr int kGvThreads = (kGvConsumers + 1) * 32;
+constexpr int kGvConsumers = 8;                         // warps that multiply
+constexpr int kGvProducer = kGvConsumers;               // warp that refills the ring
+constexpr int kGvReducer = kGvConsumers + 1;            // warp that reduces and stores
+constexpr int kGvThreads = (kGvConsumers + 2) * 32;
+constexpr int kGvKS = kGvConsumers;                     // k-stages per load group (one per warp)
+constexpr int kGvMaxSG = 8;                             // ring depth limit, in load groups
 
-// BITS: 4 or 8.  NT: 8-token n-tiles (M <= 8 NT).  MT: 16-row m-tiles per
-// consumer warp.  SSC: scales staged in shared memory by the producer warp (needs the
-// stage's groups to be all valid or all past the end: G % groups-per-stage
-// == 0); otherwise consumers load them from global memory.
-template <int BITS, int NT, int MT, bool SSC>
+// BITS: 4 or 8.  NMAT: matrices sharing x (1, or 3 for fused R/K/V).  MTM:
+// 16-row m-tiles per matrix in a row tile.  NT: 8-token n-tiles (M <= 8 NT).
+template <int BITS, int NMAT, int MTM, int NT>
 struct GvCfg {
-    static constexpr int kRows = kGvConsumers * 16 * MT;      // weight rows per CTA
-    static constexpr int kKPS = BITS == 4 ? 256 : 128;        // k per stage (128 code bytes)
-    static constexpr int kGPS = kKPS / 64;                    // groups per stage
-    static constexpr int kTok = 8 * NT;                       // tokens per CTA
-    static constexpr int kWStage = kRows * 128;
-    static constexpr int kXStage = kGPS * kTok * 128;
-    static constexpr int kSStage = SSC ? ((kRows * kGPS * 2 + 1023) / 1024) * 1024 : 0;
-    static constexpr int kStage = kWStage + kXStage + kSStage;
-    static constexpr int kBudget = (NT == 1 && MT == 1 ? 100 : 196) * 1024;   // two CTAs per SM when NT == MT == 1
-    static constexpr int kSS = kBudget / kStage > 8 ? 8 : (kBudget / kStage < 2 ? 2 : kBudget / kStage);
-    static constexpr int kRing = kSS * kStage;
-    static constexpr int kRed = kTok * kRows * 4;
-    static constexpr int kData = kRing > kRed ? kRing : kRed;
-    static constexpr int kSmem = 1024 + kData + 256;
-    static_assert(kWStage % 1024 == 0 && kXStage % 1024 == 0 && kSStage % 1024 == 0,
-                  "stage alignment");
+    static constexpr int kMT = NMAT * MTM;                   // m-tiles per row tile
+    static constexpr int kRBM = 16 * MTM;                    // rows per matrix
+    static constexpr int kRB = 16 * kMT;                     // rows per row tile
+    static constexpr int kKPS = BITS == 4 ? 256 : 128;       // k per stage (128 code bytes)
+    static constexpr int kGPS = kKPS / 64;                   // groups per stage
+    static constexpr int kTok = 8 * NT;
+    // a load group: ks stages of a row tile, per matrix [ks][RBM rows][128 B]
+    static constexpr int kCStage = kRBM * 128;               // code bytes per matrix and stage
+    // scales: per matrix [RBM rows][SROW] fp16, SROW = the group's KS*GPS
+    // groups plus 8 of slack, so the box can start at a 16-byte boundary
+    static constexpr int kSRow = kGvKS * kGPS + 8;
+    static constexpr int kSMat = kRBM * kSRow * 2;
+    static constexpr int kSGroup = NMAT * kSMat;
+    static constexpr int kXRow = kKPS * 2 + 16;              // x bytes per token row (+16: banks)
+    static constexpr int kRedStride = kRB + 4;               // floats per token row (bank spread)
+    static constexpr int kRedTok = kTok < 16 ? kTok : 16;    // tokens per reduction round
+    static constexpr int kRedWarp = kRedTok * kRedStride;    // floats per warp
+    static constexpr int kRedBuf = kGvConsumers * kRedWarp;  // floats per reduction buffer
+    static_assert(kCStage % 1024 == 0, "group alignment");
+    static_assert((kSRow * 2) % 16 == 0, "scale rows must be 16-byte multiples");
+    static_assert(kSMat % 128 == 0, "TMA destinations must be 128-byte aligned");
 };
 
-__device__ __forceinline__ uint32_t lop3_bmux(uint32_t a, uint32_t b, uint32_t c) {
-    // b ? (a ^ c) : c, bitwise
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
+// Barriers and flags after the buffers.
+struct GvBars {
+    uint64_t full[kGvMaxSG];   // ring slot holds its group's codes and scales
+    uint64_t empty[kGvMaxSG];  // every consumer warp is done with the slot
+    uint64_t red_full[2];      // every warp has deposited its partial sums
+    uint64_t red_free[2];      // the reducing warp has read the buffer
+    int issued_hi[kGvMaxSG];   // last group issued into each slot
+    int abort;
+};
 
-__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
-__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
-
-// Code unpacking to EXACT fp16 codes, without integer->float conversions:
-// the biased code is placed in the mantissa of an fp16 in [1024, 2048) and
-// the bias is removed with one exact fp16 operation (the bit placement of
-// Kim et al., "Who Says Elephants Can't Run?", arXiv:2211.10017).
-
-// int4, permuted order: one code word (positions 0..7 of a row, position 2i
-// in the low nibble of byte i) -> pairs (p0,p4), (p1,p5), (p2,p6), (p3,p7).
-// 9 instructions per 8 codes; x is permuted to the same order.
-__device__ __forceinline__ void i4_word_to_pairs_perm(uint32_t w, uint32_t (&P)[4]) {
-    const __half2 bias_lo = u32_as_h2(0x64086408u);                      // 1032, 1032
-    const __half2 inv16 = u32_as_h2(0x2C002C00u);                        // 1/16
-    const __half2 bias_hi = u32_as_h2(0xD480D480u);                      // -72
-    const uint32_t w8 = w >> 8;
-    // low nibbles of bytes 0 and 2 -> 1024 + (nibble ^ 8); high nibbles -> 1024 + 16*(nibble ^ 8)
-    P[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_bmux(w, 0x000F000Fu, 0x64086408u)), bias_lo));
-    P[1] = h2_as_u32(__hfma2(u32_as_h2(lop3_bmux(w, 0x00F000F0u, 0x64806480u)), inv16, bias_hi));
-    P[2] = h2_as_u32(__hsub2(u32_as_h2(lop3_bmux(w8, 0x000F000Fu, 0x64086408u)), bias_lo));
-    P[3] = h2_as_u32(__hfma2(u32_as_h2(lop3_bmux(w8, 0x00F000F0u, 0x64806480u)), inv16, bias_hi));
-}
-
-// int4, natural order: one code word -> pairs (p0,p1), (p2,p3), (p4,p5), (p6,p7)
-// (the two nibbles of each byte).  13 instructions per 8 codes; x is used as is.
-__device__ __forceinline__ void i4_word_to_pairs_nat(uint32_t w, uint32_t (&P)[4]) {
-    const __half2 bias = u32_as_h2(0x64086408u);                         // 1032, 1032
-    const uint32_t w4 = w >> 4;   // byte b of w4 holds the high nibble of byte b of w in its low bits
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-        const uint32_t v = __byte_perm(w, w4, static_cast<uint32_t>(b) | ((4u + b) << 8));
-        P[b] = h2_as_u32(__hsub2(u32_as_h2(lop3_bmux(v, 0x000F000Fu, 0x64086408u)), bias));
-    }
-}
-
-// int8: one 32-bit word (positions 0..3) -> exact pairs (p0, p1), (p2, p3).
-__device__ __forceinline__ void i8_word_to_pairs(uint32_t w, uint32_t (&Q)[2]) {
-    const __half2 bias = u32_as_h2(0x64806480u);                         // 1152 = 1024 + 128
-    w ^= 0x80808080u;
-    Q[0] = h2_as_u32(__hsub2(u32_as_h2(__byte_perm(w, 0x64646464u, 0x5140u)), bias));
-    Q[1] = h2_as_u32(__hsub2(u32_as_h2(__byte_perm(w, 0x64646464u, 0x5342u)), bias));
-}
-
-// Not volatile: a pure function of its operands, so the compiler may
-// interleave independent accumulation chains (different groups / n-tiles).
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1, bool zero_c) {
-    if (zero_c) {
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-            "{%8,%9}, {%10,%10,%10,%10};"
-            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
-    } else {
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-            "{%8,%9}, {%0,%1,%2,%3};"
-            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-    }
-}
-
-// Physical row (within a 16-row m-tile) of MMA row g (0..7); MMA row g + 8 is
-// that plus 8.  Chosen so that the rows read together by one shared-memory
-// wavefront land on distinct 16-byte chunks of the 128-byte swizzle:
-// int4 (8-byte reads, half-warps = g 0..3 / 4..7): rows 0,2,4,6 / 1,3,5,7;
-// int8 (16-byte reads, quarter-warps = g pairs): rows 0,4 / 1,5 / 2,6 / 3,7.
-template <int BITS>
-__device__ __forceinline__ int phys_row(int g) {
-    if constexpr (BITS == 4) return g < 4 ? 2 * g : 2 * (g - 4) + 1;
-    else return (g >> 1) + 4 * (g & 1);
-}
-
-// First work unit of CTA c: the first ur CTAs take uq + 1 units, the rest uq.
+// First work chunk of CTA c: the first ur CTAs take uq + 1 chunks, the rest uq.
 __device__ __forceinline__ int range_begin(int c, int uq, int ur) {
     return c * uq + (c < ur ? c : ur);
 }
 
-// The CTA whose unit range holds unit u.
+// The CTA whose unit range holds unit u (stream-K: chunks of one unit).
 __device__ __forceinline__ int range_owner(int u, int uq, int ur) {
     const int big = ur * (uq + 1);
     return u < big ? u / (uq + 1) : ur + (u - big) / uq;
 }
 
-// Named barrier over the eight consumer warps (the producer warp is not in it).
-__device__ __forceinline__ void consumers_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kGvConsumers * 32) : "memory");
-}
+// Walks a CTA's units as load groups: up to KS consecutive stages of one row
+// tile, never past the tile or the CTA's range.
+struct GvWalk {
+    int tile, st, left, ks;
+    __device__ __forceinline__ int next(int S, int& g_tile, int& g_st) {   // returns the group's units
+        int n = S - st;
+        if (n > ks) n = ks;
+        if (n > left) n = left;
+        g_tile = tile;
+        g_st = st;
+        st += n;
+        left -= n;
+        if (st == S) {
+            st = 0;
+            ++tile;
+        }
+        return n;
+    }
+};
 
-template <int BITS, int NT, int MT, bool SSC>
-__global__ void __launch_bounds__(kGvThreads, (NT == 1 && MT == 1) ? 2 : 1)
-    gemv_wq_kernel(const __grid_constant__ GvParams p) {
-    using Cfg = GvCfg<BITS, NT, MT, SSC>;
-    constexpr int SS = Cfg::kSS;
-    constexpr int ROWS = Cfg::kRows;
+template <int BITS, int NMAT, int MTM, int NT>
+__global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_constant__ GvParams p) {
+    using Cfg = GvCfg<BITS, NMAT, MTM, NT>;
+    constexpr int MT = Cfg::kMT;
+    constexpr int RBM = Cfg::kRBM;
+    constexpr int RB = Cfg::kRB;
     constexpr int GPS = Cfg::kGPS;
-    constexpr int TOK = Cfg::kTok;
+    constexpr int KPS = Cfg::kKPS;
+    constexpr int RS = Cfg::kRedStride;
+    constexpr int NW = kGvConsumers;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    uint8_t* ring = smem;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kData);
-    uint64_t* empty = full + SS;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + SS);
-    volatile int* last_flag = abort_flag + 1;
+    const int SG = p.sg;
+    const int cmat = p.ks * Cfg::kCStage;                   // code bytes per matrix and group
+    const int cgroup = NMAT * cmat;                         // code bytes per group
+    uint8_t* cring = smem;                                  // [SG][NMAT][ks][RBM][128 B], swizzled
+    uint8_t* sring = smem + p.s_ring_off;                   // [SG][NMAT][RBM][SROW] fp16
+    float* red = reinterpret_cast<float*>(smem + p.red_off);   // [red_nbuf][NW][kRedTok][RS]
+    GvBars* bars = reinterpret_cast<GvBars*>(smem + p.bar_off);
+    volatile int* abort_flag = &bars->abort;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int G = static_cast<int>(gridDim.x);
     const int cta = static_cast<int>(blockIdx.x);
     const int S = p.kstages;
-    const int u0 = range_begin(cta, p.uq, p.ur);
-    const int nu = p.uq + (cta < p.ur ? 1 : 0);
-    // position of the first unit: tile (matrix, row tile) and k-stage
+    const int M = p.M;
+    const int u0 = range_begin(cta, p.uq, p.ur) * p.chunk;
+    const int nu = (p.uq + (cta < p.ur ? 1 : 0)) * p.chunk;
     const int tile0 = u0 / S;
     const int st0 = u0 - tile0 * S;
+    const int nbuf = p.x_nbuf;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < SS; ++s) {
-            mbar_init(&full[s], SSC ? 1 + 32 : 1);
-            mbar_init(&empty[s], kGvConsumers);
+        for (int s = 0; s < SG; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], NW);
+            bars->issued_hi[s] = -1;
         }
-        *abort_flag = 0;
-        *last_flag = 0;
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->red_full[b], NW);
+            mbar_init(&bars->red_free[b], 1);
+        }
+        bars->abort = 0;
         fence_mbar_init();
-    }
-    if (warp == kGvConsumers && lane == 0) {
-        tma_prefetch_desc(&p.tm_x);
-        for (int m = 0; m < 3; ++m)
-            if (p.y[m] != nullptr) tma_prefetch_desc(&p.tm_w[m]);
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+            tma_prefetch_desc(&p.tm_w[m]);
+            if (p.ssc) tma_prefetch_desc(&p.tm_s[m]);
+        }
     }
     __syncthreads();
     pdl_launch_dependents();
 
-    if (warp == kGvConsumers) {
-        // ---------------------------------------------- producer warp --
-        // lane 0 issues the TMA copies; with SSC every lane also copies the
-        // unit's scales (rows lane, lane+32, ...) with cp.async completing on
-        // the same barrier.
-        const bool leader = lane == 0;
-        const uint64_t pol_w = l2_policy_evict_first();
-        const uint64_t pol_x = l2_policy_evict_last();
-        // position of the next unit to issue, advanced one unit at a time
-        int c_st = st0, c_tm = tile0 % p.n_tiles, c_mat = tile0 / p.n_tiles;
-        auto unit_codes = [&](int s) {
-            const int st = c_st;
-            const int mat = c_mat;
-            const int n0 = c_tm * ROWS;
-            if (leader) {
-                mbar_arrive_expect_tx(&full[s], Cfg::kWStage + Cfg::kXStage);
-                tma_load_2d(ring + s * Cfg::kStage, &p.tm_w[mat], &full[s], st * 128, n0, pol_w);
-            }
-            if constexpr (SSC) {
-                uint8_t* dst = ring + s * Cfg::kStage + Cfg::kWStage + Cfg::kXStage;
-                const int grp = st * GPS;
-                const uint16_t* sbase = p.scales[mat];
+    if (warp == kGvProducer) {
+        // ================================================= producer warp ==
+        // Fills the ring, one load group per slot: the first SG groups
+        // before waiting on the previous grid (codes and scales do not depend
+        // on it), then group i as soon as every consumer warp is done with
+        // group i - SG, which used the same slot.
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_first();
+            GvWalk wk{tile0, st0, nu, p.ks};
+            int slot = 0;
+            for (int i = 0; wk.left > 0; ++i) {
+                if (i >= SG && !mbar_wait(&bars->empty[slot], static_cast<uint32_t>(i / SG - 1) & 1,
+                                          abort_flag, p.timeout_ns, p.status))
+                    break;
+                int g_tile, g_st;
+                wk.next(S, g_tile, g_st);
+                bars->issued_hi[slot] = i;
+                mbar_arrive_expect_tx(&bars->full[slot],
+                                      static_cast<uint32_t>(cgroup + (p.ssc ? Cfg::kSGroup : 0)));
+                uint8_t* cdst = cring + slot * cgroup;
+                uint8_t* sdst = sring + slot * Cfg::kSGroup;
+                const int sx = (g_st * GPS) & ~7;   // 16-byte aligned first scale group
 #pragma unroll
-                for (int rr = lane; rr < ROWS; rr += 32) {
-                    const int n = n0 + rr;
-                    const bool ok = n < p.N && grp < p.groups;
-                    const uint16_t* src = ok ? sbase + static_cast<int64_t>(n) * p.groups + grp : sbase;
-                    if constexpr (GPS == 4) cp_async_8(dst + rr * 8, src, ok ? 8u : 0u);
-                    else cp_async_4(dst + rr * 4, src, ok ? 4u : 0u);
+                for (int m = 0; m < NMAT; ++m) {
+                    if (p.ks > 1)
+                        tma_load_3d(cdst + m * cmat, &p.tm_w[m], &bars->full[slot], 0,
+                                    g_tile * RBM, g_st, pol_w);
+                    else
+                        tma_load_2d(cdst + m * cmat, &p.tm_w[m], &bars->full[slot], g_st * 128,
+                                    g_tile * RBM, pol_w);
+                    if (p.ssc)
+                        tma_load_2d(sdst + m * Cfg::kSMat, &p.tm_s[m], &bars->full[slot], sx,
+                                    g_tile * RBM, pol_w);
                 }
-                cp_async_arrive_noinc(&full[s]);
-            }
-        };
-        auto advance = [&]() {
-            if (++c_st == S) {
-                c_st = 0;
-                if (++c_tm == p.n_tiles) {
-                    c_tm = 0;
-                    ++c_mat;
-                }
-            }
-        };
-        auto unit_x = [&](int st, int s) {
-#pragma unroll
-            for (int q = 0; q < GPS; ++q)
-                tma_load_2d(ring + s * Cfg::kStage + Cfg::kWStage + q * TOK * 128, &p.tm_x,
-                            &full[s], st * Cfg::kKPS + q * 64, 0, pol_x);
-        };
-        const int pre = nu < SS ? nu : SS;
-        // Weights do not depend on the previous kernel: fetch them first.
-        for (int i = 0; i < pre; ++i) {
-            unit_codes(i);
-            advance();
-        }
-        if (leader) {
-            pdl_wait();   // x may be produced by the previous kernel
-            int st = st0;
-            for (int i = 0; i < pre; ++i) {
-                unit_x(st, i);
-                if (++st == S) st = 0;
+                if (++slot == SG) slot = 0;
             }
         }
-        int issued = pre;
-        for (int i = SS; i < nu; ++i) {
-            const int s = i % SS;
-            if (!mbar_wait(&empty[s], static_cast<uint32_t>(i / SS - 1) & 1, abort_flag,
-                           p.timeout_ns, p.status))
-                break;
-            const int st = c_st;
-            unit_codes(s);
-            if (leader) unit_x(st, s);
-            advance();
-            issued = i + 1;
-        }
-        // Wait (bounded, regardless of abort) until every copy this warp
-        // issued has landed, so none is in flight when the CTA exits.
-        int dummy_abort = 0;
-        const int first = issued > SS ? issued - SS : 0;
-        for (int i = first; i < issued; ++i)
-            mbar_wait(&full[i % SS], static_cast<uint32_t>(i / SS) & 1, &dummy_abort,
-                      p.timeout_ns, p.status);
         __syncwarp();
+        pdl_wait();
+    } else if (warp == kGvReducer) {
+        // ================================================ reduction warp ==
+        // Walks the same row tiles as the compute warps; for every round it
+        // adds the 8 deposits in warp order (deterministic) and stores the
+        // tile, or this CTA's piece of a tile that several CTAs share.  It
+        // issues no loads of its own, so its fences are cheap.
+        pdl_wait();   // (its stores follow the compute warps' waits anyway)
+        const int rounds = (M + Cfg::kRedTok - 1) / Cfg::kRedTok;
+        const int nbl = p.red_nbuf - 1;                 // log2 of the buffer count (0 or 1)
+        int j = 0, tile = tile0, st_seg = st0;
+        for (int k = 0; j < nu; ++k) {
+            const int len = (S - st_seg) < (nu - j) ? (S - st_seg) : (nu - j);
+            const bool whole = st_seg == 0 && len == S;
+            const int n_out = M * RB;
+            const int slotw = 2 * cta + (j == 0 ? 0 : 1);   // workspace slot of a shared tile
+            bool ok_all = true;
+            for (int pi = 0; pi < rounds; ++pi) {
+                const int r = k * rounds + pi;
+                const int b = r & nbl;
+                const float* rb = red + b * Cfg::kRedBuf;
+                const bool ok = mbar_wait(&bars->red_full[b], static_cast<uint32_t>(r >> nbl) & 1,
+                                          abort_flag, p.timeout_ns, p.status);
+                ok_all = ok_all && ok;
+                const int tok0 = pi * Cfg::kRedTok;
+                const int ntok = (M - tok0) < Cfg::kRedTok ? (M - tok0) : Cfg::kRedTok;
+                if (ok && *abort_flag == 0) {
+                    for (int o = lane; o < ntok * RB; o += 32) {
+                        const int tl = o / RB;
+                        const int rho = o - tl * RB;
+                        float v = 0.0f;
+#pragma unroll
+                        for (int w = 0; w < NW; ++w) v += rb[w * Cfg::kRedWarp + tl * RS + rho];
+                        const int tok = tok0 + tl;
+                        if (whole) {
+                            const int m = rho / RBM;
+                            const int n = tile * RBM + (rho - m * RBM);
+                            if (n < p.N) p.y[m][static_cast<int64_t>(tok) * p.N + n] = v;
+                        } else {
+                            // slot 2c for the CTA's first segment, 2c+1 for its last
+                            p.ws[static_cast<int64_t>(slotw) * n_out + tok * RB + rho] = v;
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->red_free[b]);
+            }
+            if (!whole) {
+                // combine the pieces: the last of the tile's CTAs to arrive
+                // sums every piece in CTA order and writes the tile
+                const int tb = tile * S;
+                const int c_first = range_owner(tb, p.uq, p.ur);
+                const int c_last = range_owner(tb + S - 1, p.uq, p.ur);
+                int last = 0;
+                if (lane == 0 && ok_all && *abort_flag == 0) {
+                    __threadfence();
+                    last = atomicAdd(&p.cnt[tile], 1) == c_last - c_first;
+                }
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last) {
+                    __threadfence();
+                    for (int o = lane; o < n_out; o += 32) {
+                        float v = 0.0f;
+                        for (int c = c_first; c <= c_last; ++c) {
+                            const int sl = 2 * c + (range_begin(c, p.uq, p.ur) < tb ? 1 : 0);
+                            v += __ldcg(p.ws + static_cast<int64_t>(sl) * n_out + o);
+                        }
+                        const int tok = o / RB;
+                        const int rho = o - tok * RB;
+                        const int m = rho / RBM;
+                        const int n = tile * RBM + (rho - m * RBM);
+                        if (n < p.N) p.y[m][static_cast<int64_t>(tok) * p.N + n] = v;
+                    }
+                    if (lane == 0) p.cnt[tile] = 0;   // ready for the next launch
+                }
+            }
+            j += len;
+            ++tile;
+            st_seg = 0;
+        }
     } else {
-        // ---------------------------------------------------- consumers --
+        // ================================================= compute warps ==
+        // Warp w takes stage w of every load group (if the group has that
+        // many stages), so it alone consumes that position of every ring
+        // slot, round after round.
+        // [ks warps][x_nbuf][M][x_row]; warps w >= ks never hold a stage
+        uint8_t* xbuf = smem + p.x_off + (warp < p.ks ? warp : 0) * (nbuf * M * p.x_row);
+        constexpr int XCH = KPS / 8;                         // 16-byte chunks per token row
+        // x slice of stage st (M token rows of KPS fp16) into buffer b, 16
+        // bytes per lane and copy; k past K reads zeros
+        auto issue_x = [&](int st, int b) {
+            uint8_t* dst = xbuf + b * (M * p.x_row);
+            const int k0 = st * KPS;
+            for (int idx = lane; idx < M * XCH; idx += 32) {
+                const int tok = idx / XCH;
+                const int c = idx - tok * XCH;
+                const int k = k0 + c * 8;
+                const bool ok = k < p.K;
+                const uint16_t* src = ok ? p.x + static_cast<int64_t>(tok) * p.K + k : p.x;
+                cp_async_16(dst + tok * p.x_row + c * 16, src, ok ? 16u : 0u);
+            }
+        };
+        pdl_wait();   // x may be produced by the previous kernel
+        // x for this warp's units of the first nbuf groups
+        GvWalk wx{tile0, st0, nu, p.ks};
+        for (int b = 0; b < nbuf; ++b) {
+            int gt, gs;
+            const int n = wx.left > 0 ? wx.next(S, gt, gs) : 0;
+            if (warp < n) issue_x(gs + warp, b);
+            cp_async_commit();
+        }
+
         const int g = lane >> 2;
         const int t = lane & 3;
-        const int rbase = warp * 16 * MT;       // this warp's first row in a tile
-        int rloc[MT][2];                        // physical rows (within the tile)
+        const int prow = phys_row<BITS>(g);
+        const int xr = p.x_row;
+        int xoff[NT];   // byte offset of this thread's x row (token nt*8+g, clamped to M-1) and k-chunk
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) xoff[nt] = min(nt * 8 + g, M - 1) * xr + t * 32;
+        const int rounds = (M + Cfg::kRedTok - 1) / Cfg::kRedTok;
+        const int nbl = p.red_nbuf - 1;
+        bool dead = false;
+        GvWalk wk{tile0, st0, nu, p.ks};
+        int gi = 0, slot = 0;             // load group index and its ring slot
+        int k = 0;                        // segment (row tile) index
+        float acc[MT][NT][4];
 #pragma unroll
         for (int i = 0; i < MT; ++i)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) rloc[i][h] = rbase + 16 * i + phys_row<BITS>(g) + 8 * h;
-
-        float acc[MT][NT][4];
-        int seg_first_i = 0;                    // unit index where the current segment began
-        // After a timeout a warp keeps walking the units without working, so
-        // every consumer warp reaches the same named barriers: none can wait
-        // at one that another warp has left.
-        bool dead = false;
-        int st = st0, tile = tile0, tm = tile0 % p.n_tiles, mat = tile0 / p.n_tiles;
-        for (int i = 0; i < nu; ++i) {
-            if (i > 0 && ++st == S) {     // next unit: next stage, or next row tile
-                st = 0;
-                ++tile;
-                if (++tm == p.n_tiles) {
-                    tm = 0;
-                    ++mat;
-                }
-            }
-            const int n0 = tm * ROWS;
-            if (i == 0 || st == 0) {
-                seg_first_i = i;
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int a = 0; a < MT; ++a)
-#pragma unroll
-                    for (int j = 0; j < NT; ++j)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) acc[a][j][e] = 0.0f;
-            }
-            const int s = i % SS;
-            if (!dead && !mbar_wait(&full[s], static_cast<uint32_t>(i / SS) & 1, abort_flag,
-                                    p.timeout_ns, p.status))
-                dead = true;
-            if (!dead) {
-            const uint8_t* wt = ring + s * Cfg::kStage;
-            const uint8_t* xt = wt + Cfg::kWStage;
-            // int4 with one n-tile uses the permuted pair order (cheapest
-            // unpacking; x permuted once per group and n-tile)
-            constexpr bool PERM = BITS == 4 && NT == 1;
-            constexpr int CW = BITS == 4 ? 2 : 4;            // code words per row and group
-            // ---- the unit's shared-memory operands, all loaded up front
-            float sv[MT][2][GPS];                             // scales [m-tile][half][group]
-            uint32_t cw[GPS][MT][2][CW];                      // code words
-#pragma unroll
-            for (int a = 0; a < MT; ++a)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int r = rloc[a][h];
-                    const uint8_t* crow = wt + r * 128;
-                    const int sw = r & 7;
-#pragma unroll
-                    for (int q = 0; q < GPS; ++q) {
-                        if constexpr (BITS == 4) {
-                            // bytes [32q + 8t, +8): chunk 2q + t/2, offset (t&1)*8
-                            const uint2 v = *reinterpret_cast<const uint2*>(
-                                crow + (((2 * q + (t >> 1)) ^ sw) << 4) + ((t & 1) << 3));
-                            cw[q][a][h][0] = v.x;
-                            cw[q][a][h][1] = v.y;
-                        } else {
-                            // bytes [64q + 16t, +16): chunk 4q + t
-                            const uint4 v = *reinterpret_cast<const uint4*>(
-                                crow + (((4 * q + t) ^ sw) << 4));
-                            cw[q][a][h][0] = v.x; cw[q][a][h][1] = v.y;
-                            cw[q][a][h][2] = v.z; cw[q][a][h][3] = v.w;
-                        }
-                    }
-                    if constexpr (SSC) {
-                        const uint8_t* sp = xt + Cfg::kXStage + r * GPS * 2;
-                        if constexpr (GPS == 4) {
-                            const uint2 uu = *reinterpret_cast<const uint2*>(sp);
-                            const float2 f0 = __half22float2(u32_as_h2(uu.x));
-                            const float2 f1 = __half22float2(u32_as_h2(uu.y));
-                            sv[a][h][0] = f0.x; sv[a][h][1] = f0.y;
-                            sv[a][h][2] = f1.x; sv[a][h][3] = f1.y;
-                        } else {
-                            const float2 f0 = __half22float2(u32_as_h2(*reinterpret_cast<const uint32_t*>(sp)));
-                            sv[a][h][0] = f0.x; sv[a][h][1] = f0.y;
-                        }
-                    } else {
-                        const int n = n0 + r;
-                        const uint16_t* srow = p.scales[mat] + static_cast<int64_t>(n < p.N ? n : 0) * p.groups;
-#pragma unroll
-                        for (int q = 0; q < GPS; ++q) {
-                            const int grp = st * GPS + q;
-                            sv[a][h][q] = (n < p.N && grp < p.groups)
-                                              ? __half2float(__ushort_as_half(__ldg(srow + grp)))
-                                              : 0.0f;
-                        }
-                    }
-                }
-#pragma unroll
-            for (int q = 0; q < GPS; ++q) {
-                // ---- x fragments of this group: B registers per n-tile and step
-                // (thread (g, t): token g of the n-tile, positions 16t .. 16t+15
-                // of the group; step j covers positions 4j .. 4j+3)
-                uint32_t b[NT][4][2];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const int tok = nt * 8 + g;
-                    const uint8_t* xrow = xt + q * TOK * 128 + tok * 128;
-                    const int sw = tok & 7;
-                    const uint4 x0 = *reinterpret_cast<const uint4*>(xrow + (((2 * t) ^ sw) << 4));
-                    const uint4 x1 = *reinterpret_cast<const uint4*>(xrow + (((2 * t + 1) ^ sw) << 4));
-                    const uint32_t X[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if constexpr (PERM) {
-                            // step j pairs (p0,p4),(p1,p5) or (p2,p6),(p3,p7) of word j/2
-                            const int wb = (j >> 1) * 4 + (j & 1);
-                            b[nt][j][0] = __byte_perm(X[wb], X[wb + 2], 0x5410);
-                            b[nt][j][1] = __byte_perm(X[wb], X[wb + 2], 0x7632);
-                        } else {
-                            b[nt][j][0] = X[2 * j];
-                            b[nt][j][1] = X[2 * j + 1];
-                        }
-                    }
-                }
-                // ---- per m-tile: exact fp16 codes -> A registers, 4 MMA steps,
-                // the group's scale in fp32
-#pragma unroll
-                for (int mi = 0; mi < MT; ++mi) {
-                    uint32_t A[4][4];   // [step][a-reg]
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if constexpr (BITS == 4) {
-                            uint32_t P0[4], P1[4];
-                            if constexpr (PERM) {
-                                i4_word_to_pairs_perm(cw[q][mi][h][0], P0);
-                                i4_word_to_pairs_perm(cw[q][mi][h][1], P1);
-                            } else {
-                                i4_word_to_pairs_nat(cw[q][mi][h][0], P0);
-                                i4_word_to_pairs_nat(cw[q][mi][h][1], P1);
-                            }
-                            // step j: a0a1 (h = 0) / a2a3 (h = 1), and a4a5 / a6a7
-                            A[0][h] = P0[0]; A[0][h + 2] = P0[1];
-                            A[1][h] = P0[2]; A[1][h + 2] = P0[3];
-                            A[2][h] = P1[0]; A[2][h + 2] = P1[1];
-                            A[3][h] = P1[2]; A[3][h + 2] = P1[3];
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                uint32_t Q[2];
-                                i8_word_to_pairs(cw[q][mi][h][j], Q);
-                                A[j][h] = Q[0];
-                                A[j][h + 2] = Q[1];
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        float part[4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) mma16816(part, A[j], b[nt][j][0], b[nt][j][1], j == 0);
-                        acc[mi][nt][0] = fmaf(part[0], sv[mi][0][q], acc[mi][nt][0]);
-                        acc[mi][nt][1] = fmaf(part[1], sv[mi][0][q], acc[mi][nt][1]);
-                        acc[mi][nt][2] = fmaf(part[2], sv[mi][1][q], acc[mi][nt][2]);
-                        acc[mi][nt][3] = fmaf(part[3], sv[mi][1][q], acc[mi][nt][3]);
-                    }
-                }
-            }
-            }   // !dead
+                for (int e = 0; e < 4; ++e) acc[i][nt][e] = 0.0f;
+        while (wk.left > 0) {
+            int g_tile, g_st;
+            const int n = wk.next(S, g_tile, g_st);
+            const bool seg_end = wk.left == 0 || wk.st == 0;   // the group ends this CTA's part of the tile
+            const int xb = nbuf == 2 ? (gi & 1) : 0;
+            // x of this group's unit: all but the newest committed group have landed
+            if (nbuf == 2) cp_async_wait<1>();
+            else cp_async_wait<0>();
             __syncwarp();
-            if (lane == 0 && !dead) mbar_arrive(&empty[s]);
+            // Every warp waits for the group, also one without a stage in it:
+            // it must not release the slot (and later wait on the slot's next
+            // round) before this round has completed.
+            if (!dead && !mbar_wait(&bars->full[slot], static_cast<uint32_t>(gi / SG) & 1,
+                                    abort_flag, p.timeout_ns, p.status))
+                dead = true;
+            if (warp < n) {
+                if (!dead) {
+                    const int st = g_st + warp;
+                    const uint8_t* wt = cring + slot * cgroup + warp * Cfg::kCStage;
+                    // the stage's first group within the slack-padded scale rows
+                    const uint8_t* sc = sring + slot * Cfg::kSGroup +
+                                        (((g_st * GPS) & 7) + warp * GPS) * 2;
+                    const uint8_t* xt = xbuf + xb * (M * xr);
+                    gv_unit<BITS, MT, NT, MTM, Cfg::kSRow, Cfg::kSMat>(
+                        wt, cmat, sc, xt, xoff, prow, t, p.ssc != 0, p.scales, g_tile, st, p.N,
+                        p.groups, acc);
+                }
+            }
+            // ---- the slot and this warp's x buffer are read: release the
+            // slot to the producer, fetch x for the group nbuf ahead
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->empty[slot]);
+            {
+                int gt, gs;
+                const int nx = wx.left > 0 ? wx.next(S, gt, gs) : 0;
+                if (!dead && warp < nx) issue_x(gs + warp, xb);
+                cp_async_commit();
+            }
+            ++gi;
+            if (++slot == SG) slot = 0;
 
-            // ---- end of a tile segment: store it, or combine partial tiles
-            if (st == S - 1 || i == nu - 1) {
-                float* y = p.y[mat];
-                const bool whole = (i - seg_first_i) == st && st == S - 1;   // began at stage 0
-                if (whole && !dead) {
+            if (seg_end) {
+                // ---- end of the segment: deposit this warp's partial sums,
+                // in rounds of up to 16 tokens, for the reduction warp
 #pragma unroll
-                    for (int mi = 0; mi < MT; ++mi)
+                for (int pi = 0; pi < (NT * 8 + Cfg::kRedTok - 1) / Cfg::kRedTok; ++pi) {
+                    if (pi >= rounds) break;                    // uniform over the CTA
+                    const int r = k * rounds + pi;              // reduction round of this CTA
+                    const int b = r & nbl;
+                    float* rw = red + b * Cfg::kRedBuf + warp * Cfg::kRedWarp;
+                    if (r > nbl && !mbar_wait(&bars->red_free[b],
+                                              static_cast<uint32_t>((r >> nbl) - 1) & 1,
+                                              abort_flag, p.timeout_ns, p.status))
+                        dead = true;
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
+                    for (int i = 0; i < MT; ++i)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            if (nt * 8 < pi * Cfg::kRedTok || nt * 8 >= (pi + 1) * Cfg::kRedTok)
+                                continue;
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                const int n = n0 + rloc[mi][e >> 1];
                                 const int tok = nt * 8 + 2 * t + (e & 1);
-                                if (n < p.N && tok < p.M)
-                                    y[static_cast<int64_t>(tok) * p.N + n] = acc[mi][nt][e];
+                                if (tok < M)
+                                    rw[(tok - pi * Cfg::kRedTok) * RS + 16 * i + 8 * (e >> 1) + prow] =
+                                        acc[i][nt][e];
                             }
-                } else if (!whole) {
-                    // This CTA's piece of a tile that several CTAs share: slot 2c
-                    // for the CTA's first segment, 2c+1 for its last one.
-                    const int slot = 2 * cta + (seg_first_i == 0 ? 0 : 1);
-                    float* wsl = p.ws + static_cast<int64_t>(slot) * (TOK * ROWS);
-                    if (!dead)
-#pragma unroll
-                    for (int mi = 0; mi < MT; ++mi)
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                wsl[(nt * 8 + 2 * t + (e & 1)) * ROWS + rloc[mi][e >> 1]] = acc[mi][nt][e];
-                    const int tb = tile * S;
-                    const int c_first = range_owner(tb, p.uq, p.ur);
-                    const int c_last = range_owner(tb + S - 1, p.uq, p.ur);
-                    consumers_sync();
-                    if (threadIdx.x == 0) {
-                        if (*abort_flag) {
-                            *last_flag = 0;
-                        } else {
-                            __threadfence();
-                            const int arrived = atomicAdd(&p.cnt[tile], 1);
-                            *last_flag = arrived == c_last - c_first;
                         }
-                    }
-                    consumers_sync();
-                    if (*last_flag) {
-                        // Last arrival: sum every contributor's piece in CTA
-                        // order (deterministic) and write the tile.
-                        __threadfence();
-                        float sum[MT][NT][4];
-#pragma unroll
-                        for (int mi = 0; mi < MT; ++mi)
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) sum[mi][nt][e] = 0.0f;
-                        for (int c = c_first; c <= c_last; ++c) {
-                            const int sl = 2 * c + (range_begin(c, p.uq, p.ur) < tb ? 1 : 0);
-                            const float* src = p.ws + static_cast<int64_t>(sl) * (TOK * ROWS);
-#pragma unroll
-                            for (int mi = 0; mi < MT; ++mi)
-#pragma unroll
-                                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e)
-                                        sum[mi][nt][e] += __ldcg(src + (nt * 8 + 2 * t + (e & 1)) * ROWS +
-                                                                 rloc[mi][e >> 1]);
-                        }
-#pragma unroll
-                        for (int mi = 0; mi < MT; ++mi)
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int n = n0 + rloc[mi][e >> 1];
-                                    const int tok = nt * 8 + 2 * t + (e & 1);
-                                    if (n < p.N && tok < p.M)
-                                        y[static_cast<int64_t>(tok) * p.N + n] = sum[mi][nt][e];
-                                }
-                        if (threadIdx.x == 0) p.cnt[tile] = 0;   // ready for the next launch
-                    }
-                    consumers_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->red_full[b]);
                 }
+                ++k;
+#pragma unroll
+                for (int i = 0; i < MT; ++i)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[i][nt][e] = 0.0f;
             }
+        }
+        cp_async_wait<0>();   // (only empty or already-landed groups remain)
+    }
+    // After a timeout some issued copies may never have been waited for:
+    // wait (bounded) for the last one of every slot, so none is in flight
+    // when the CTA exits.
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag) {
+        int dummy_abort = 0;
+        for (int s = 0; s < SG; ++s) {
+            const int il = bars->issued_hi[s];
+            if (il >= 0)
+                mbar_wait(&bars->full[s], static_cast<uint32_t>(il / SG) & 1, &dummy_abort,
+                          p.timeout_ns, p.status);
         }
     }
 }
@@ -581,42 +500,131 @@ static int gv_num_sms() {
     return sms;
 }
 
-template <int BITS, int NT, int MT, bool SSC>
-static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* codes, int nmat,
-                             cudaStream_t s, const GemvScratch* scratch) {
-    using Cfg = GvCfg<BITS, NT, MT, SSC>;
-    auto kern = gemv_wq_kernel<BITS, NT, MT, SSC>;
-    static int resident[64] = {};   // CTAs per SM, per device (0 = not yet set up)
+constexpr int kSmemMaxCTA = 227 * 1024;   // dynamic shared memory per CTA, opt-in limit
+
+// Shared-memory layout of one launch: code ring, scale ring, per-warp x
+// buffers, two reduction buffers, barriers.
+struct GvLayout {
+    int ks, sg, x_nbuf, red_nbuf, s_ring_off, x_off, x_row, red_off, bar_off, smem;
+};
+
+static int align_up(int v, int a) { return (v + a - 1) / a * a; }
+
+template <int BITS, int NMAT, int MTM, int NT>
+static GvLayout gv_layout_for(int M, int ks, int sg, int nbuf, int red_nbuf) {
+    using Cfg = GvCfg<BITS, NMAT, MTM, NT>;
+    GvLayout L;
+    L.ks = ks;
+    L.sg = sg;
+    L.x_nbuf = nbuf;
+    L.red_nbuf = red_nbuf;
+    L.s_ring_off = sg * NMAT * ks * Cfg::kCStage;
+    L.x_row = Cfg::kXRow;
+    L.x_off = align_up(L.s_ring_off + sg * Cfg::kSGroup, 16);
+    L.red_off = align_up(L.x_off + ks * nbuf * M * L.x_row, 16);
+    L.bar_off = align_up(L.red_off + red_nbuf * Cfg::kRedBuf * 4, 16);
+    L.smem = 1024 /* alignment slack */ + L.bar_off + static_cast<int>(sizeof(GvBars));
+    return L;
+}
+
+// Within the shared memory of one CTA: the largest load group (ks stages,
+// at most ks_max), then the deepest ring (2..8 groups, no deeper than the
+// busiest CTA's groups), then, if possible, two x buffers per warp and two
+// reduction buffers.
+template <int BITS, int NMAT, int MTM, int NT>
+static bool gv_layout(int M, int ks_max, int nu_max, int S, GvLayout* out) {
+    for (int ks = ks_max; ks >= 1; ks /= 2) {
+        const int groups_max = (nu_max + ks - 1) / ks + (nu_max + S - 1) / S + 1;
+        const int want = groups_max < 2 ? 2 : (groups_max > kGvMaxSG ? kGvMaxSG : groups_max);
+        for (int sg = want; sg >= 2; --sg)
+            for (int nbuf = 2; nbuf >= 1; --nbuf)
+                for (int rbuf = 2; rbuf >= 1; --rbuf) {
+                    const GvLayout L = gv_layout_for<BITS, NMAT, MTM, NT>(M, ks, sg, nbuf, rbuf);
+                    if (L.smem <= kSmemMaxCTA) {
+                        *out = L;
+                        return true;
+                    }
+                }
+        if (ks == 1) break;
+    }
+    return false;
+}
+
+// Share of the SMs' time spent working when whole row tiles are dealt to
+// one CTA per SM: tiles / (SMs * the busiest CTA's tiles).
+static double gv_tile_balance(int tiles, int sms) {
+    const int per = (tiles + sms - 1) / sms;
+    return static_cast<double>(tiles) / (static_cast<double>(per) * sms);
+}
+
+// Whole tiles per CTA when there are no more tiles than SMs (a small
+// projection: nothing then waits on another CTA), or when they balance.
+static bool gv_whole_tiles(int tiles, int sms) {
+    return tiles <= sms || gv_tile_balance(tiles, sms) >= 0.85;
+}
+
+template <int BITS, int NMAT, int MTM, int NT>
+static cudaError_t gv_launch(GvParams& prm, const void* const* codes, cudaStream_t s,
+                             const GemvScratch* scratch) {
+    using Cfg = GvCfg<BITS, NMAT, MTM, NT>;
+    auto kern = gemv_wq_kernel<BITS, NMAT, MTM, NT>;
+    static bool attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (resident[dev] == 0) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+    if (!attr_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMaxCTA);
         if (e != cudaSuccess) return e;
-        int occ = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGvThreads, Cfg::kSmem);
-        if (e != cudaSuccess) return e;
-        resident[dev] = occ > 0 ? occ : 1;
+        attr_set[dev] = true;
     }
-    prm.n_tiles = (prm.N + Cfg::kRows - 1) / Cfg::kRows;
-    prm.kstages = (prm.K + Cfg::kKPS - 1) / Cfg::kKPS;
-    const int64_t tiles = static_cast<int64_t>(nmat) * prm.n_tiles;
-    const int64_t units = tiles * prm.kstages;
+    prm.tiles = (prm.N + Cfg::kRBM - 1) / Cfg::kRBM;
+    const int64_t row_bytes = static_cast<int64_t>(prm.K) * BITS / 8;
+    prm.kstages = static_cast<int>((row_bytes + 127) / 128);
+    const int64_t units = static_cast<int64_t>(prm.tiles) * prm.kstages;
     if (units >= (int64_t{1} << 31)) return cudaErrorInvalidValue;
     prm.units = static_cast<int>(units);
-    // One wave of resident CTAs, each taking an equal run of units.
-    const int64_t slots = static_cast<int64_t>(resident[dev]) * gv_num_sms();
-    const int grid = static_cast<int>(units < slots ? units : slots);
-    prm.uq = prm.units / grid;
-    prm.ur = prm.units % grid;
 
-    const size_t ws_bytes = static_cast<size_t>(2) * grid * Cfg::kTok * Cfg::kRows * sizeof(float);
+    // Grid: one CTA per SM at most.  Whole row tiles per CTA (nothing is
+    // reduced across CTAs) when they balance over the SMs -- one tile per CTA
+    // for small projections; otherwise stream-K over equal runs of units.
+    const int sms = gv_num_sms();
+    int grid = 0;
+    if (gv_whole_tiles(prm.tiles, sms)) {
+        grid = prm.tiles < sms ? prm.tiles : sms;
+        prm.chunk = prm.kstages;
+    } else {
+        grid = static_cast<int>(units < sms ? units : sms);
+        prm.chunk = 1;
+    }
+    const int chunks = prm.units / prm.chunk;
+    prm.uq = chunks / grid;
+    prm.ur = chunks % grid;
+    // The 3D code view needs rows of whole 128-byte stages; otherwise one
+    // stage per group.
+    const int nu_max = (prm.uq + 1) * prm.chunk;
+    GvLayout L;
+    if (!gv_layout<BITS, NMAT, MTM, NT>(prm.M, row_bytes % 128 == 0 ? kGvKS : 1, nu_max,
+                                        prm.kstages, &L))
+        return cudaErrorInvalidValue;
+    prm.ks = L.ks;
+    prm.sg = L.sg;
+    prm.s_ring_off = L.s_ring_off;
+    prm.x_off = L.x_off;
+    prm.x_row = L.x_row;
+    prm.x_nbuf = L.x_nbuf;
+    prm.red_off = L.red_off;
+    prm.red_nbuf = L.red_nbuf;
+    prm.bar_off = L.bar_off;
+    // scales by TMA when a scale row is a multiple of 16 bytes
+    prm.ssc = (prm.groups * 2) % 16 == 0 ? 1 : 0;
+
+    const size_t ws_bytes = static_cast<size_t>(2) * grid * prm.M * Cfg::kRB * sizeof(float);
     if (scratch == nullptr) {
-        e = workspace_get(ws_bytes, static_cast<size_t>(tiles), &prm.ws, &prm.cnt);
+        e = workspace_get(ws_bytes, static_cast<size_t>(prm.tiles), &prm.ws, &prm.cnt);
         if (e != cudaSuccess) return e;
     } else {
-        if (ws_bytes > scratch->ws_bytes || static_cast<size_t>(tiles) > scratch->n_cnt) {
+        if (ws_bytes > scratch->ws_bytes || static_cast<size_t>(prm.tiles) > scratch->n_cnt) {
             if (scratch->too_large) *scratch->too_large = true;
             return cudaErrorInvalidValue;
         }
@@ -624,23 +632,34 @@ static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* co
         prm.cnt = scratch->cnt;
     }
 
-    // codes tensor maps (box rows = ROWS) and x map (box rows = 8*NT)
-    const uint64_t row_bytes = static_cast<uint64_t>(prm.K) * BITS / 8;
-    for (int i = 0; i < nmat; ++i) {
-        if (!make_tmap_2d(&prm.tm_w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, codes[i], row_bytes,
-                          static_cast<uint64_t>(prm.N), row_bytes, 128, Cfg::kRows,
-                          CU_TENSOR_MAP_SWIZZLE_128B))
+    // Codes as {128 B of a stage, row, stage}: a box is ks consecutive stages
+    // of RBM rows, stage-major in shared memory (each stage a [RBM][128 B]
+    // block, 128-byte swizzled like a 2D box).  With one stage per group, a
+    // 2D map, whose columns past the row's end read zeros.
+    for (int i = 0; i < NMAT; ++i) {
+        const bool ok3 =
+            prm.ks > 1
+                ? make_tmap_3d(&prm.tm_w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, codes[i], 128,
+                               static_cast<uint64_t>(prm.N), static_cast<uint64_t>(prm.kstages),
+                               static_cast<uint64_t>(row_bytes), 128, 128, Cfg::kRBM,
+                               static_cast<uint32_t>(prm.ks), CU_TENSOR_MAP_SWIZZLE_128B)
+                : make_tmap_2d(&prm.tm_w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, codes[i],
+                               static_cast<uint64_t>(row_bytes), static_cast<uint64_t>(prm.N),
+                               static_cast<uint64_t>(row_bytes), 128, Cfg::kRBM,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+        if (!ok3) return cudaErrorInvalidValue;
+        if (prm.ssc &&
+            !make_tmap_2d(&prm.tm_s[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, prm.scales[i],
+                          static_cast<uint64_t>(prm.groups), static_cast<uint64_t>(prm.N),
+                          static_cast<uint64_t>(prm.groups) * 2, Cfg::kSRow, Cfg::kRBM,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
-    if (!make_tmap_2d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x,
-                      static_cast<uint64_t>(prm.K), static_cast<uint64_t>(prm.M),
-                      static_cast<uint64_t>(prm.K) * 2, 64, Cfg::kTok, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
     cfg.blockDim = dim3(kGvThreads, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::kSmem);
+    cfg.dynamicSmemBytes = static_cast<size_t>(L.smem);
     cfg.stream = s;
     cudaLaunchAttribute attrs[1];
     int na = 0;
@@ -654,28 +673,65 @@ static cudaError_t gv_launch(GvParams& prm, const void* x, const void* const* co
     return cudaLaunchKernelEx(&cfg, kern, static_cast<const GvParams&>(prm));
 }
 
-template <int BITS, bool SSC>
-static cudaError_t gv_dispatch_ssc(GvParams& prm, const void* x, const void* const* codes, int nmat,
-                                   cudaStream_t s, const GemvScratch* sc) {
-    // 8 tokens per n-tile
-    if (prm.M <= 8) return gv_launch<BITS, 1, 1, SSC>(prm, x, codes, nmat, s, sc);
-    if (prm.M <= 16) return gv_launch<BITS, 2, 1, SSC>(prm, x, codes, nmat, s, sc);
-    if (prm.M <= 24) return gv_launch<BITS, 3, 1, SSC>(prm, x, codes, nmat, s, sc);
-    return gv_launch<BITS, 4, 1, SSC>(prm, x, codes, nmat, s, sc);
+// Rows per matrix in a row tile (16 * MTM): 16 while that gives at most one
+// tile per SM (small projections then run as one wave of whole tiles, no
+// reduction across CTAs); else the largest tile whose whole tiles balance
+// over the SMs (more rows share each x fragment); else 32-row tiles split by
+// stream-K (64 for M > 8, whose x slices are then shared by more rows).
+static int gv_pick_mtm(int N, int M) {
+    const int sms = gv_num_sms();
+    if ((N + 15) / 16 <= sms) return 1;
+    // relative speed of a warp's unit by m-tiles per unit (x fragments are
+    // shared by more rows), measured on B200: 44 / 47 / 49 weights per cycle
+    // and SM for 1 / 2 / 4 m-tiles
+    const double speed[5] = {0.0, 44.0, 47.0, 0.0, 49.0};
+    int best = 0;
+    double best_score = 0.0;
+    for (int mtm = 4; mtm >= 1; mtm /= 2) {
+        const int tiles = (N + 16 * mtm - 1) / (16 * mtm);
+        const double bal = gv_tile_balance(tiles, sms);
+        if (bal >= 0.85 && bal * speed[mtm] > best_score) {
+            best = mtm;
+            best_score = bal * speed[mtm];
+        }
+    }
+    if (best) return best;
+    return M > 8 ? 4 : 2;   // stream-K
 }
 
-template <int BITS>
-static cudaError_t gv_dispatch(GvParams& prm, const void* x, const void* const* codes, int nmat,
-                               cudaStream_t s, const GemvScratch* sc) {
-    constexpr int gps = BITS == 4 ? 4 : 2;
-    if (prm.groups % gps == 0) return gv_dispatch_ssc<BITS, true>(prm, x, codes, nmat, s, sc);
-    return gv_dispatch_ssc<BITS, false>(prm, x, codes, nmat, s, sc);
+template <int BITS, int NMAT, int NT>
+static cudaError_t gv_dispatch_mt(GvParams& prm, const void* const* codes, cudaStream_t s,
+                                  const GemvScratch* sc) {
+    if constexpr (NMAT == 3) {
+        return gv_launch<BITS, 3, 1, NT>(prm, codes, s, sc);
+    } else {
+        int mtm = gv_pick_mtm(prm.N, prm.M);
+        // large M: the per-warp x buffers leave less room; fall back to fewer rows
+        GvLayout L;
+        if (mtm == 4 && !(gv_layout<BITS, 1, 4, NT>(prm.M, kGvKS, kGvKS, kGvKS, &L) && L.ks == kGvKS))
+            mtm = 2;
+        if (mtm == 2 && !(gv_layout<BITS, 1, 2, NT>(prm.M, kGvKS, kGvKS, kGvKS, &L) && L.ks == kGvKS))
+            mtm = 1;
+        if (mtm == 1) return gv_launch<BITS, 1, 1, NT>(prm, codes, s, sc);
+        if (mtm == 2) return gv_launch<BITS, 1, 2, NT>(prm, codes, s, sc);
+        return gv_launch<BITS, 1, 4, NT>(prm, codes, s, sc);
+    }
+}
+
+template <int BITS, int NMAT>
+static cudaError_t gv_dispatch_nt(GvParams& prm, const void* const* codes, cudaStream_t s,
+                                  const GemvScratch* sc) {
+    // 8 tokens per n-tile
+    if (prm.M <= 8) return gv_dispatch_mt<BITS, NMAT, 1>(prm, codes, s, sc);
+    if (prm.M <= 16) return gv_dispatch_mt<BITS, NMAT, 2>(prm, codes, s, sc);
+    return gv_dispatch_mt<BITS, NMAT, 4>(prm, codes, s, sc);
 }
 
 static cudaError_t gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
                                 const WOperand* w, int nmat, cudaStream_t s, const GemvScratch* sc) {
     GvParams prm;
     memset(&prm, 0, sizeof(prm));
+    prm.x = x;
     prm.M = static_cast<int>(M);
     prm.N = static_cast<int>(N);
     prm.K = static_cast<int>(K);
@@ -688,8 +744,11 @@ static cudaError_t gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t
         prm.scales[i] = w[i].scales;
         prm.y[i] = w[i].y;
     }
-    return bits == 4 ? gv_dispatch<4>(prm, x, codes, nmat, s, sc)
-                     : gv_dispatch<8>(prm, x, codes, nmat, s, sc);
+    if (nmat == 3)
+        return bits == 4 ? gv_dispatch_nt<4, 3>(prm, codes, s, sc)
+                         : gv_dispatch_nt<8, 3>(prm, codes, s, sc);
+    return bits == 4 ? gv_dispatch_nt<4, 1>(prm, codes, s, sc)
+                     : gv_dispatch_nt<8, 1>(prm, codes, s, sc);
 }
 
 cudaError_t launch_gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,

@@ -57,6 +57,12 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                   uint64_t inner_elems, uint64_t rows, uint64_t row_stride_bytes,
                   uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz);
 
+// 3D tiled tensor map: dims {d0 (contiguous), d1, d2}, byte strides s1, s2
+// (any order), box {b0, b1, b2}.
+bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0,
+                  uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1,
+                  uint32_t b2, CUtensorMapSwizzle swz);
+
 // Whether programmatic dependent launch is requested for kernel launches.
 bool pdl_enabled();
 
