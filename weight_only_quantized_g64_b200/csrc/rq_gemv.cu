@@ -60,10 +60,10 @@
 namespace rq {
 
 struct GvParams {
-    CUtensorMap tm_w[3];  // codes [N, K*bits/8] u8; ks == KS: 3D {128 B, N rows, stages}, box
-                          // {128, RBM, KS}; ks == 1: 2D {row bytes, N}, box {128, RBM}; SWIZZLE_128B
+    CUtensorMap tm_w[3];  // codes [N, K*bits/8] u8; ks > 1: 3D {128 B, N rows, stages}, box
+                          // {128, RBM, ks}; ks == 1: 2D {row bytes, N}, box {128, RBM}; SWIZZLE_128B
     CUtensorMap tm_s[3];  // scales [N, K/64] fp16: box {SROW groups, RBM}, no swizzle (when ssc)
-    const uint16_t* x;    // [M, K] fp16
+    CUtensorMap tm_x;     // x [M, K] fp16 as 3D {64, M tokens, K/64 groups}: box {64, M, ks*GPS}, SWIZZLE_128B
     const uint16_t* scales[3];
     float* y[3];
     int M, N, K;
@@ -74,13 +74,10 @@ struct GvParams {
     int chunk;            // units are dealt in chunks: kstages (whole tiles) or 1 (stream-K)
     int uq, ur;           // chunks / gridDim.x and chunks % gridDim.x: CTA c owns chunks
                           // [c*uq + min(c, ur), (c+1)*uq + min(c+1, ur))
-    int ks;               // stages per load group (8, 4 when shared memory is short, or 1 when
-                          // rows are not whole stages); warps w < ks compute
+    int ks;               // stages per load group: WK, or 1 when rows are not whole stages
     int sg;               // ring depth in load groups (2..8)
-    int s_ring_off;       // offset of the scale ring (after the code ring)
-    int x_off;            // offset of the per-warp x buffers
-    int x_row;            // bytes per token row of an x buffer
-    int x_nbuf;           // x buffers per warp (1 or 2)
+    int slot_bytes;       // bytes per ring slot: codes, then scales, then x
+    int s_off, x_off;     // offsets of the scales and x within a slot
     int red_off;          // offset of the reduction buffers
     int red_nbuf;         // reduction buffers (1 or 2)
     int bar_off;          // offset of the barriers
@@ -92,34 +89,36 @@ struct GvParams {
 };
 
 constexpr int kGvConsumers = 8;                         // warps that multiply
-constexpr int kGvProducer = kGvConsumers;               // warp that refills the ring
+constexpr int kGvProducer = kGvConsumers;               // warp that fills the ring
 constexpr int kGvReducer = kGvConsumers + 1;            // warp that reduces and stores
 constexpr int kGvThreads = (kGvConsumers + 2) * 32;
-constexpr int kGvKS = kGvConsumers;                     // k-stages per load group (one per warp)
 constexpr int kGvMaxSG = 8;                             // ring depth limit, in load groups
 
-// BITS: 4 or 8.  NMAT: matrices sharing x (1, or 3 for fused R/K/V).  MTM:
-// 16-row m-tiles per matrix in a row tile.  NT: 8-token n-tiles (M <= 8 NT).
-template <int BITS, int NMAT, int MTM, int NT>
+// BITS: 4 or 8.  NMAT: matrices sharing x (1, or 3 for fused R/K/V).  MTW:
+// 16-row m-tiles per warp and matrix.  NT: 8-token n-tiles (M <= 8 NT).  WK:
+// compute warps along k (8, 2 or 1); the other factor WR = 8 / WK splits the
+// rows.  Warp w takes stage w % WK of each load group and rows block w / WK.
+template <int BITS, int NMAT, int MTW, int NT, int WK>
 struct GvCfg {
-    static constexpr int kMT = NMAT * MTM;                   // m-tiles per row tile
-    static constexpr int kRBM = 16 * MTM;                    // rows per matrix
-    static constexpr int kRB = 16 * kMT;                     // rows per row tile
+    static constexpr int kWR = kGvConsumers / WK;            // warps along rows
+    static constexpr int kMT = NMAT * MTW;                   // m-tiles per warp
+    static constexpr int kRBM = kWR * 16 * MTW;              // rows per matrix in a row tile
+    static constexpr int kRB = NMAT * kRBM;                  // rows per row tile
     static constexpr int kKPS = BITS == 4 ? 256 : 128;       // k per stage (128 code bytes)
     static constexpr int kGPS = kKPS / 64;                   // groups per stage
     static constexpr int kTok = 8 * NT;
-    // a load group: ks stages of a row tile, per matrix [ks][RBM rows][128 B]
+    // a load group: ks <= WK stages of a row tile, per matrix [ks][RBM rows][128 B]
     static constexpr int kCStage = kRBM * 128;               // code bytes per matrix and stage
-    // scales: per matrix [RBM rows][SROW] fp16, SROW = the group's KS*GPS
-    // groups plus 8 of slack, so the box can start at a 16-byte boundary
-    static constexpr int kSRow = kGvKS * kGPS + 8;
+    // scales: per matrix [RBM rows][SROW] fp16, SROW = the group's WK*GPS
+    // groups plus 8 of slack (so the box can start at a 16-byte boundary),
+    // rounded up to 16 bytes
+    static constexpr int kSRow = (WK * kGPS + 8 + 7) / 8 * 8;
     static constexpr int kSMat = kRBM * kSRow * 2;
     static constexpr int kSGroup = NMAT * kSMat;
-    static constexpr int kXRow = kKPS * 2 + 16;              // x bytes per token row (+16: banks)
     static constexpr int kRedStride = kRB + 4;               // floats per token row (bank spread)
     static constexpr int kRedTok = kTok < 16 ? kTok : 16;    // tokens per reduction round
-    static constexpr int kRedWarp = kRedTok * kRedStride;    // floats per warp
-    static constexpr int kRedBuf = kGvConsumers * kRedWarp;  // floats per reduction buffer
+    static constexpr int kRedWarp = kRedTok * kRedStride;    // floats per k-warp deposit
+    static constexpr int kRedBuf = WK * kRedWarp;            // floats per reduction buffer
     static_assert(kCStage % 1024 == 0, "group alignment");
     static_assert((kSRow * 2) % 16 == 0, "scale rows must be 16-byte multiples");
     static_assert(kSMat % 128 == 0, "TMA destinations must be 128-byte aligned");
@@ -127,8 +126,8 @@ struct GvCfg {
 
 // Barriers and flags after the buffers.
 struct GvBars {
-    uint64_t full[kGvMaxSG];   // ring slot holds its group's codes and scales
-    uint64_t empty[kGvMaxSG];  // every consumer warp is done with the slot
+    uint64_t full[kGvMaxSG];   // ring slot holds its group's codes, scales and x
+    uint64_t empty[kGvMaxSG];  // every compute warp is done with the slot
     uint64_t red_full[2];      // every warp has deposited its partial sums
     uint64_t red_free[2];      // the reducing warp has read the buffer
     int issued_hi[kGvMaxSG];   // last group issued into each slot
@@ -146,7 +145,7 @@ __device__ __forceinline__ int range_owner(int u, int uq, int ur) {
     return u < big ? u / (uq + 1) : ur + (u - big) / uq;
 }
 
-// Walks a CTA's units as load groups: up to KS consecutive stages of one row
+// Walks a CTA's units as load groups: up to ks consecutive stages of one row
 // tile, never past the tile or the CTA's range.
 struct GvWalk {
     int tile, st, left, ks;
@@ -166,14 +165,13 @@ struct GvWalk {
     }
 };
 
-template <int BITS, int NMAT, int MTM, int NT>
+template <int BITS, int NMAT, int MTW, int NT, int WK>
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_constant__ GvParams p) {
-    using Cfg = GvCfg<BITS, NMAT, MTM, NT>;
+    using Cfg = GvCfg<BITS, NMAT, MTW, NT, WK>;
     constexpr int MT = Cfg::kMT;
     constexpr int RBM = Cfg::kRBM;
     constexpr int RB = Cfg::kRB;
     constexpr int GPS = Cfg::kGPS;
-    constexpr int KPS = Cfg::kKPS;
     constexpr int RS = Cfg::kRedStride;
     constexpr int NW = kGvConsumers;
     extern __shared__ uint8_t smem_raw[];
@@ -181,10 +179,10 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
                                                ~static_cast<uintptr_t>(1023));
     const int SG = p.sg;
     const int cmat = p.ks * Cfg::kCStage;                   // code bytes per matrix and group
-    const int cgroup = NMAT * cmat;                         // code bytes per group
-    uint8_t* cring = smem;                                  // [SG][NMAT][ks][RBM][128 B], swizzled
-    uint8_t* sring = smem + p.s_ring_off;                   // [SG][NMAT][RBM][SROW] fp16
-    float* red = reinterpret_cast<float*>(smem + p.red_off);   // [red_nbuf][NW][kRedTok][RS]
+    // ring slot: codes [NMAT][ks][RBM][128 B] (swizzled), scales
+    // [NMAT][RBM][SROW] fp16, x [ks*GPS groups][M][128 B] (swizzled)
+    uint8_t* ring = smem;
+    float* red = reinterpret_cast<float*>(smem + p.red_off);   // [red_nbuf][WK][kRedTok][RS]
     GvBars* bars = reinterpret_cast<GvBars*>(smem + p.bar_off);
     volatile int* abort_flag = &bars->abort;
 
@@ -197,7 +195,6 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
     const int nu = (p.uq + (cta < p.ur ? 1 : 0)) * p.chunk;
     const int tile0 = u0 / S;
     const int st0 = u0 - tile0 * S;
-    const int nbuf = p.x_nbuf;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SG; ++s) {
@@ -211,6 +208,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
         }
         bars->abort = 0;
         fence_mbar_init();
+        tma_prefetch_desc(&p.tm_x);
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
             tma_prefetch_desc(&p.tm_w[m]);
@@ -222,38 +220,60 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
 
     if (warp == kGvProducer) {
         // ================================================= producer warp ==
-        // Fills the ring, one load group per slot: the first SG groups
-        // before waiting on the previous grid (codes and scales do not depend
-        // on it), then group i as soon as every consumer warp is done with
-        // group i - SG, which used the same slot.
+        // Fills the ring, one load group per slot: codes and scales of the
+        // first SG groups before waiting on the previous grid (they do not
+        // depend on it), their x after; then group i (codes, scales, x) as
+        // soon as every compute warp is done with group i - SG, which used
+        // the same slot.
         if (lane == 0) {
             const uint64_t pol_w = l2_policy_evict_first();
-            GvWalk wk{tile0, st0, nu, p.ks};
-            int slot = 0;
-            for (int i = 0; wk.left > 0; ++i) {
-                if (i >= SG && !mbar_wait(&bars->empty[slot], static_cast<uint32_t>(i / SG - 1) & 1,
-                                          abort_flag, p.timeout_ns, p.status))
-                    break;
-                int g_tile, g_st;
-                wk.next(S, g_tile, g_st);
-                bars->issued_hi[slot] = i;
+            const uint64_t pol_x = l2_policy_evict_last();
+            const uint32_t x_bytes = static_cast<uint32_t>(p.ks * GPS * M * 128);
+            auto issue_w = [&](int slot, int g_tile, int g_st) {
+                uint8_t* dst = ring + slot * p.slot_bytes;
                 mbar_arrive_expect_tx(&bars->full[slot],
-                                      static_cast<uint32_t>(cgroup + (p.ssc ? Cfg::kSGroup : 0)));
-                uint8_t* cdst = cring + slot * cgroup;
-                uint8_t* sdst = sring + slot * Cfg::kSGroup;
+                                      static_cast<uint32_t>(NMAT * cmat + (p.ssc ? Cfg::kSGroup : 0)) +
+                                          x_bytes);
                 const int sx = (g_st * GPS) & ~7;   // 16-byte aligned first scale group
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) {
                     if (p.ks > 1)
-                        tma_load_3d(cdst + m * cmat, &p.tm_w[m], &bars->full[slot], 0,
-                                    g_tile * RBM, g_st, pol_w);
+                        tma_load_3d(dst + m * cmat, &p.tm_w[m], &bars->full[slot], 0, g_tile * RBM,
+                                    g_st, pol_w);
                     else
-                        tma_load_2d(cdst + m * cmat, &p.tm_w[m], &bars->full[slot], g_st * 128,
+                        tma_load_2d(dst + m * cmat, &p.tm_w[m], &bars->full[slot], g_st * 128,
                                     g_tile * RBM, pol_w);
                     if (p.ssc)
-                        tma_load_2d(sdst + m * Cfg::kSMat, &p.tm_s[m], &bars->full[slot], sx,
-                                    g_tile * RBM, pol_w);
+                        tma_load_2d(dst + p.s_off + m * Cfg::kSMat, &p.tm_s[m], &bars->full[slot],
+                                    sx, g_tile * RBM, pol_w);
                 }
+            };
+            auto issue_x = [&](int slot, int g_st) {
+                tma_load_3d(ring + slot * p.slot_bytes + p.x_off, &p.tm_x, &bars->full[slot], 0, 0,
+                            g_st * GPS, pol_x);
+            };
+            GvWalk wk{tile0, st0, nu, p.ks};
+            int first_st[kGvMaxSG];
+            int i = 0;
+            for (; i < SG && wk.left > 0; ++i) {
+                int g_tile, g_st;
+                wk.next(S, g_tile, g_st);
+                bars->issued_hi[i] = i;
+                issue_w(i, g_tile, g_st);
+                first_st[i] = g_st;
+            }
+            pdl_wait();   // x may be produced by the previous kernel
+            for (int j = 0; j < i; ++j) issue_x(j, first_st[j]);
+            int slot = i == SG ? 0 : i;
+            for (; wk.left > 0; ++i) {
+                if (!mbar_wait(&bars->empty[slot], static_cast<uint32_t>(i / SG - 1) & 1, abort_flag,
+                               p.timeout_ns, p.status))
+                    break;
+                int g_tile, g_st;
+                wk.next(S, g_tile, g_st);
+                bars->issued_hi[slot] = i;
+                issue_w(slot, g_tile, g_st);
+                issue_x(slot, g_st);
                 if (++slot == SG) slot = 0;
             }
         }
@@ -262,9 +282,9 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
     } else if (warp == kGvReducer) {
         // ================================================ reduction warp ==
         // Walks the same row tiles as the compute warps; for every round it
-        // adds the 8 deposits in warp order (deterministic) and stores the
-        // tile, or this CTA's piece of a tile that several CTAs share.  It
-        // issues no loads of its own, so its fences are cheap.
+        // adds the WK deposits of each row in k order (deterministic) and
+        // stores the tile, or this CTA's piece of a tile that several CTAs
+        // share.  It issues no loads of its own, so its fences are cheap.
         pdl_wait();   // (its stores follow the compute warps' waits anyway)
         const int rounds = (M + Cfg::kRedTok - 1) / Cfg::kRedTok;
         const int nbl = p.red_nbuf - 1;                 // log2 of the buffer count (0 or 1)
@@ -290,7 +310,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
                         const int rho = o - tl * RB;
                         float v = 0.0f;
 #pragma unroll
-                        for (int w = 0; w < NW; ++w) v += rb[w * Cfg::kRedWarp + tl * RS + rho];
+                        for (int kw = 0; kw < WK; ++kw) v += rb[kw * Cfg::kRedWarp + tl * RS + rho];
                         const int tok = tok0 + tl;
                         if (whole) {
                             const int m = rho / RBM;
@@ -319,17 +339,43 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
                 last = __shfl_sync(0xffffffffu, last, 0);
                 if (last) {
                     __threadfence();
-                    for (int o = lane; o < n_out; o += 32) {
-                        float v = 0.0f;
-                        for (int c = c_first; c <= c_last; ++c) {
-                            const int sl = 2 * c + (range_begin(c, p.uq, p.ur) < tb ? 1 : 0);
-                            v += __ldcg(p.ws + static_cast<int64_t>(sl) * n_out + o);
+                    // 4 outputs per lane and step, every contributor's piece
+                    // loaded before any is added (loads in flight together);
+                    // the sum runs over the contributors in CTA order
+                    constexpr int kMaxC = 16;
+                    const int nc = c_last - c_first + 1;
+                    for (int o4 = lane * 4; o4 < n_out; o4 += 128) {
+                        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int c0 = 0; c0 < nc; c0 += kMaxC) {
+                            float4 part[kMaxC];
+#pragma unroll
+                            for (int ci = 0; ci < kMaxC; ++ci) {
+                                const int c = c_first + c0 + ci;
+                                if (c0 + ci < nc) {
+                                    const int sl = 2 * c + (range_begin(c, p.uq, p.ur) < tb ? 1 : 0);
+                                    part[ci] = __ldcg(reinterpret_cast<const float4*>(
+                                        p.ws + static_cast<int64_t>(sl) * n_out + o4));
+                                }
+                            }
+#pragma unroll
+                            for (int ci = 0; ci < kMaxC; ++ci)
+                                if (c0 + ci < nc) {
+                                    v.x += part[ci].x;
+                                    v.y += part[ci].y;
+                                    v.z += part[ci].z;
+                                    v.w += part[ci].w;
+                                }
                         }
-                        const int tok = o / RB;
-                        const int rho = o - tok * RB;
-                        const int m = rho / RBM;
-                        const int n = tile * RBM + (rho - m * RBM);
-                        if (n < p.N) p.y[m][static_cast<int64_t>(tok) * p.N + n] = v;
+                        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int o = o4 + e;
+                            const int tok = o / RB;
+                            const int rho = o - tok * RB;
+                            const int m = rho / RBM;
+                            const int n = tile * RBM + (rho - m * RBM);
+                            if (n < p.N) p.y[m][static_cast<int64_t>(tok) * p.N + n] = vv[e];
+                        }
                     }
                     if (lane == 0) p.cnt[tile] = 0;   // ready for the next launch
                 }
@@ -340,43 +386,17 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
         }
     } else {
         // ================================================= compute warps ==
-        // Warp w takes stage w of every load group (if the group has that
-        // many stages), so it alone consumes that position of every ring
-        // slot, round after round.
-        // [ks warps][x_nbuf][M][x_row]; warps w >= ks never hold a stage
-        uint8_t* xbuf = smem + p.x_off + (warp < p.ks ? warp : 0) * (nbuf * M * p.x_row);
-        constexpr int XCH = KPS / 8;                         // 16-byte chunks per token row
-        // x slice of stage st (M token rows of KPS fp16) into buffer b, 16
-        // bytes per lane and copy; k past K reads zeros
-        auto issue_x = [&](int st, int b) {
-            uint8_t* dst = xbuf + b * (M * p.x_row);
-            const int k0 = st * KPS;
-            for (int idx = lane; idx < M * XCH; idx += 32) {
-                const int tok = idx / XCH;
-                const int c = idx - tok * XCH;
-                const int k = k0 + c * 8;
-                const bool ok = k < p.K;
-                const uint16_t* src = ok ? p.x + static_cast<int64_t>(tok) * p.K + k : p.x;
-                cp_async_16(dst + tok * p.x_row + c * 16, src, ok ? 16u : 0u);
-            }
-        };
-        pdl_wait();   // x may be produced by the previous kernel
-        // x for this warp's units of the first nbuf groups
-        GvWalk wx{tile0, st0, nu, p.ks};
-        for (int b = 0; b < nbuf; ++b) {
-            int gt, gs;
-            const int n = wx.left > 0 ? wx.next(S, gt, gs) : 0;
-            if (warp < n) issue_x(gs + warp, b);
-            cp_async_commit();
-        }
-
+        // Warp w takes stage w % WK of every load group (if the group has that
+        // many stages) and row block w / WK, so it alone consumes that part
+        // of every ring slot, round after round.
+        const int kw = warp % WK;
+        const int rw = warp / WK;
         const int g = lane >> 2;
         const int t = lane & 3;
         const int prow = phys_row<BITS>(g);
-        const int xr = p.x_row;
-        int xoff[NT];   // byte offset of this thread's x row (token nt*8+g, clamped to M-1) and k-chunk
+        int xtok[NT];   // this thread's token per n-tile, clamped to a valid one
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) xoff[nt] = min(nt * 8 + g, M - 1) * xr + t * 32;
+        for (int nt = 0; nt < NT; ++nt) xtok[nt] = min(nt * 8 + g, M - 1);
         const int rounds = (M + Cfg::kRedTok - 1) / Cfg::kRedTok;
         const int nbl = p.red_nbuf - 1;
         bool dead = false;
@@ -394,40 +414,26 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
             int g_tile, g_st;
             const int n = wk.next(S, g_tile, g_st);
             const bool seg_end = wk.left == 0 || wk.st == 0;   // the group ends this CTA's part of the tile
-            const int xb = nbuf == 2 ? (gi & 1) : 0;
-            // x of this group's unit: all but the newest committed group have landed
-            if (nbuf == 2) cp_async_wait<1>();
-            else cp_async_wait<0>();
-            __syncwarp();
             // Every warp waits for the group, also one without a stage in it:
             // it must not release the slot (and later wait on the slot's next
             // round) before this round has completed.
             if (!dead && !mbar_wait(&bars->full[slot], static_cast<uint32_t>(gi / SG) & 1,
                                     abort_flag, p.timeout_ns, p.status))
                 dead = true;
-            if (warp < n) {
-                if (!dead) {
-                    const int st = g_st + warp;
-                    const uint8_t* wt = cring + slot * cgroup + warp * Cfg::kCStage;
-                    // the stage's first group within the slack-padded scale rows
-                    const uint8_t* sc = sring + slot * Cfg::kSGroup +
-                                        (((g_st * GPS) & 7) + warp * GPS) * 2;
-                    const uint8_t* xt = xbuf + xb * (M * xr);
-                    gv_unit<BITS, MT, NT, MTM, Cfg::kSRow, Cfg::kSMat>(
-                        wt, cmat, sc, xt, xoff, prow, t, p.ssc != 0, p.scales, g_tile, st, p.N,
-                        p.groups, acc);
-                }
+            if (kw < n && !dead) {
+                const int st = g_st + kw;
+                const uint8_t* base = ring + slot * p.slot_bytes;
+                const uint8_t* wt = base + kw * Cfg::kCStage + rw * (16 * MTW * 128);
+                // the stage's first group within the slack-padded scale rows
+                const uint8_t* sc = base + p.s_off + rw * (16 * MTW) * Cfg::kSRow * 2 +
+                                    (((g_st * GPS) & 7) + kw * GPS) * 2;
+                gv_unit<BITS, MT, NT, MTW, Cfg::kSRow, Cfg::kSMat>(
+                    wt, cmat, sc, base + p.x_off, kw * GPS, M, xtok, prow, t, p.ssc != 0, p.scales,
+                    g_tile * RBM + rw * 16 * MTW, st, p.N, p.groups, acc);
             }
-            // ---- the slot and this warp's x buffer are read: release the
-            // slot to the producer, fetch x for the group nbuf ahead
+            // ---- the slot is read: release it to the producer
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->empty[slot]);
-            {
-                int gt, gs;
-                const int nx = wx.left > 0 ? wx.next(S, gt, gs) : 0;
-                if (!dead && warp < nx) issue_x(gs + warp, xb);
-                cp_async_commit();
-            }
             ++gi;
             if (++slot == SG) slot = 0;
 
@@ -439,13 +445,15 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
                     if (pi >= rounds) break;                    // uniform over the CTA
                     const int r = k * rounds + pi;              // reduction round of this CTA
                     const int b = r & nbl;
-                    float* rw = red + b * Cfg::kRedBuf + warp * Cfg::kRedWarp;
+                    float* rw_ = red + b * Cfg::kRedBuf + kw * Cfg::kRedWarp;
                     if (r > nbl && !mbar_wait(&bars->red_free[b],
                                               static_cast<uint32_t>((r >> nbl) - 1) & 1,
                                               abort_flag, p.timeout_ns, p.status))
                         dead = true;
 #pragma unroll
-                    for (int i = 0; i < MT; ++i)
+                    for (int i = 0; i < MT; ++i) {
+                        // m-tile i: matrix i / MTW, rows rw*16*MTW + 16*(i % MTW) of it
+                        const int rbase = (i / MTW) * RBM + rw * 16 * MTW + 16 * (i % MTW);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
                             if (nt * 8 < pi * Cfg::kRedTok || nt * 8 >= (pi + 1) * Cfg::kRedTok)
@@ -454,10 +462,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
                             for (int e = 0; e < 4; ++e) {
                                 const int tok = nt * 8 + 2 * t + (e & 1);
                                 if (tok < M)
-                                    rw[(tok - pi * Cfg::kRedTok) * RS + 16 * i + 8 * (e >> 1) + prow] =
+                                    rw_[(tok - pi * Cfg::kRedTok) * RS + rbase + 8 * (e >> 1) + prow] =
                                         acc[i][nt][e];
                             }
                         }
+                    }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->red_full[b]);
                 }
@@ -470,7 +479,6 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
                         for (int e = 0; e < 4; ++e) acc[i][nt][e] = 0.0f;
             }
         }
-        cp_async_wait<0>();   // (only empty or already-landed groups remain)
     }
     // After a timeout some issued copies may never have been waited for:
     // wait (bounded) for the last one of every slot, so none is in flight
@@ -502,51 +510,45 @@ static int gv_num_sms() {
 
 constexpr int kSmemMaxCTA = 227 * 1024;   // dynamic shared memory per CTA, opt-in limit
 
-// Shared-memory layout of one launch: code ring, scale ring, per-warp x
-// buffers, two reduction buffers, barriers.
-struct GvLayout {
-    int ks, sg, x_nbuf, red_nbuf, s_ring_off, x_off, x_row, red_off, bar_off, smem;
-};
-
 static int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
-template <int BITS, int NMAT, int MTM, int NT>
-static GvLayout gv_layout_for(int M, int ks, int sg, int nbuf, int red_nbuf) {
-    using Cfg = GvCfg<BITS, NMAT, MTM, NT>;
+// Shared-memory layout of one launch: SG ring slots (codes, scales, x of a
+// load group), reduction buffers, barriers.
+struct GvLayout {
+    int ks, sg, red_nbuf, slot_bytes, s_off, x_off, red_off, bar_off, smem;
+};
+
+template <int BITS, int NMAT, int MTW, int NT, int WK>
+static GvLayout gv_layout_for(int M, int ks, int sg, int red_nbuf) {
+    using Cfg = GvCfg<BITS, NMAT, MTW, NT, WK>;
     GvLayout L;
     L.ks = ks;
     L.sg = sg;
-    L.x_nbuf = nbuf;
     L.red_nbuf = red_nbuf;
-    L.s_ring_off = sg * NMAT * ks * Cfg::kCStage;
-    L.x_row = Cfg::kXRow;
-    L.x_off = align_up(L.s_ring_off + sg * Cfg::kSGroup, 16);
-    L.red_off = align_up(L.x_off + ks * nbuf * M * L.x_row, 16);
+    L.s_off = NMAT * ks * Cfg::kCStage;                    // a multiple of 1024
+    L.x_off = align_up(L.s_off + Cfg::kSGroup, 1024);      // swizzled x box: 1024-aligned
+    L.slot_bytes = align_up(L.x_off + ks * Cfg::kGPS * M * 128, 1024);
+    L.red_off = sg * L.slot_bytes;
     L.bar_off = align_up(L.red_off + red_nbuf * Cfg::kRedBuf * 4, 16);
     L.smem = 1024 /* alignment slack */ + L.bar_off + static_cast<int>(sizeof(GvBars));
     return L;
 }
 
-// Within the shared memory of one CTA: the largest load group (ks stages,
-// at most ks_max), then the deepest ring (2..8 groups, no deeper than the
-// busiest CTA's groups), then, if possible, two x buffers per warp and two
-// reduction buffers.
-template <int BITS, int NMAT, int MTM, int NT>
-static bool gv_layout(int M, int ks_max, int nu_max, int S, GvLayout* out) {
-    for (int ks = ks_max; ks >= 1; ks /= 2) {
-        const int groups_max = (nu_max + ks - 1) / ks + (nu_max + S - 1) / S + 1;
-        const int want = groups_max < 2 ? 2 : (groups_max > kGvMaxSG ? kGvMaxSG : groups_max);
-        for (int sg = want; sg >= 2; --sg)
-            for (int nbuf = 2; nbuf >= 1; --nbuf)
-                for (int rbuf = 2; rbuf >= 1; --rbuf) {
-                    const GvLayout L = gv_layout_for<BITS, NMAT, MTM, NT>(M, ks, sg, nbuf, rbuf);
-                    if (L.smem <= kSmemMaxCTA) {
-                        *out = L;
-                        return true;
-                    }
-                }
-        if (ks == 1) break;
-    }
+// Within the shared memory of one CTA: the deepest ring (2..8 groups, no
+// deeper than the busiest CTA's groups), with two reduction buffers if
+// possible, for groups of ks stages.
+template <int BITS, int NMAT, int MTW, int NT, int WK>
+static bool gv_layout(int M, int ks, int nu_max, int S, GvLayout* out) {
+    const int groups_max = (nu_max + ks - 1) / ks + (nu_max + S - 1) / S + 1;
+    const int want = groups_max < 2 ? 2 : (groups_max > kGvMaxSG ? kGvMaxSG : groups_max);
+    for (int sg = want; sg >= 2; --sg)
+        for (int rbuf = 2; rbuf >= 1; --rbuf) {
+            const GvLayout L = gv_layout_for<BITS, NMAT, MTW, NT, WK>(M, ks, sg, rbuf);
+            if (L.smem <= kSmemMaxCTA) {
+                *out = L;
+                return true;
+            }
+        }
     return false;
 }
 
@@ -557,17 +559,17 @@ static double gv_tile_balance(int tiles, int sms) {
     return static_cast<double>(tiles) / (static_cast<double>(per) * sms);
 }
 
-// Whole tiles per CTA when there are no more tiles than SMs (a small
-// projection: nothing then waits on another CTA), or when they balance.
+// Whole tiles per CTA (nothing then waits on another CTA) when they keep the
+// SMs at least 85% busy, e.g. 128 16-row tiles of a 2048-row projection.
 static bool gv_whole_tiles(int tiles, int sms) {
-    return tiles <= sms || gv_tile_balance(tiles, sms) >= 0.85;
+    return gv_tile_balance(tiles, sms) >= 0.85;
 }
 
-template <int BITS, int NMAT, int MTM, int NT>
-static cudaError_t gv_launch(GvParams& prm, const void* const* codes, cudaStream_t s,
-                             const GemvScratch* scratch) {
-    using Cfg = GvCfg<BITS, NMAT, MTM, NT>;
-    auto kern = gemv_wq_kernel<BITS, NMAT, MTM, NT>;
+template <int BITS, int NMAT, int MTW, int NT, int WK>
+static cudaError_t gv_launch(GvParams& prm, const uint16_t* x, const void* const* codes,
+                             cudaStream_t s, const GemvScratch* scratch) {
+    using Cfg = GvCfg<BITS, NMAT, MTW, NT, WK>;
+    auto kern = gemv_wq_kernel<BITS, NMAT, MTW, NT, WK>;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -601,30 +603,33 @@ static cudaError_t gv_launch(GvParams& prm, const void* const* codes, cudaStream
     prm.uq = chunks / grid;
     prm.ur = chunks % grid;
     // The 3D code view needs rows of whole 128-byte stages; otherwise one
-    // stage per group.
-    const int nu_max = (prm.uq + 1) * prm.chunk;
+    // stage per group.  Fewer stages per group (fewer warps busy) when WK
+    // stages of codes and x do not fit twice in shared memory.
     GvLayout L;
-    if (!gv_layout<BITS, NMAT, MTM, NT>(prm.M, row_bytes % 128 == 0 ? kGvKS : 1, nu_max,
-                                        prm.kstages, &L))
-        return cudaErrorInvalidValue;
+    bool fits = false;
+    for (int ks = row_bytes % 128 == 0 ? WK : 1; ks >= 1 && !fits; ks /= 2)
+        fits = gv_layout<BITS, NMAT, MTW, NT, WK>(prm.M, ks, (prm.uq + 1) * prm.chunk, prm.kstages, &L);
+    if (!fits) return cudaErrorInvalidValue;
     prm.ks = L.ks;
     prm.sg = L.sg;
-    prm.s_ring_off = L.s_ring_off;
+    prm.slot_bytes = L.slot_bytes;
+    prm.s_off = L.s_off;
     prm.x_off = L.x_off;
-    prm.x_row = L.x_row;
-    prm.x_nbuf = L.x_nbuf;
     prm.red_off = L.red_off;
     prm.red_nbuf = L.red_nbuf;
     prm.bar_off = L.bar_off;
     // scales by TMA when a scale row is a multiple of 16 bytes
     prm.ssc = (prm.groups * 2) % 16 == 0 ? 1 : 0;
 
-    const size_t ws_bytes = static_cast<size_t>(2) * grid * prm.M * Cfg::kRB * sizeof(float);
+    // partial-tile slots and arrival counters: stream-K only
+    const bool sk = prm.chunk == 1;
+    const size_t ws_bytes = sk ? static_cast<size_t>(2) * grid * prm.M * Cfg::kRB * sizeof(float) : 0;
+    const size_t n_cnt = sk ? static_cast<size_t>(prm.tiles) : 0;
     if (scratch == nullptr) {
-        e = workspace_get(ws_bytes, static_cast<size_t>(prm.tiles), &prm.ws, &prm.cnt);
+        e = workspace_get(ws_bytes, n_cnt, &prm.ws, &prm.cnt);
         if (e != cudaSuccess) return e;
     } else {
-        if (ws_bytes > scratch->ws_bytes || static_cast<size_t>(prm.tiles) > scratch->n_cnt) {
+        if (ws_bytes > scratch->ws_bytes || n_cnt > scratch->n_cnt) {
             if (scratch->too_large) *scratch->too_large = true;
             return cudaErrorInvalidValue;
         }
@@ -637,7 +642,7 @@ static cudaError_t gv_launch(GvParams& prm, const void* const* codes, cudaStream
     // block, 128-byte swizzled like a 2D box).  With one stage per group, a
     // 2D map, whose columns past the row's end read zeros.
     for (int i = 0; i < NMAT; ++i) {
-        const bool ok3 =
+        const bool okw =
             prm.ks > 1
                 ? make_tmap_3d(&prm.tm_w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, codes[i], 128,
                                static_cast<uint64_t>(prm.N), static_cast<uint64_t>(prm.kstages),
@@ -647,7 +652,7 @@ static cudaError_t gv_launch(GvParams& prm, const void* const* codes, cudaStream
                                static_cast<uint64_t>(row_bytes), static_cast<uint64_t>(prm.N),
                                static_cast<uint64_t>(row_bytes), 128, Cfg::kRBM,
                                CU_TENSOR_MAP_SWIZZLE_128B);
-        if (!ok3) return cudaErrorInvalidValue;
+        if (!okw) return cudaErrorInvalidValue;
         if (prm.ssc &&
             !make_tmap_2d(&prm.tm_s[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, prm.scales[i],
                           static_cast<uint64_t>(prm.groups), static_cast<uint64_t>(prm.N),
@@ -655,6 +660,13 @@ static cudaError_t gv_launch(GvParams& prm, const void* const* codes, cudaStream
                           CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
+    // x as {64 k of a group, token, group}: a box is the ks stages' groups
+    // of all M tokens, group-major in shared memory, 128-byte swizzled
+    if (!make_tmap_3d(&prm.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, 64,
+                      static_cast<uint64_t>(prm.M), static_cast<uint64_t>(prm.groups),
+                      static_cast<uint64_t>(prm.K) * 2, 128, 64, static_cast<uint32_t>(prm.M),
+                      static_cast<uint32_t>(prm.ks * Cfg::kGPS), CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -673,65 +685,70 @@ static cudaError_t gv_launch(GvParams& prm, const void* const* codes, cudaStream
     return cudaLaunchKernelEx(&cfg, kern, static_cast<const GvParams&>(prm));
 }
 
-// Rows per matrix in a row tile (16 * MTM): 16 while that gives at most one
-// tile per SM (small projections then run as one wave of whole tiles, no
-// reduction across CTAs); else the largest tile whose whole tiles balance
-// over the SMs (more rows share each x fragment); else 32-row tiles split by
-// stream-K (64 for M > 8, whose x slices are then shared by more rows).
-static int gv_pick_mtm(int N, int M) {
+// Row tile and warp split.  M <= 16: warps split k (WK = 8) and a tile has
+// 16 * MTW rows per matrix: 16 while that gives at most one tile per SM
+// (small projections then run as one wave of whole tiles, no reduction
+// across CTAs); else the tile height whose whole tiles balance best over the
+// SMs, weighted by the unit speed (x fragments shared by more rows); else
+// stream-K.  M > 16: warps split the rows of 128-row tiles (WK = 1), so the
+// x of a stage, large at this M, is loaded once for all 8 warps.
+static int gv_pick_mtw(int N) {
     const int sms = gv_num_sms();
     if ((N + 15) / 16 <= sms) return 1;
-    // relative speed of a warp's unit by m-tiles per unit (x fragments are
-    // shared by more rows), measured on B200: 44 / 47 / 49 weights per cycle
-    // and SM for 1 / 2 / 4 m-tiles
+    // relative speed of a warp's unit by m-tiles per unit, measured on B200:
+    // 44 / 47 / 49 weights per cycle and SM for 1 / 2 / 4 m-tiles
     const double speed[5] = {0.0, 44.0, 47.0, 0.0, 49.0};
     int best = 0;
     double best_score = 0.0;
-    for (int mtm = 4; mtm >= 1; mtm /= 2) {
-        const int tiles = (N + 16 * mtm - 1) / (16 * mtm);
+    for (int mtw = 4; mtw >= 1; mtw /= 2) {
+        const int tiles = (N + 16 * mtw - 1) / (16 * mtw);
         const double bal = gv_tile_balance(tiles, sms);
-        if (bal >= 0.85 && bal * speed[mtm] > best_score) {
-            best = mtm;
-            best_score = bal * speed[mtm];
+        if (bal >= 0.85 && bal * speed[mtw] > best_score) {
+            best = mtw;
+            best_score = bal * speed[mtw];
         }
     }
-    if (best) return best;
-    return M > 8 ? 4 : 2;   // stream-K
+    return best ? best : 2;   // stream-K
 }
 
 template <int BITS, int NMAT, int NT>
-static cudaError_t gv_dispatch_mt(GvParams& prm, const void* const* codes, cudaStream_t s,
-                                  const GemvScratch* sc) {
-    if constexpr (NMAT == 3) {
-        return gv_launch<BITS, 3, 1, NT>(prm, codes, s, sc);
+static cudaError_t gv_dispatch_mt(GvParams& prm, const uint16_t* x, const void* const* codes,
+                                  cudaStream_t s, const GemvScratch* sc) {
+    if constexpr (NT == 4) {
+        // rows split over the warps (x of a stage loaded once for 8 warps) when
+        // whole 128-row tiles balance; else k split with fewer stages per
+        // group (the x of 8 stages of 32 tokens does not fit twice)
+        if (gv_whole_tiles((prm.N + 127) / 128, gv_num_sms()))
+            return gv_launch<BITS, NMAT, 1, 4, 1>(prm, x, codes, s, sc);
+        return gv_launch<BITS, NMAT, 1, 4, 8>(prm, x, codes, s, sc);
+    } else if constexpr (NMAT == 3) {
+        return gv_launch<BITS, 3, 1, NT, 8>(prm, x, codes, s, sc);
     } else {
-        int mtm = gv_pick_mtm(prm.N, prm.M);
-        // large M: the per-warp x buffers leave less room; fall back to fewer rows
-        GvLayout L;
-        if (mtm == 4 && !(gv_layout<BITS, 1, 4, NT>(prm.M, kGvKS, kGvKS, kGvKS, &L) && L.ks == kGvKS))
-            mtm = 2;
-        if (mtm == 2 && !(gv_layout<BITS, 1, 2, NT>(prm.M, kGvKS, kGvKS, kGvKS, &L) && L.ks == kGvKS))
-            mtm = 1;
-        if (mtm == 1) return gv_launch<BITS, 1, 1, NT>(prm, codes, s, sc);
-        if (mtm == 2) return gv_launch<BITS, 1, 2, NT>(prm, codes, s, sc);
-        return gv_launch<BITS, 1, 4, NT>(prm, codes, s, sc);
+        int mtw = gv_pick_mtw(prm.N);
+        // M up to 16 with 8-stage groups: the x of a group (8 stages of M
+        // tokens) shares the slot with the codes; fall back to fewer rows
+        if constexpr (NT == 2)
+            if (mtw > 2) mtw = 2;
+        if (mtw == 1) return gv_launch<BITS, 1, 1, NT, 8>(prm, x, codes, s, sc);
+        if (mtw == 2) return gv_launch<BITS, 1, 2, NT, 8>(prm, x, codes, s, sc);
+        if constexpr (NT == 1) return gv_launch<BITS, 1, 4, NT, 8>(prm, x, codes, s, sc);
+        return cudaErrorInvalidValue;
     }
 }
 
 template <int BITS, int NMAT>
-static cudaError_t gv_dispatch_nt(GvParams& prm, const void* const* codes, cudaStream_t s,
-                                  const GemvScratch* sc) {
+static cudaError_t gv_dispatch_nt(GvParams& prm, const uint16_t* x, const void* const* codes,
+                                  cudaStream_t s, const GemvScratch* sc) {
     // 8 tokens per n-tile
-    if (prm.M <= 8) return gv_dispatch_mt<BITS, NMAT, 1>(prm, codes, s, sc);
-    if (prm.M <= 16) return gv_dispatch_mt<BITS, NMAT, 2>(prm, codes, s, sc);
-    return gv_dispatch_mt<BITS, NMAT, 4>(prm, codes, s, sc);
+    if (prm.M <= 8) return gv_dispatch_mt<BITS, NMAT, 1>(prm, x, codes, s, sc);
+    if (prm.M <= 16) return gv_dispatch_mt<BITS, NMAT, 2>(prm, x, codes, s, sc);
+    return gv_dispatch_mt<BITS, NMAT, 4>(prm, x, codes, s, sc);
 }
 
 static cudaError_t gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
                                 const WOperand* w, int nmat, cudaStream_t s, const GemvScratch* sc) {
     GvParams prm;
     memset(&prm, 0, sizeof(prm));
-    prm.x = x;
     prm.M = static_cast<int>(M);
     prm.N = static_cast<int>(N);
     prm.K = static_cast<int>(K);
@@ -745,10 +762,10 @@ static cudaError_t gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t
         prm.y[i] = w[i].y;
     }
     if (nmat == 3)
-        return bits == 4 ? gv_dispatch_nt<4, 3>(prm, codes, s, sc)
-                         : gv_dispatch_nt<8, 3>(prm, codes, s, sc);
-    return bits == 4 ? gv_dispatch_nt<4, 1>(prm, codes, s, sc)
-                     : gv_dispatch_nt<8, 1>(prm, codes, s, sc);
+        return bits == 4 ? gv_dispatch_nt<4, 3>(prm, x, codes, s, sc)
+                         : gv_dispatch_nt<8, 3>(prm, x, codes, s, sc);
+    return bits == 4 ? gv_dispatch_nt<4, 1>(prm, x, codes, s, sc)
+                     : gv_dispatch_nt<8, 1>(prm, x, codes, s, sc);
 }
 
 cudaError_t launch_gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,

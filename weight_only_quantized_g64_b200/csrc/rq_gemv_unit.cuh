@@ -106,19 +106,23 @@ __device__ __forceinline__ int phys_row(int g) {
 //   sc    scales of the stage, matrix 0: rows of SROW fp16, offset to the
 //         stage's first group (when ssc); matrix m's rows start SMSTR bytes
 //         further per m
-//   xt    x of the stage: per token row (stride x_row) KPS fp16, unswizzled;
-//         xoff[nt] = this thread's row (token nt*8+g, any valid row for
-//         tokens >= M: those columns are never stored) * x_row + 32 t
+//   xt    x of the load group: [groups][M tokens][64 fp16], SWIZZLE_128B
+//         (TMA layout: 128-byte row r's 16-byte chunks permuted by r & 7);
+//         the unit's groups start at group row gq0; xtok[nt] = this thread's
+//         token nt*8+g (any valid token for tokens >= M: those columns of the
+//         MMA are never stored)
 //   prow  phys_row<BITS>(g)
 //   ssc   scales are staged; otherwise read from global memory (ragged K:
-//         groups past the end get scale 0), needing scales/tile/st/N/groups
+//         groups past the end get scale 0), needing scales/row0/st/N/groups,
+//         row0 = the global row of the warp's first m-tile in each matrix
 // The shared-memory operands of QB groups at a time are loaded into registers
 // first (one burst of loads, so their latency is paid once per batch), then
 // the batch is unpacked and multiplied.
 template <int BITS, int MT, int NT, int MTM, int SROW, int SMSTR>
-__device__ __forceinline__ void gv_unit(const uint8_t* wt, int cmstr, const uint8_t* sc, const uint8_t* xt,
-                                        const int (&xoff)[NT], int prow, int t, bool ssc,
-                                        const uint16_t* const* scales, int tile, int st, int N,
+__device__ __forceinline__ void gv_unit(const uint8_t* wt, int cmstr, const uint8_t* sc,
+                                        const uint8_t* xt, int gq0, int M, const int (&xtok)[NT],
+                                        int prow, int t, bool ssc,
+                                        const uint16_t* const* scales, int row0, int st, int N,
                                         int groups, float (&acc)[MT][NT][4]) {
     constexpr int GPS = BITS == 4 ? 4 : 2;
     constexpr bool PERM = BITS == 4 && 2 * MT >= NT;   // permuted pair order (x permuted per group)
@@ -135,9 +139,12 @@ __device__ __forceinline__ void gv_unit(const uint8_t* wt, int cmstr, const uint
             const int q = q0 + qq;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const uint8_t* xp = xt + xoff[nt] + q * 128;
-                xv[qq][nt][0] = lds128(xp);
-                xv[qq][nt][1] = lds128(xp + 16);
+                // positions 16t .. 16t+15 of the group: chunks 2t and 2t+1
+                const int row = (gq0 + q) * M + xtok[nt];
+                const uint8_t* xr = xt + row * 128;
+                const int c0 = ((2 * t) ^ (row & 7)) << 4;
+                xv[qq][nt][0] = lds128(xr + c0);
+                xv[qq][nt][1] = lds128(xr + (c0 ^ 16));
             }
             // this thread's codes of group q in row `prow` of the stage
             // (rows 16i + 8h + prow share the swizzle phase prow & 7)
@@ -187,7 +194,7 @@ __device__ __forceinline__ void gv_unit(const uint8_t* wt, int cmstr, const uint
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int m = i / MTM;
-                    const int n = tile * (16 * MTM) + 16 * (i % MTM) + 8 * h + prow;
+                    const int n = row0 + 16 * (i % MTM) + 8 * h + prow;
                     uint16_t v[QB];
 #pragma unroll
                     for (int qq = 0; qq < QB; ++qq) {

@@ -53,39 +53,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// As mbar_try_wait, but the thread may sleep up to `hint_ns` nanoseconds for
-// the phase to complete (it wakes as soon as it does), so a waiting warp
-// takes no issue slots from the warps that have work.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
-                                                    uint32_t hint_ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
-}
-
 // Bounded wait for the phase of the given parity.  On timeout it raises the
 // library's device status word `status` to RQ_ERR_TIMEOUT, sets *abort_flag
 // (shared memory, so the CTA's other roles stop too) and returns false.  A set
-// *abort_flag also makes it return false at once.  The limit is checked after
-// every sleep of at most 20 us.
+// *abort_flag also makes it return false at once.  (mbarrier.try_wait itself
+// suspends the thread for a while before it reports "not yet".)
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile int* abort_flag, uint64_t limit_ns,
                                           int* status) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
+    uint32_t spins = 0;
     while (true) {
-        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
-        if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > limit_ns) {
-            *abort_flag = 1;
-            if (status) atomicMax(status, 7 /* RQ_ERR_TIMEOUT */);
-            return false;
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((++spins & 63u) == 0u) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                *abort_flag = 1;
+                if (status) atomicMax(status, 7 /* RQ_ERR_TIMEOUT */);
+                return false;
+            }
         }
     }
 }
