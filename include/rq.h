@@ -146,8 +146,10 @@ rq_status rq_gemm_wq(const uint16_t *x, int64_t M, int64_t K, const void *codes,
  * otherwise RQ_ERR_SHAPE is returned and nothing is launched.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current) -- make it before any stream capture.
- * Each call clears the counters it uses (an asynchronous memset on `stream`)
- * and then launches the product.  All calls share the one array: calls that
+ * A call that runs on the row-tile kernel (see rq_set_decode_kernel) clears
+ * the counters it uses (an asynchronous memset on `stream`) and then launches
+ * the product; one that runs on the cluster kernel needs no scratch and
+ * launches only the product.  All calls share the one array: calls that
  * overlap on the GPU (different streams, or several devices' calls mixed
  * without ordering) race with each other and give wrong results.
  */
@@ -165,6 +167,24 @@ rq_status rq_gemv_wq_noalloc(const uint16_t *x, int64_t M, int64_t K, const void
  * call's codes or scales.  Off by default.  Not thread-safe.
  */
 rq_status rq_set_pdl(int enable);
+
+/*
+ * rq_set_decode_kernel -- which kernel computes the decode products
+ * (rq_gemv_wq, rq_gemv_wq_noalloc, rq_rkv_fused) launched afterwards by this
+ * process.  Both compute the same sums (within the products' tolerance; each
+ * is deterministic for a given shape):
+ *   RQ_DECODE_AUTO     (0) chosen per shape and batch size (default);
+ *   RQ_DECODE_ROWTILE  (1) row tiles dealt over the SMs (stream-K), partial
+ *                          tiles summed through a workspace;
+ *   RQ_DECODE_CLUSTER  (2) K split over the CTAs of a thread-block cluster,
+ *                          each CTA's x held in shared memory, partial sums
+ *                          added through distributed shared memory.
+ * Any other value is rejected with RQ_ERR_RANGE.  Not thread-safe.
+ */
+#define RQ_DECODE_AUTO 0
+#define RQ_DECODE_ROWTILE 1
+#define RQ_DECODE_CLUSTER 2
+rq_status rq_set_decode_kernel(int kernel);
 
 /*
  * rq_set_wait_limit_ns -- time limit of every bounded on-chip wait of the

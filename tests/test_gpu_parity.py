@@ -105,30 +105,37 @@ def product_case(N, K, bits, M, seed, massive=None):
     return x, codes, scales
 
 
+DECODE_KERNELS = ["rowtile", "cluster"]
+
+
+@pytest.mark.parametrize("kernel", DECODE_KERNELS)
 @pytest.mark.parametrize("bits", [4, 8])
-@pytest.mark.parametrize("M", [1, 2, 3, 8, 16, 17, 31, 32])
-@pytest.mark.parametrize("N,K", [(300, 640), (1, 64), (129, 128), (256, 2048)])
-def test_gemv_parity(bits, M, N, K):
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16, 17, 31, 32])
+@pytest.mark.parametrize("N,K", [(300, 640), (1, 64), (129, 128), (256, 2048), (390, 1792), (256, 16384)])
+def test_gemv_parity(kernel, bits, M, N, K):
     x, codes, scales = product_case(N, K, bits, M, seed=1000 + M + N + K)
     cd, sd = upload(codes, scales)
-    y = rq.gemv_wq(x, cd, sd, N, bits)
+    with rq.decode_kernel(kernel):
+        y = rq.gemv_wq(x, cd, sd, N, bits)
     torch.cuda.synchronize()
     y_ref, bound = oracle.matmul(to_host(x), codes, scales, bits)
-    check_close(to_host(y), y_ref, bound, f"gemv bits={bits} M={M} N={N} K={K}")
+    check_close(to_host(y), y_ref, bound, f"gemv {kernel} bits={bits} M={M} N={N} K={K}")
 
 
+@pytest.mark.parametrize("kernel", DECODE_KERNELS)
 @pytest.mark.parametrize("bits", [4, 8])
-@pytest.mark.parametrize("M", [1, 8, 32])
-def test_rkv_fused_parity(bits, M):
-    N, K = 200, 512
+@pytest.mark.parametrize("M", [1, 8, 13, 32])
+@pytest.mark.parametrize("N,K", [(200, 512), (256, 2048)])
+def test_rkv_fused_parity(kernel, bits, M, N, K):
     cases = [product_case(N, K, bits, M, seed=2000 + i) for i in range(3)]
     x = cases[0][0]
     ws = [upload(c[1], c[2]) for c in cases]
-    ys = rq.rkv_fused(x, ws[0], ws[1], ws[2], N, bits)
+    with rq.decode_kernel(kernel):
+        ys = rq.rkv_fused(x, ws[0], ws[1], ws[2], N, bits)
     torch.cuda.synchronize()
     for i in range(3):
         y_ref, bound = oracle.matmul(to_host(x), cases[i][1], cases[i][2], bits)
-        check_close(to_host(ys[i]), y_ref, bound, f"rkv[{i}] bits={bits} M={M}")
+        check_close(to_host(ys[i]), y_ref, bound, f"rkv[{i}] {kernel} bits={bits} M={M} N={N} K={K}")
 
 
 @pytest.mark.parametrize("bits", [4, 8])
@@ -210,8 +217,9 @@ def quantize_checked(W, bits, sample_rows=64, seed=0):
     return codes, scales
 
 
+@pytest.mark.parametrize("kernel", DECODE_KERNELS)
 @pytest.mark.parametrize("wl", [1, 2, 3, 5])
-def test_decode_workload_shapes(wl):
+def test_decode_workload_shapes(kernel, wl):
     w = synth.WORKLOADS[wl]
     for pi, pj in enumerate(w.projs):
         W = synth.weights(pj.N, pj.K, seed=synth.seed_for(wl, 0, pi), device="cuda")
@@ -220,12 +228,14 @@ def test_decode_workload_shapes(wl):
         for M in w.Ms:
             x = synth.activations(M, pj.K, seed=synth.seed_for(wl, 0, pi) + M, device="cuda",
                                   massive_channel=w.massive_channel)
-            y = rq.gemv_wq(x, codes, scales, pj.N, w.bits)
+            with rq.decode_kernel(kernel):
+                y = rq.gemv_wq(x, codes, scales, pj.N, w.bits)
             torch.cuda.synchronize()
             sampled_check(y, x, codes, scales, pj.N, pj.K, w.bits, seed=M)
 
 
-def test_decode_workload_rkv_fused():
+@pytest.mark.parametrize("kernel", DECODE_KERNELS)
+def test_decode_workload_rkv_fused(kernel):
     for wl in (2, 3, 5):
         w = synth.WORKLOADS[wl]
         D = w.projs[0].N
@@ -236,7 +246,8 @@ def test_decode_workload_rkv_fused():
             del W
         for M in (w.Ms[0], w.Ms[-1]):
             x = synth.activations(M, D, seed=M, device="cuda", massive_channel=w.massive_channel)
-            ys = rq.rkv_fused(x, ws[0], ws[1], ws[2], D, w.bits)
+            with rq.decode_kernel(kernel):
+                ys = rq.rkv_fused(x, ws[0], ws[1], ws[2], D, w.bits)
             torch.cuda.synchronize()
             for i in range(3):
                 sampled_check(ys[i], x, ws[i][0], ws[i][1], D, D, w.bits, n_samples=256, seed=i)
@@ -274,24 +285,25 @@ def test_bounded_wait_times_out_cleanly():
     assert rq.read_device_status() == rq.OK
 
 
-def test_pdl_chain_matches():
+@pytest.mark.parametrize("kernel,M", [("rowtile", 4), ("cluster", 4), ("cluster", 24)])
+def test_pdl_chain_matches(kernel, M):
     """With programmatic dependent launch on, a chain of dependent products
     (each reading the previous output as its input) still matches."""
     N = K = 512
     bits = 4
-    M = 4
     W = [synth.weights(N, K, seed=40 + i, device="cuda") for i in range(3)]
     qs = [rq.quantize_g64(w, bits) for w in W]
     torch.cuda.synchronize()
     x0 = synth.activations(M, K, seed=40, device="cuda")
     rq.set_pdl(True)
     try:
-        x = x0
-        outs = []
-        for c, s in qs:
-            y = rq.gemv_wq(x, c, s, N, bits)
-            x = (y * 0.05).to(torch.float16)   # torch op between: still ordered
-            outs.append(y)
+        with rq.decode_kernel(kernel):
+            x = x0
+            outs = []
+            for c, s in qs:
+                y = rq.gemv_wq(x, c, s, N, bits)
+                x = (y * 0.05).to(torch.float16)   # torch op between: still ordered
+                outs.append(y)
         torch.cuda.synchronize()
     finally:
         rq.set_pdl(False)
@@ -305,22 +317,26 @@ def test_pdl_chain_matches():
 
 # ------------------------------------------------------------ repeatability ---
 
-@pytest.mark.parametrize("path", ["gemv", "gemm"])
+@pytest.mark.parametrize("path", ["gemv", "gemv-cluster", "gemv-cluster-m32", "gemm"])
 def test_repeat_runs_bit_identical(path):
     """Both kernels sum in a fixed order, so repeated runs must agree bit for
     bit; a pipeline race (a stage read before or after its data) shows up here
     even when it stays within tolerance."""
-    if path == "gemv":
-        N, K, M, bits = 4096, 4096, 5, 4
-    else:
+    kernel = "cluster" if path.startswith("gemv-cluster") else "rowtile"
+    if path == "gemm":
         N, K, M, bits = 1024, 8192, 512, 4
+    elif path == "gemv-cluster-m32":
+        N, K, M, bits = 2048, 8192, 32, 4
+    else:
+        N, K, M, bits = 4096, 4096, 5, 4
     W = synth.weights(N, K, seed=31, device="cuda")
     codes, scales = rq.quantize_g64(W, bits)
     x = synth.activations(M, K, seed=31, device="cuda")
-    fn = rq.gemv_wq if path == "gemv" else rq.gemm_wq
-    ref = fn(x, codes, scales, N, bits)
-    torch.cuda.synchronize()
-    for _ in range(20):
-        y = fn(x, codes, scales, N, bits)
+    fn = rq.gemm_wq if path == "gemm" else rq.gemv_wq
+    with rq.decode_kernel(kernel):
+        ref = fn(x, codes, scales, N, bits)
         torch.cuda.synchronize()
-        assert torch.equal(y, ref)
+        for _ in range(20):
+            y = fn(x, codes, scales, N, bits)
+            torch.cuda.synchronize()
+            assert torch.equal(y, ref)

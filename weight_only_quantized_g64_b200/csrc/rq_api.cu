@@ -37,6 +37,22 @@ int* device_status_ptr() {
 uint64_t wait_limit_ns() { return g_wait_limit_ns; }
 bool pdl_enabled() { return g_pdl; }
 
+static int g_decode_kernel = RQ_DECODE_AUTO;
+
+int decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat) {
+    const bool fits = gemv_cluster_fits(M, K, bits);
+    if (g_decode_kernel == RQ_DECODE_CLUSTER) return fits ? RQ_DECODE_CLUSTER : -1;
+    if (g_decode_kernel == RQ_DECODE_ROWTILE) return RQ_DECODE_ROWTILE;
+    // measured on B200 (graph-replayed chains, int4): the cluster kernel is
+    // ahead for M > 16 on every projection shape, and for M 9..16 on tall
+    // ones (>= 6144 rows per launch, K <= 4096); the row-tile kernel
+    // elsewhere
+    if (!fits || M <= 8) return RQ_DECODE_ROWTILE;
+    if (M > 16 || (static_cast<int64_t>(nmat) * N >= 6144 && K <= 4096)) return RQ_DECODE_CLUSTER;
+    return RQ_DECODE_ROWTILE;
+}
+
+
 // ------------------------------------------------------------- workspace --
 struct Workspace {
     float* ws = nullptr;
@@ -191,6 +207,15 @@ static rq_status check_operand(const void* codes, const uint16_t* scales, const 
     return RQ_OK;
 }
 
+static rq_status launch_decode(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
+                               const WOperand* w, int nmat, cudaStream_t s) {
+    const int which = decode_kernel_for(M, K, N, bits, nmat);
+    if (which < 0) return RQ_ERR_SHAPE;
+    const cudaError_t e = which == RQ_DECODE_CLUSTER ? launch_gemv_cluster(x, M, K, N, bits, w, nmat, s)
+                                                     : launch_gemv_product(x, M, K, N, bits, w, nmat, s);
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
 extern "C" {
 
 size_t rq_codes_bytes(int64_t N, int64_t K, int bits) {
@@ -221,8 +246,7 @@ rq_status rq_gemv_wq(const uint16_t* x, int64_t M, int64_t K, const void* codes,
     if (st != RQ_OK) return st;
     if ((st = check_operand(codes, scales, y)) != RQ_OK) return st;
     WOperand w = {codes, scales, y};
-    cudaError_t e = launch_gemv_product(x, M, K, N, bits, &w, 1, reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+    return launch_decode(x, M, K, N, bits, &w, 1, reinterpret_cast<cudaStream_t>(stream));
 }
 
 rq_status rq_rkv_fused(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
@@ -235,8 +259,7 @@ rq_status rq_rkv_fused(const uint16_t* x, int64_t M, int64_t K, int64_t N, int b
     if ((st = check_operand(codes_k, scales_k, y_k)) != RQ_OK) return st;
     if ((st = check_operand(codes_v, scales_v, y_v)) != RQ_OK) return st;
     WOperand w[3] = {{codes_r, scales_r, y_r}, {codes_k, scales_k, y_k}, {codes_v, scales_v, y_v}};
-    cudaError_t e = launch_gemv_product(x, M, K, N, bits, w, 3, reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+    return launch_decode(x, M, K, N, bits, w, 3, reinterpret_cast<cudaStream_t>(stream));
 }
 
 rq_status rq_gemm_wq(const uint16_t* x, int64_t M, int64_t K, const void* codes,
@@ -252,6 +275,13 @@ rq_status rq_gemm_wq(const uint16_t* x, int64_t M, int64_t K, const void* codes,
 
 rq_status rq_set_pdl(int enable) {
     g_pdl = enable != 0;
+    return RQ_OK;
+}
+
+rq_status rq_set_decode_kernel(int kernel) {
+    if (kernel != RQ_DECODE_AUTO && kernel != RQ_DECODE_ROWTILE && kernel != RQ_DECODE_CLUSTER)
+        return RQ_ERR_RANGE;
+    g_decode_kernel = kernel;
     return RQ_OK;
 }
 

@@ -99,6 +99,77 @@ __device__ __forceinline__ int phys_row(int g) {
 }
 
 
+// The math of one group of 64 k for one warp: x fragments xv[nt] (positions
+// 16t .. 16t+15 of token nt*8+g, two 16-byte chunks), code words cw[i][h]
+// (this thread's 16 k of row 8h + g of m-tile i) and fp32 scales sv[i][h].
+// Codes become exact fp16 A registers, 4 MMA steps per n-tile sum x * code in
+// fp32, and the group's scale is applied in fp32.
+template <int BITS, int MT, int NT>
+__device__ __forceinline__ void gv_group_math(const uint4 (&xv)[NT][2],
+                                              const uint32_t (&cw)[MT][2][BITS == 4 ? 2 : 4],
+                                              const float (&sv)[MT][2], float (&acc)[MT][NT][4]) {
+    constexpr bool PERM = BITS == 4 && 2 * MT >= NT;   // permuted pair order (x permuted per group)
+    // x fragments of this group: token nt*8+g, positions 16t .. 16t+15
+    uint32_t b[NT][4][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t X[8] = {xv[nt][0].x, xv[nt][0].y, xv[nt][0].z, xv[nt][0].w,
+                               xv[nt][1].x, xv[nt][1].y, xv[nt][1].z, xv[nt][1].w};
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            if constexpr (PERM) {
+                // step jj pairs (p0,p4),(p1,p5) or (p2,p6),(p3,p7) of word jj/2
+                const int wb = (jj >> 1) * 4 + (jj & 1);
+                b[nt][jj][0] = __byte_perm(X[wb], X[wb + 2], 0x5410);
+                b[nt][jj][1] = __byte_perm(X[wb], X[wb + 2], 0x7632);
+            } else {
+                b[nt][jj][0] = X[2 * jj];
+                b[nt][jj][1] = X[2 * jj + 1];
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < MT; ++i) {
+        uint32_t A[4][4];   // [step][a-reg]
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            if constexpr (BITS == 4) {
+                uint32_t P0[4], P1[4];
+                if constexpr (PERM) {
+                    i4_word_to_pairs_perm(cw[i][h][0], P0);
+                    i4_word_to_pairs_perm(cw[i][h][1], P1);
+                } else {
+                    i4_word_to_pairs_nat(cw[i][h][0], P0);
+                    i4_word_to_pairs_nat(cw[i][h][1], P1);
+                }
+                // step jj: a0a1 (h = 0) / a2a3 (h = 1), and a4a5 / a6a7
+                A[0][h] = P0[0]; A[0][h + 2] = P0[1];
+                A[1][h] = P0[2]; A[1][h + 2] = P0[3];
+                A[2][h] = P1[0]; A[2][h + 2] = P1[1];
+                A[3][h] = P1[2]; A[3][h + 2] = P1[3];
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    uint32_t Q[2];
+                    i8_word_to_pairs(cw[i][h][jj], Q);
+                    A[jj][h] = Q[0];
+                    A[jj][h + 2] = Q[1];
+                }
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float part[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) mma16816(part, A[jj], b[nt][jj][0], b[nt][jj][1], jj == 0);
+            acc[i][nt][0] = fmaf(part[0], sv[i][0], acc[i][nt][0]);
+            acc[i][nt][1] = fmaf(part[1], sv[i][0], acc[i][nt][1]);
+            acc[i][nt][2] = fmaf(part[2], sv[i][1], acc[i][nt][2]);
+            acc[i][nt][3] = fmaf(part[3], sv[i][1], acc[i][nt][3]);
+        }
+    }
+}
+
 // One unit of one warp.  MT = NMAT * MTM m-tiles: m-tile i is rows
 // [16 (i % MTM), +16) of matrix i / MTM.
 //   wt    codes of the stage, matrix 0: [16*MTM rows][128 B], SWIZZLE_128B
@@ -125,7 +196,6 @@ __device__ __forceinline__ void gv_unit(const uint8_t* wt, int cmstr, const uint
                                         const uint16_t* const* scales, int row0, int st, int N,
                                         int groups, float (&acc)[MT][NT][4]) {
     constexpr int GPS = BITS == 4 ? 4 : 2;
-    constexpr bool PERM = BITS == 4 && 2 * MT >= NT;   // permuted pair order (x permuted per group)
     constexpr int CW = BITS == 4 ? 2 : 4;              // code words per row and group
     constexpr int QB = MT * NT <= 2 ? GPS : (MT * NT <= 4 ? 2 : 1);   // groups per load batch
 #pragma unroll
@@ -212,77 +282,87 @@ __device__ __forceinline__ void gv_unit(const uint8_t* wt, int cmstr, const uint
         // ---------------------------------------------------- math --------
 #pragma unroll
         for (int qq = 0; qq < QB; ++qq) {
-            // x fragments of this group: token nt*8+g, positions 16t .. 16t+15
-            uint32_t b[NT][4][2];
+            float sv[MT][2];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const uint32_t X[8] = {xv[qq][nt][0].x, xv[qq][nt][0].y, xv[qq][nt][0].z,
-                                       xv[qq][nt][0].w, xv[qq][nt][1].x, xv[qq][nt][1].y,
-                                       xv[qq][nt][1].z, xv[qq][nt][1].w};
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    if constexpr (PERM) {
-                        // step jj pairs (p0,p4),(p1,p5) or (p2,p6),(p3,p7) of word jj/2
-                        const int wb = (jj >> 1) * 4 + (jj & 1);
-                        b[nt][jj][0] = __byte_perm(X[wb], X[wb + 2], 0x5410);
-                        b[nt][jj][1] = __byte_perm(X[wb], X[wb + 2], 0x7632);
-                    } else {
-                        b[nt][jj][0] = X[2 * jj];
-                        b[nt][jj][1] = X[2 * jj + 1];
-                    }
-                }
-            }
-            // per m-tile: codes -> exact fp16 A registers, 4 MMA steps per
-            // n-tile, the group's scale in fp32
-#pragma unroll
-            for (int i = 0; i < MT; ++i) {
-                float sv[2];
+            for (int i = 0; i < MT; ++i)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const uint32_t w2 = sw[i][h][qq >> 1];
-                    sv[h] = __half2float(__ushort_as_half(
+                    sv[i][h] = __half2float(__ushort_as_half(
                         static_cast<unsigned short>((qq & 1) ? (w2 >> 16) : (w2 & 0xFFFFu))));
                 }
-                uint32_t A[4][4];   // [step][a-reg]
+            gv_group_math<BITS, MT, NT>(xv[qq], cw[qq], sv, acc);
+        }
+    }
+}
+
+// One warp's share of one stage when WK warps split the stage's groups:
+// groups q = kw, kw + WK, ... of the stage (GPS / WK of them).  Operands as
+// for gv_unit with one matrix (MTM = MT); scales, when staged, are rows of
+// SROW fp16 starting at the stage's first group.
+template <int BITS, int MT, int NT, int WK, int SROW>
+__device__ __forceinline__ void gv_unit_strided(const uint8_t* wt, const uint8_t* sc,
+                                                const uint8_t* xt, int gq0, int kw, int M,
+                                                const int (&xtok)[NT], int prow, int t, bool ssc,
+                                                const uint16_t* scales, int row0, int st, int N,
+                                                int groups, float (&acc)[MT][NT][4]) {
+    constexpr int GPS = BITS == 4 ? 4 : 2;
+    constexpr int NQ = GPS / WK;                       // groups of the stage for this warp
+    constexpr int CW = BITS == 4 ? 2 : 4;
+    constexpr int QB = NQ < 2 ? NQ : (MT * NT <= 4 ? 2 : 1);
+    static_assert(GPS % WK == 0 && NQ % QB == 0, "warps must split the stage's groups evenly");
+#pragma unroll
+    for (int qb = 0; qb < NQ; qb += QB) {
+        uint4 xv[QB][NT][2];
+        uint32_t cw[QB][MT][2][CW];
+        float sv[QB][MT][2];
+#pragma unroll
+        for (int qq = 0; qq < QB; ++qq) {
+            const int q = kw + WK * (qb + qq);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int row = (gq0 + q) * M + xtok[nt];
+                const uint8_t* xr = xt + row * 128;
+                const int c0 = ((2 * t) ^ (row & 7)) << 4;
+                xv[qq][nt][0] = lds128(xr + c0);
+                xv[qq][nt][1] = lds128(xr + (c0 ^ 16));
+            }
+            int coff;
+            if constexpr (BITS == 4)
+                coff = prow * 128 + (((2 * q + (t >> 1)) ^ (prow & 7)) << 4) + ((t & 1) << 3);
+            else
+                coff = prow * 128 + (((4 * q + t) ^ (prow & 7)) << 4);
+#pragma unroll
+            for (int i = 0; i < MT; ++i)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
+                    const uint8_t* cp = wt + coff + (16 * i + 8 * h) * 128;
                     if constexpr (BITS == 4) {
-                        uint32_t P0[4], P1[4];
-                        if constexpr (PERM) {
-                            i4_word_to_pairs_perm(cw[qq][i][h][0], P0);
-                            i4_word_to_pairs_perm(cw[qq][i][h][1], P1);
-                        } else {
-                            i4_word_to_pairs_nat(cw[qq][i][h][0], P0);
-                            i4_word_to_pairs_nat(cw[qq][i][h][1], P1);
-                        }
-                        // step jj: a0a1 (h = 0) / a2a3 (h = 1), and a4a5 / a6a7
-                        A[0][h] = P0[0]; A[0][h + 2] = P0[1];
-                        A[1][h] = P0[2]; A[1][h + 2] = P0[3];
-                        A[2][h] = P1[0]; A[2][h + 2] = P1[1];
-                        A[3][h] = P1[2]; A[3][h + 2] = P1[3];
+                        const uint2 v = lds64(cp);
+                        cw[qq][i][h][0] = v.x;
+                        cw[qq][i][h][1] = v.y;
                     } else {
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            uint32_t Q[2];
-                            i8_word_to_pairs(cw[qq][i][h][jj], Q);
-                            A[jj][h] = Q[0];
-                            A[jj][h + 2] = Q[1];
-                        }
+                        const uint4 v = lds128(cp);
+                        cw[qq][i][h][0] = v.x; cw[qq][i][h][1] = v.y;
+                        cw[qq][i][h][2] = v.z; cw[qq][i][h][3] = v.w;
                     }
+                    uint16_t s16;
+                    if (ssc) {
+                        s16 = *reinterpret_cast<const uint16_t*>(
+                            sc + ((16 * i + 8 * h + prow) * SROW + q) * 2);
+                    } else {
+                        // ragged K: the stage may run past the last group (scale 0)
+                        const int n = row0 + 16 * i + 8 * h + prow;
+                        const int grp = st * GPS + q;
+                        s16 = (n < N && grp < groups)
+                                  ? __ldg(scales + static_cast<int64_t>(n) * groups + grp)
+                                  : static_cast<uint16_t>(0);
+                    }
+                    sv[qq][i][h] = __half2float(__ushort_as_half(s16));
                 }
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    float part[4];
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-                        mma16816(part, A[jj], b[nt][jj][0], b[nt][jj][1], jj == 0);
-                    acc[i][nt][0] = fmaf(part[0], sv[0], acc[i][nt][0]);
-                    acc[i][nt][1] = fmaf(part[1], sv[0], acc[i][nt][1]);
-                    acc[i][nt][2] = fmaf(part[2], sv[1], acc[i][nt][2]);
-                    acc[i][nt][3] = fmaf(part[3], sv[1], acc[i][nt][3]);
-                }
-            }
         }
+#pragma unroll
+        for (int qq = 0; qq < QB; ++qq) gv_group_math<BITS, MT, NT>(xv[qq], cw[qq], sv[qq], acc);
     }
 }
 

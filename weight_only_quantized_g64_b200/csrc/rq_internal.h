@@ -34,6 +34,20 @@ cudaError_t launch_tc_product(const uint16_t* x, int64_t M, int64_t K, int64_t N
 cudaError_t launch_gemv_product(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
                                 const WOperand* w, int nmat, cudaStream_t s);
 
+// Decode product (M <= 32), K split over the CTAs of a cluster, partial sums
+// added through distributed shared memory.  Needs no workspace.
+cudaError_t launch_gemv_cluster(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
+                                const WOperand* w, int nmat, cudaStream_t s);
+
+// Whether the cluster kernel's shared memory holds a product with this M and
+// K (each CTA keeps the x of its K range on chip).
+bool gemv_cluster_fits(int64_t M, int64_t K, int bits);
+
+// The decode kernel a product of this shape runs on: RQ_DECODE_ROWTILE or
+// RQ_DECODE_CLUSTER (the selection of rq_set_decode_kernel, or the automatic
+// choice), or -1 when the selected cluster kernel cannot take the shape.
+int decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat);
+
 // Caller-provided scratch for the decode product instead of the library's
 // workspace: partial-tile slots (ws, ws_bytes) and per-tile counters (cnt,
 // n_cnt, zero between launches).  If a launch would need more, nothing is

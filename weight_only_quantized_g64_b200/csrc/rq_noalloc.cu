@@ -74,6 +74,20 @@ extern "C" rq_status rq_gemv_wq_noalloc(const uint16_t* x, int64_t M, int64_t K,
     const int64_t tiles = (N + 31) / 32;
     if (tiles > static_cast<int64_t>(kMaxTiles)) return RQ_ERR_SHAPE;
 
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    WOperand w = {codes, scales, y};
+    const int which = decode_kernel_for(M, K, N, bits, 1);
+    if (which < 0) return RQ_ERR_SHAPE;
+    if (which == RQ_DECODE_CLUSTER) {
+        // the cluster kernel keeps its partial sums on chip: no scratch at all
+        cudaError_t ec = launch_gemv_cluster(x, M, K, N, bits, &w, 1, s);
+        if (ec != cudaSuccess) {
+            record_cuda_error(ec);
+            return RQ_ERR_CUDA;
+        }
+        return RQ_OK;
+    }
+
     unsigned char* base = nullptr;
     cudaError_t e = scratch_address(&base);
     if (e != cudaSuccess) {
@@ -82,7 +96,6 @@ extern "C" rq_status rq_gemv_wq_noalloc(const uint16_t* x, int64_t M, int64_t K,
     }
     float* ws = reinterpret_cast<float*>(base);
     int* cnt = reinterpret_cast<int*>(base + kSlotBytes);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // The counters must start at zero; a completed launch leaves them at zero,
     // an aborted one might not, so clear the ones this call uses.
     // (row tiles are 16 to 64 rows: clear enough counters for the smallest)
@@ -95,7 +108,6 @@ extern "C" rq_status rq_gemv_wq_noalloc(const uint16_t* x, int64_t M, int64_t K,
     }
     bool too_large = false;
     GemvScratch sc = {ws, kSlotBytes, cnt, kMaxTiles, &too_large};
-    WOperand w = {codes, scales, y};
     e = launch_gemv_product_scratch(x, M, K, N, bits, &w, 1, s, &sc);
     if (too_large) return RQ_ERR_SHAPE;
     if (e != cudaSuccess) {

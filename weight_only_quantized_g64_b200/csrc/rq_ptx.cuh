@@ -53,6 +53,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase has not completed is suspended
+// until it completes or about suspend_ns nanoseconds pass, so waiting warps
+// leave the issue slots to the warps that work.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity,
+                                                      uint32_t suspend_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase of the given parity.  On timeout it raises the
 // library's device status word `status` to RQ_ERR_TIMEOUT, sets *abort_flag
 // (shared memory, so the CTA's other roles stop too) and returns false.  A set
@@ -73,6 +89,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                 if (status) atomicMax(status, 7 /* RQ_ERR_TIMEOUT */);
                 return false;
             }
+        }
+    }
+}
+
+// Bounded wait as mbar_wait, suspending between checks (mbar_try_wait_suspend)
+// instead of spinning.
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag, uint64_t limit_ns,
+                                                  int* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            if (status) atomicMax(status, 7 /* RQ_ERR_TIMEOUT */);
+            return false;
         }
     }
 }
@@ -284,10 +318,54 @@ __device__ __forceinline__ void cluster_sync() {
                      : "memory");
 }
 
+// Split cluster barrier: arrive (no ordering of earlier memory operations)
+// and wait.  Every thread of every CTA in the cluster executes both, in order.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// Asynchronous stores into the shared memory of a CTA of the cluster (caddr
+// and the barrier are shared::cluster addresses of that CTA): the bytes are
+// counted on that CTA's mbarrier as they land.
+__device__ __forceinline__ void st_async_f32x2(uint32_t caddr, float a, float b, uint32_t cbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
+                 ::"r"(caddr), "f"(a), "f"(b), "r"(cbar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_f32(uint32_t caddr, float a, uint32_t cbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];"
+                 ::"r"(caddr), "f"(a), "r"(cbar)
+                 : "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from this CTA's shared memory into the shared memory of a CTA of the
+// cluster (dst and the barrier are shared::cluster addresses of that CTA);
+// the bytes are counted on that CTA's mbarrier as they land.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_caddr, const void* src,
+                                                  uint32_t bytes, uint32_t cbar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst_caddr), "r"(smem_u32(src)), "r"(bytes), "r"(cbar)
+        : "memory");
+}
+
 __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
+}
+
+// Plain store of 16 bytes into the shared memory of a CTA of the cluster
+// (caddr: shared::cluster address); made visible by a release/acquire
+// cluster barrier.
+__device__ __forceinline__ void st_dsmem_f32x4(uint32_t caddr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
+                 ::"r"(caddr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
 }
 
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t caddr) {

@@ -22,6 +22,7 @@ MAX_DECODE_M = 32
 STATUS = {0: "RQ_OK", 1: "RQ_ERR_NULL", 2: "RQ_ERR_BITS", 3: "RQ_ERR_SHAPE", 4: "RQ_ERR_ALIGN",
           5: "RQ_ERR_NONFINITE", 6: "RQ_ERR_RANGE", 7: "RQ_ERR_TIMEOUT", 8: "RQ_ERR_CUDA"}
 OK, ERR_NULL, ERR_BITS, ERR_SHAPE, ERR_ALIGN, ERR_NONFINITE, ERR_RANGE, ERR_TIMEOUT, ERR_CUDA = range(9)
+DECODE_KERNELS = {"auto": 0, "rowtile": 1, "cluster": 2}
 
 _lib = None
 
@@ -61,6 +62,8 @@ def lib():
     L.rq_rkv_fused.restype = i32
     L.rq_set_pdl.argtypes = [i32]
     L.rq_set_pdl.restype = i32
+    L.rq_set_decode_kernel.argtypes = [i32]
+    L.rq_set_decode_kernel.restype = i32
     L.rq_set_wait_limit_ns.argtypes = [u64]
     L.rq_set_wait_limit_ns.restype = i32
     L.rq_read_device_status.argtypes = [ctypes.POINTER(ctypes.c_int), i32]
@@ -168,6 +171,26 @@ def rkv_fused(x: torch.Tensor, wr, wk, wv, N: int, bits: int, ys=None, stream=No
 
 def set_pdl(enable: bool):
     _check(lib().rq_set_pdl(1 if enable else 0), "rq_set_pdl")
+
+
+def set_decode_kernel(kind: str):
+    """Decode kernel for later products: "auto", "rowtile" or "cluster"."""
+    _check(lib().rq_set_decode_kernel(DECODE_KERNELS[kind]), "rq_set_decode_kernel")
+
+
+class decode_kernel:
+    """Context manager: run the enclosed decode products on one kernel."""
+
+    def __init__(self, kind: str):
+        self.kind = kind
+
+    def __enter__(self):
+        set_decode_kernel(self.kind)
+        return self
+
+    def __exit__(self, *exc):
+        set_decode_kernel("auto")
+        return False
 
 
 def set_wait_limit_ns(ns: int):

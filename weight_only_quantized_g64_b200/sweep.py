@@ -38,9 +38,14 @@ def main(argv=None):
     ap.add_argument("--iters", type=int, default=200)
     ap.add_argument("--pdl", default="1", help="comma list of 0/1")
     ap.add_argument("--once", action="store_true")
+    ap.add_argument("--decode-kernel", default="auto", choices=sorted(rq.DECODE_KERNELS),
+                    help="kernel of the decode products (M <= 32)")
+    ap.add_argument("--product", default="auto", choices=("auto", "gemm"),
+                    help="gemm: time rq_gemm_wq at every M (single projections only)")
     a = ap.parse_args(argv)
     rq_build.build()
     rq.lib()
+    rq.set_decode_kernel(a.decode_kernel)
     for sh in a.shapes.split(","):
         nmat, N, K = parse_shape(sh)
         per = synth.algorithmic_weight_bytes(N, K, a.bits) * nmat
@@ -55,12 +60,19 @@ def main(argv=None):
             x = synth.activations(M, K, seed=synth.seed_for(9, 0, 1), device="cuda")
             ys = [torch.empty((M, N), dtype=torch.float32, device="cuda") for _ in range(3)]
 
+            if nmat == 3:
+                kind = "rkv_fused"
+            elif M <= rq.MAX_DECODE_M and a.product == "auto":
+                kind = "gemv_wq"
+            else:
+                kind = "gemm_wq"
+
             def run():
                 for i in range(copies):
                     if nmat == 3:
                         j = [(i + t) % nw for t in range(3)]
                         rq.rkv_fused(x, ws[j[0]], ws[j[1]], ws[j[2]], N, a.bits, ys=ys)
-                    elif M <= rq.MAX_DECODE_M:
+                    elif M <= rq.MAX_DECODE_M and a.product == "auto":
                         rq.gemv_wq(x, ws[i][0], ws[i][1], N, a.bits, y=ys[0])
                     else:
                         rq.gemm_wq(x, ws[i][0], ws[i][1], N, a.bits, y=ys[0])
@@ -87,6 +99,7 @@ def main(argv=None):
                 torch.cuda.synchronize()
                 ms = e0.elapsed_time(e1) / (reps * copies)
                 print(json.dumps({"shape": sh, "M": M, "bits": a.bits, "pdl": pdl,
+                                  "product": kind, "decode_kernel": a.decode_kernel,
                                   "us": ms * 1e3, "GB/s": per / ms / 1e6, "MB": per / 1e6}),
                       flush=True)
                 del g
