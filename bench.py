@@ -39,22 +39,31 @@ METRIC = "decode w4g64 GEMV weight GB/s (% of B200 HBM peak); prefill TFLOP/s; 1
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# DRAM traffic of the decode kernel, from one ncu launch list of a timed step
+# DRAM traffic of the decode kernels, from one ncu launch list of a timed step
 # (dram__bytes_read.sum + dram__bytes_write.sum over the step's 480 launches,
 # averaged per launch; profiles/launches_decode_1p5b_int4_24layers.md).  It
-# is valid only for the kernel sources it was taken on: when their hash
-# differs, the bench reports traffic as null until a new capture is taken.
-DECODE_SOURCES = ("rq_gemv.cu", "rq_gemv_unit.cuh", "rq_ptx.cuh", "rq_internal.h")
-DECODE_TRAFFIC = {"sources_sha256_16": "f619bba85e6c0a06", "bytes_per_launch": 6827551}
+# is valid only for the kernel code it was taken on: when the code's hash
+# (comments and whitespace ignored) differs, the bench reports traffic as null
+# until a new capture is taken.
+DECODE_SOURCES = ("rq_api.cu", "rq_gemv.cu", "rq_gemv_ck.cu", "rq_gemv_unit.cuh", "rq_ptx.cuh",
+                  "rq_internal.h")
+DECODE_TRAFFIC = {"code_sha256_16": "3119f9017d25c7f4", "bytes_per_launch": 6823801}
+
+
+def decode_code_hash():
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "weight_only_quantized_g64_b200", "csrc", f)) as fh:
+            text = fh.read()
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update("".join(text.split()).encode())
+    return h.hexdigest()[:16]
 
 
 def decode_traffic():
-    import hashlib
-    h = hashlib.sha256()
-    for f in DECODE_SOURCES:
-        with open(os.path.join(ROOT, "weight_only_quantized_g64_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    if h.hexdigest()[:16] != DECODE_TRAFFIC["sources_sha256_16"]:
+    if decode_code_hash() != DECODE_TRAFFIC["code_sha256_16"]:
         return None
     return DECODE_TRAFFIC["bytes_per_launch"]
 
@@ -492,7 +501,8 @@ def main():
             "per_M": per_m,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": decode_traffic(),
-                         "kernel": "gemv_wq_kernel (decode: fused RKV + O + key + value, all M)",
+                         "kernel": "decode products (fused RKV + O + key + value, all M): "
+                                   "gemv_wq_kernel (row tiles) and gemv_ck_kernel (cluster split-K)",
                          "bytes_per_launch": bytes_per_step / launches_per_step,
                          "us_per_launch": ms_per_step * 1e3 / launches_per_step,
                          "peak_kind": peak_kind + " copy bandwidth"},

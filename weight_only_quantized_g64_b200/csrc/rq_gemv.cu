@@ -16,35 +16,27 @@
 // 128 / 64 / 32 weights per cycle per SM for M <= 8 / 16 / 32.  (Both figures
 // measured on this hardware.)
 //
-// Work decomposition.  A row tile is RBM = 16*MTM consecutive rows of each of
-// the NMAT matrices (NMAT = 3 for the fused R/K/V call, whose matrices share
-// x), i.e. MT = NMAT*MTM MMA m-tiles of 16 rows.  A unit is one row tile times
-// one 128-byte column stage of codes (int4: 256 k = 4 groups; int8: 128 k = 2
-// groups).  The units, tile-major, are cut into equal contiguous runs, one per
-// CTA (stream-K).  Inside a CTA the units are dealt round-robin to the 8
-// warps (unit j of the CTA to warp j % 8): every warp works on all MT m-tiles
-// of its units, so
-// each x fragment it loads serves MT m-tiles, and the warps' partial sums are
-// added in shared memory when the tile ends.  When the CTAs outnumber the
-// tiles' needs the host picks one tile per CTA, and then nothing is reduced
-// across CTAs; otherwise a tile shared by several CTAs is stored as pieces in
-// a global workspace and summed, in a fixed CTA order, by whichever
-// contributor arrives last (an atomic counter per tile), so results stay
-// deterministic.
+// Work decomposition.  A row tile is RBM = WR * 16 * MTW consecutive rows of
+// each of the NMAT matrices (NMAT = 3 for the fused R/K/V call, whose
+// matrices share x).  A unit is one row tile times one 128-byte column stage
+// of codes (int4: 256 k = 4 groups; int8: 128 k = 2 groups).  The units,
+// tile-major, are cut into equal contiguous runs, one per CTA (stream-K), or
+// whole tiles are dealt one run per CTA when they balance over the SMs.  A
+// CTA walks its run as load groups: up to ks consecutive stages of one row
+// tile.  The 8 compute warps split a group WK ways along k (warp w takes
+// stage w % WK) and 8 / WK ways along rows; the k-split warps' partial sums
+// are added in shared memory, in warp order, by a reduction warp.  A tile
+// shared by several CTAs is stored as pieces in a global workspace and
+// summed, in a fixed CTA order, by whichever contributor arrives last (an
+// atomic counter per tile), so results stay deterministic.
 //
-// Data path (one CTA = 8 warps, no dedicated producer):
-//   codes   TMA 2D tiles [RBM rows x 128 B] per matrix, SWIZZLE_128B, into a
-//           ring of SS stages (SS = 8, 16 or 32); the first SS units are
-//           fetched by warp 0 before the kernel waits on the previous grid
-//           (codes and scales do not depend on it);
-//   scales  cp.async into a parallel ring, completing on the same barrier;
-//   x       per warp: cp.async of the M x 256 k (int4; 128 k for int8) slice
-//           of its unit into a buffer of its own, one unit ahead (two
-//           buffers when shared memory allows), after the wait; token rows
-//           >= M are never read (their B fragments are zero).
-// A warp that has read a stage refills that slot itself with the unit SS
-// places ahead, so no slot needs an "empty" barrier and no warp waits to
-// issue; 8 warps leave room for two CTAs per SM at up to 128 registers.
+// Data path: a producer warp fills a ring of 2..8 load-group slots, each
+// holding the group's codes (one 3D TMA box per matrix: ks stages x RBM
+// rows, 128-byte swizzled), its scales (one box per matrix) and its x (one
+// 3D box of the group's 64-k groups x M tokens).  Codes and scales of the
+// first slots are requested before the kernel waits on the previous grid;
+// x after.  Compute warps release a slot with an mbarrier arrive and the
+// producer refills it.
 // Thread (g = lane/4, t = lane%4) owns, per group of 64 k, the 16 k
 // [16t, 16t+16) of rows g and g+8 of each m-tile: MMA k-slot sigma of step j
 // maps to one of those k, the same map on the A (weights) and B (x) side, so

@@ -41,10 +41,9 @@
 
 namespace rq {
 
-// Eight warps, all computing (two per SM sub-partition, so up to 255
-// registers a thread); loads are issued by single lanes between their math.
-constexpr int kCkWarps = 8;
-constexpr int kCkThreads = kCkWarps * 32;
+// NW warps, all computing; loads are issued by single lanes between their
+// math.  With eight warps (two per SM sub-partition) a thread may use up to
+// 255 registers.
 constexpr int kCkMaxSlots = 8;
 constexpr int kCkMaxCluster = 8;
 constexpr int kCkSRow = 16;                              // staged scale row: 16 fp16 (32 B)
@@ -80,11 +79,12 @@ struct CkBars {
     int abort;
 };
 
-// WK: warps along k (groups of a stage dealt round-robin); WR = 8 / WK row
-// strips of MTW m-tiles.  R = WR * 16 * MTW rows per row block.
-template <int BITS, int MTW, int NT, int WK>
+// NW warps; WK of them along k (groups of a stage dealt round-robin); WR =
+// NW / WK row strips of MTW m-tiles.  R = WR * 16 * MTW rows per row block.
+template <int BITS, int MTW, int NT, int WK, int NW>
 struct CkCfg {
-    static constexpr int kWR = kCkWarps / WK;
+    static constexpr int kThreads = NW * 32;
+    static constexpr int kWR = NW / WK;
     static constexpr int kR = kWR * 16 * MTW;
     static constexpr int kGPS = BITS == 4 ? 4 : 2;
     static constexpr int kKPS = BITS == 4 ? 256 : 128;    // k per 128-byte stage
@@ -94,10 +94,12 @@ struct CkCfg {
     static_assert(kCkMaxKs * kGPS + 7 <= kCkSRow, "scale box holds a piece's groups");
 };
 
-template <int BITS, int MTW, int NT, int WK>
-__global__ void __launch_bounds__(kCkThreads, (NT == 1 ? 2 : 1))
+template <int BITS, int MTW, int NT, int WK, int NW>
+__global__ void __launch_bounds__(NW * 32, (NW == 8 && NT == 1 ? 2 : 1))
     gemv_ck_kernel(const __grid_constant__ CkParams p) {
-    using Cfg = CkCfg<BITS, MTW, NT, WK>;
+    using Cfg = CkCfg<BITS, MTW, NT, WK, NW>;
+    constexpr int kCkWarps = NW;
+    constexpr int kCkThreads = Cfg::kThreads;
     constexpr int R = Cfg::kR;
     constexpr int GPS = Cfg::kGPS;
     constexpr int MT = MTW;
@@ -343,9 +345,9 @@ struct CkPlan {
 
 // Shared-memory layout for a cluster size: ring slots (codes, scales and x of
 // a piece), the received partial sums, the barriers.
-template <int BITS, int MTW, int NT, int WK>
+template <int BITS, int MTW, int NT, int WK, int NW>
 static bool ck_layout(int M, int S, int C, bool three_d, CkPlan* L) {
-    using Cfg = CkCfg<BITS, MTW, NT, WK>;
+    using Cfg = CkCfg<BITS, MTW, NT, WK, NW>;
     const int sc_max = (S + C - 1) / C;                    // stages of the busiest rank
     L->C = C;
     L->ks = three_d ? (sc_max < kCkMaxKs ? sc_max : kCkMaxKs) : 1;
@@ -370,14 +372,14 @@ static bool ck_layout(int M, int S, int C, bool three_d, CkPlan* L) {
 }
 
 // Clusters of C CTAs with this shared memory that fit on the GPU at once.
-template <int BITS, int MTW, int NT, int WK>
+template <int BITS, int MTW, int NT, int WK, int NW>
 static int ck_max_clusters(int C, int smem) {
     static int cache[kCkMaxCluster + 1][64] = {};
     const int sb = smem / 4096;
     if (sb < 64 && cache[C][sb] > 0) return cache[C][sb];
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(C), 1, 1);
-    cfg.blockDim = dim3(kCkThreads, 1, 1);
+    cfg.blockDim = dim3(NW * 32, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>((sb + 1) * 4096 < kCkSmemMax ? (sb + 1) * 4096 : kCkSmemMax);
     cudaLaunchAttribute a;
     a.id = cudaLaunchAttributeClusterDimension;
@@ -387,7 +389,7 @@ static int ck_max_clusters(int C, int smem) {
     cfg.attrs = &a;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemv_ck_kernel<BITS, MTW, NT, WK>, &cfg) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveClusters(&n, gemv_ck_kernel<BITS, MTW, NT, WK, NW>, &cfg) != cudaSuccess ||
         n <= 0) {
         cudaGetLastError();
         n = ck_num_sms() / C;
@@ -402,17 +404,17 @@ static int ck_max_clusters(int C, int smem) {
 // at about half of the 1024 MAC per cycle and SM; waves add up; a cluster's
 // reduction adds a fixed latency.  So the estimate favours enough CTAs to
 // cover the SMs with the least work each.
-template <int BITS, int MTW, int NT, int WK>
+template <int BITS, int MTW, int NT, int WK, int NW>
 static bool ck_choose(int M, int N, int S, int nmat, bool three_d, CkPlan* best) {
-    using Cfg = CkCfg<BITS, MTW, NT, WK>;
+    using Cfg = CkCfg<BITS, MTW, NT, WK, NW>;
     const int rbt = nmat * ((N + Cfg::kR - 1) / Cfg::kR);
     bool found = false;
     for (int C = 1; C <= kCkMaxCluster && C <= S; ++C) {
         CkPlan L;
-        if (!ck_layout<BITS, MTW, NT, WK>(M, S, C, three_d, &L)) continue;
+        if (!ck_layout<BITS, MTW, NT, WK, NW>(M, S, C, three_d, &L)) continue;
         const int sc_max = (S + C - 1) / C;
         const int64_t ctas = static_cast<int64_t>(rbt) * C;
-        const int64_t cap = static_cast<int64_t>(ck_max_clusters<BITS, MTW, NT, WK>(C, L.smem)) * C;
+        const int64_t cap = static_cast<int64_t>(ck_max_clusters<BITS, MTW, NT, WK, NW>(C, L.smem)) * C;
         const int64_t waves = (ctas + cap - 1) / cap;
         const double bytes = static_cast<double>(Cfg::kR) * sc_max * (128 + 2 * Cfg::kGPS);
         const double macs = static_cast<double>(Cfg::kR) * sc_max * Cfg::kKPS * NT * 8;
@@ -428,11 +430,11 @@ static bool ck_choose(int M, int N, int S, int nmat, bool three_d, CkPlan* best)
     return found;
 }
 
-template <int BITS, int MTW, int NT, int WK>
+template <int BITS, int MTW, int NT, int WK, int NW>
 static cudaError_t ck_launch(CkParams& prm, const uint16_t* x, const void* const* codes, int nmat,
                              cudaStream_t s) {
-    using Cfg = CkCfg<BITS, MTW, NT, WK>;
-    auto kern = gemv_ck_kernel<BITS, MTW, NT, WK>;
+    using Cfg = CkCfg<BITS, MTW, NT, WK, NW>;
+    auto kern = gemv_ck_kernel<BITS, MTW, NT, WK, NW>;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -448,7 +450,7 @@ static cudaError_t ck_launch(CkParams& prm, const uint16_t* x, const void* const
     // the 3D code view needs rows of whole 128-byte stages
     const bool three_d = row_bytes % 128 == 0;
     CkPlan L;
-    if (!ck_choose<BITS, MTW, NT, WK>(prm.M, prm.N, prm.S, nmat, three_d, &L))
+    if (!ck_choose<BITS, MTW, NT, WK, NW>(prm.M, prm.N, prm.S, nmat, three_d, &L))
         return cudaErrorInvalidValue;
     prm.C = L.C;
     prm.rbpm = (prm.N + Cfg::kR - 1) / Cfg::kR;
@@ -492,7 +494,7 @@ static cudaError_t ck_launch(CkParams& prm, const uint16_t* x, const void* const
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(L.grid), 1, 1);
-    cfg.blockDim = dim3(kCkThreads, 1, 1);
+    cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(L.smem);
     cfg.stream = s;
     cudaLaunchAttribute attrs[3];
@@ -517,35 +519,36 @@ static cudaError_t ck_launch(CkParams& prm, const uint16_t* x, const void* const
     return cudaLaunchKernelEx(&cfg, kern, static_cast<const CkParams&>(prm));
 }
 
-// Warp split by batch: M <= 8 one m-tile per warp and no k split; M <= 16
-// two m-tiles, the stage's groups split 2 ways; M <= 32 (int4) four m-tiles
-// split 4 ways, so each x fragment serves 64 rows (int8 stages hold only two
-// groups: two m-tiles, 2 ways).
+// Warp split by batch (eight warps; sixteen measured no faster): M <= 8 one
+// m-tile per warp and no k split; M <= 16 two m-tiles, the stage's groups
+// split 2 ways; M <= 32 (int4) four m-tiles split 4 ways, so each x
+// fragment serves 64 rows (int8 stages hold only two groups: two m-tiles,
+// 2 ways).
 template <int BITS>
 static cudaError_t ck_dispatch(CkParams& prm, const uint16_t* x, const void* const* codes,
                                int nmat, cudaStream_t s) {
-    if (prm.M <= 8) return ck_launch<BITS, 1, 1, 1>(prm, x, codes, nmat, s);
-    if (prm.M <= 16) return ck_launch<BITS, 2, 2, 2>(prm, x, codes, nmat, s);
-    if constexpr (BITS == 4) return ck_launch<BITS, 4, 4, 4>(prm, x, codes, nmat, s);
-    else return ck_launch<BITS, 2, 4, 2>(prm, x, codes, nmat, s);
+    if (prm.M <= 8) return ck_launch<BITS, 1, 1, 1, 8>(prm, x, codes, nmat, s);
+    if (prm.M <= 16) return ck_launch<BITS, 2, 2, 2, 8>(prm, x, codes, nmat, s);
+    if constexpr (BITS == 4) return ck_launch<BITS, 4, 4, 4, 8>(prm, x, codes, nmat, s);
+    else return ck_launch<BITS, 2, 4, 2, 8>(prm, x, codes, nmat, s);
 }
 
-template <int BITS, int MTW, int NT, int WK>
+template <int BITS, int MTW, int NT, int WK, int NW>
 static bool ck_fits_cfg(int M, int K) {
     const int64_t row_bytes = static_cast<int64_t>(K) * BITS / 8;
     const int S = static_cast<int>((row_bytes + 127) / 128);
     CkPlan L;
     for (int C = 1; C <= kCkMaxCluster && C <= S; ++C)
-        if (ck_layout<BITS, MTW, NT, WK>(M, S, C, row_bytes % 128 == 0, &L)) return true;
+        if (ck_layout<BITS, MTW, NT, WK, NW>(M, S, C, row_bytes % 128 == 0, &L)) return true;
     return false;
 }
 
 template <int BITS>
 static bool ck_fits(int M, int K) {
-    if (M <= 8) return ck_fits_cfg<BITS, 1, 1, 1>(M, K);
-    if (M <= 16) return ck_fits_cfg<BITS, 2, 2, 2>(M, K);
-    if constexpr (BITS == 4) return ck_fits_cfg<BITS, 4, 4, 4>(M, K);
-    else return ck_fits_cfg<BITS, 2, 4, 2>(M, K);
+    if (M <= 8) return ck_fits_cfg<BITS, 1, 1, 1, 8>(M, K);
+    if (M <= 16) return ck_fits_cfg<BITS, 2, 2, 2, 8>(M, K);
+    if constexpr (BITS == 4) return ck_fits_cfg<BITS, 4, 4, 4, 8>(M, K);
+    else return ck_fits_cfg<BITS, 2, 4, 2, 8>(M, K);
 }
 
 bool gemv_cluster_fits(int64_t M, int64_t K, int bits) {

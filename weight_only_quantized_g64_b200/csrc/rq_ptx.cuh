@@ -111,48 +111,6 @@ __device__ __forceinline__ bool mbar_wait_suspend(uint64_t* bar, uint32_t parity
     }
 }
 
-// ------------------------------------------------- cp.async (LDGSTS) --
-// Global -> shared copy of 4 or 8 bytes; bytes beyond src_bytes are zero-filled
-// (src_bytes = 0 reads nothing).
-__device__ __forceinline__ void cp_async_8(void* dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(dst)), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_4(void* dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-// 16-byte global -> shared copy that bypasses L1 (cp.async.cg); bytes beyond
-// src_bytes (0 or 16) are zero-filled.
-__device__ __forceinline__ void cp_async_16(void* dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-// Wait until at most N of this thread's committed cp.async groups are pending.
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// Arrive on `bar` once this thread's earlier cp.async copies have landed; the
-// arrival counts toward the barrier's expected count (no increment).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
-// Orders this thread's earlier generic-proxy accesses to shared memory before
-// its later async-proxy accesses (a TMA write into a buffer it has just read).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // -------------------------------------------------------------------- TMA --
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -318,41 +276,6 @@ __device__ __forceinline__ void cluster_sync() {
                      : "memory");
 }
 
-// Split cluster barrier: arrive (no ordering of earlier memory operations)
-// and wait.  Every thread of every CTA in the cluster executes both, in order.
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-}
-
-// Asynchronous stores into the shared memory of a CTA of the cluster (caddr
-// and the barrier are shared::cluster addresses of that CTA): the bytes are
-// counted on that CTA's mbarrier as they land.
-__device__ __forceinline__ void st_async_f32x2(uint32_t caddr, float a, float b, uint32_t cbar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
-                 ::"r"(caddr), "f"(a), "f"(b), "r"(cbar)
-                 : "memory");
-}
-__device__ __forceinline__ void st_async_f32(uint32_t caddr, float a, uint32_t cbar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];"
-                 ::"r"(caddr), "f"(a), "r"(cbar)
-                 : "memory");
-}
-
-// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
-// from this CTA's shared memory into the shared memory of a CTA of the
-// cluster (dst and the barrier are shared::cluster addresses of that CTA);
-// the bytes are counted on that CTA's mbarrier as they land.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_caddr, const void* src,
-                                                  uint32_t bytes, uint32_t cbar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(dst_caddr), "r"(smem_u32(src)), "r"(bytes), "r"(cbar)
-        : "memory");
-}
-
 __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
@@ -366,12 +289,6 @@ __device__ __forceinline__ void st_dsmem_f32x4(uint32_t caddr, float4 v) {
     asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
                  ::"r"(caddr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
                  : "memory");
-}
-
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t caddr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(caddr) : "memory");
-    return v;
 }
 
 __device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t caddr) {
