@@ -89,13 +89,14 @@ struct CkCfg {
     static constexpr int kGPS = BITS == 4 ? 4 : 2;
     static constexpr int kKPS = BITS == 4 ? 256 : 128;    // k per 128-byte stage
     static constexpr int kCStage = kR * 128;               // code bytes per stage
-    static_assert(kR == 128, "row blocks of 128 rows");
-    static_assert(kGPS % WK == 0, "k-warps split a stage's groups evenly");
+    static_assert(kR == 64 || kR == 128, "row blocks of 64 or 128 rows");
+    static_assert(kGPS % WK == 0 || WK % kGPS == 0, "k-warps split a stage's groups evenly, or "
+                                                    "take whole groups of a piece");
     static_assert(kCkMaxKs * kGPS + 7 <= kCkSRow, "scale box holds a piece's groups");
 };
 
 template <int BITS, int MTW, int NT, int WK, int NW>
-__global__ void __launch_bounds__(NW * 32, (NW == 8 && NT == 1 ? 2 : 1))
+__global__ void __launch_bounds__(NW * 32, 1)
     gemv_ck_kernel(const __grid_constant__ CkParams p) {
     using Cfg = CkCfg<BITS, MTW, NT, WK, NW>;
     constexpr int kCkWarps = NW;
@@ -206,6 +207,19 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8 && NT == 1 ? 2 : 1))
                 const int st = s0 + i * p.ks;
                 const int n = min(p.ks, s1 - st);
                 const uint8_t* base = ring + slot * p.slot_bytes;
+                if constexpr (WK > GPS) {
+                    // more k-warps than groups in a stage: warp kw takes groups
+                    // kw, kw + WK, ... of the piece, one at a time
+                    for (int gi = kw; gi < n * GPS; gi += WK) {
+                        const int j = gi / GPS;
+                        const uint8_t* wt = base + j * Cfg::kCStage + wrow * 128;
+                        const uint8_t* sc =
+                            base + p.s_off + (wrow * kCkSRow + ((st * GPS) & 7) + j * GPS) * 2;
+                        gv_unit_strided<BITS, MT, NT, GPS, kCkSRow>(
+                            wt, sc, base + p.x_off, j * GPS, gi - j * GPS, M, xtok, prow, t,
+                            p.ssc != 0, p.scales[mat], row0 + wrow, st + j, p.N, p.groups, acc);
+                    }
+                } else
                 for (int j = 0; j < n; ++j) {
                     const uint8_t* wt = base + j * Cfg::kCStage + wrow * 128;
                     const uint8_t* sc =
@@ -259,6 +273,35 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8 && NT == 1 ? 2 : 1))
             }
         }
     __syncthreads();
+    if (C == 1) {
+        // no K split: add the k-warps' sums and store y; a warp's lanes take
+        // consecutive rows, so each token's stores coalesce
+        pdl_wait();   // y may be read by the previous kernel
+        if (*abort_flag == 0) {
+            const int nq = (M + 3) / 4;
+            float* y = p.y[mat];
+            for (int o = threadIdx.x; o < R * nq; o += kCkThreads) {
+                const int q = o / R;
+                const int row = o - q * R;
+                float4 v = *reinterpret_cast<const float4*>(part + row * MP + 4 * q);
+#pragma unroll
+                for (int k2 = 1; k2 < WK; ++k2) {
+                    const float4 u = *reinterpret_cast<const float4*>(part + (k2 * R + row) * MP + 4 * q);
+                    v.x += u.x;
+                    v.y += u.y;
+                    v.z += u.z;
+                    v.w += u.w;
+                }
+                const int n = row0 + row;
+                if (n < p.N) {
+                    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (4 * q + e < M) y[static_cast<int64_t>(4 * q + e) * p.N + n] = vv[e];
+                }
+            }
+        }
+    } else {
     {
         const int nq = (M + 3) / 4;
         const uint32_t recv_s = smem_u32(recv) + static_cast<uint32_t>(rank * share * MP * 4);
@@ -308,6 +351,7 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8 && NT == 1 ? 2 : 1))
             }
         }
     }
+    }   // C > 1
     // After a timeout some copies may still be in flight: wait (bounded) for
     // the last piece of every slot, so nothing lands after the CTA exits.
     if (threadIdx.x == 0 && *abort_flag) {
@@ -335,6 +379,7 @@ static int ck_num_sms() {
 }
 
 constexpr int kCkSmemMax = 227 * 1024;
+constexpr int kCkSmemOneCta = 120 * 1024;   // more than half an SM's shared memory
 
 static int ck_align(int v, int a) { return (v + a - 1) / a * a; }
 
@@ -366,6 +411,9 @@ static bool ck_layout(int M, int S, int C, bool three_d, CkPlan* L) {
         L->recv_off = ring;
         L->bar_off = ck_align(L->recv_off + recv_bytes, 16);
         L->smem = 1024 + L->bar_off + static_cast<int>(sizeof(CkBars));
+        // one CTA per SM: two CTAs of one launch on an SM (which the block
+        // scheduler does when it can) finish last and hold the launch back
+        if (L->smem < kCkSmemOneCta) L->smem = kCkSmemOneCta;
         if (L->smem <= kCkSmemMax && (ns >= 2 || pieces == 1)) return true;
     }
     return false;
@@ -401,9 +449,10 @@ static int ck_max_clusters(int C, int smem) {
 // Cluster size: the estimated time of one launch, over C = 1..8.  A CTA
 // streams its codes at about the HBM rate divided by the SMs (~40 GB/s on
 // B200: one CTA cannot pull much more, however few run) and does its MMA work
-// at about half of the 1024 MAC per cycle and SM; waves add up; a cluster's
-// reduction adds a fixed latency.  So the estimate favours enough CTAs to
-// cover the SMs with the least work each.
+// at about half of the 1024 MAC per cycle and SM; waves add up, each with a
+// fixed latency; a cluster's reduction costs a barrier and its bytes.  So the estimate favours enough
+// CTAs to cover the SMs with the least work each, and no K split when that
+// is possible.
 template <int BITS, int MTW, int NT, int WK, int NW>
 static bool ck_choose(int M, int N, int S, int nmat, bool three_d, CkPlan* best) {
     using Cfg = CkCfg<BITS, MTW, NT, WK, NW>;
@@ -419,7 +468,12 @@ static bool ck_choose(int M, int N, int S, int nmat, bool three_d, CkPlan* best)
         const double bytes = static_cast<double>(Cfg::kR) * sc_max * (128 + 2 * Cfg::kGPS);
         const double macs = static_cast<double>(Cfg::kR) * sc_max * Cfg::kKPS * NT * 8;
         const double t_cta = bytes / 40e9 + macs / (512.0 * 1.8e9);
-        const double est = static_cast<double>(waves) * t_cta + (C > 1 ? 0.3e-6 : 0.0);
+        // a cluster's reduction: a barrier plus R x MP sums per CTA through
+        // distributed shared memory (tens of GB/s per SM)
+        const double t_red = C > 1 ? 0.3e-6 + static_cast<double>(Cfg::kR) * L.mp * 4 / 20e9 : 0.0;
+        // every wave also pays the latency of a CTA's start, first loads,
+        // barriers and exit (about 1.5 us measured)
+        const double est = static_cast<double>(waves) * (t_cta + 1.5e-6) + t_red;
         if (!found || est < best->est * 0.98) {
             L.est = est;
             L.grid = static_cast<int>(ctas);
@@ -430,28 +484,37 @@ static bool ck_choose(int M, int N, int S, int nmat, bool three_d, CkPlan* best)
     return found;
 }
 
+// The best plan of one configuration for this product (false: none fits).
 template <int BITS, int MTW, int NT, int WK, int NW>
-static cudaError_t ck_launch(CkParams& prm, const uint16_t* x, const void* const* codes, int nmat,
-                             cudaStream_t s) {
-    using Cfg = CkCfg<BITS, MTW, NT, WK, NW>;
+static bool ck_plan(const CkParams& prm, int nmat, CkPlan* L, cudaError_t* err) {
     auto kern = gemv_ck_kernel<BITS, MTW, NT, WK, NW>;
     static bool attr_set[64] = {};
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return false;
+    if (dev < 0 || dev >= 64) {
+        *err = cudaErrorInvalidDevice;
+        return false;
+    }
     if (!attr_set[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kCkSmemMax);
-        if (e != cudaSuccess) return e;
+        // (before the occupancy query, which checks it)
+        *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kCkSmemMax);
+        if (*err != cudaSuccess) return false;
         attr_set[dev] = true;
     }
     const int64_t row_bytes = static_cast<int64_t>(prm.K) * BITS / 8;
-    prm.S = static_cast<int>((row_bytes + 127) / 128);
+    const int S = static_cast<int>((row_bytes + 127) / 128);
     // the 3D code view needs rows of whole 128-byte stages
-    const bool three_d = row_bytes % 128 == 0;
-    CkPlan L;
-    if (!ck_choose<BITS, MTW, NT, WK, NW>(prm.M, prm.N, prm.S, nmat, three_d, &L))
-        return cudaErrorInvalidValue;
+    return ck_choose<BITS, MTW, NT, WK, NW>(prm.M, prm.N, S, nmat, row_bytes % 128 == 0, L);
+}
+
+template <int BITS, int MTW, int NT, int WK, int NW>
+static cudaError_t ck_launch(CkParams& prm, const uint16_t* x, const void* const* codes, int nmat,
+                             cudaStream_t s, const CkPlan& L) {
+    using Cfg = CkCfg<BITS, MTW, NT, WK, NW>;
+    auto kern = gemv_ck_kernel<BITS, MTW, NT, WK, NW>;
+    const int64_t row_bytes = static_cast<int64_t>(prm.K) * BITS / 8;
+    prm.S = static_cast<int>((row_bytes + 127) / 128);
     prm.C = L.C;
     prm.rbpm = (prm.N + Cfg::kR - 1) / Cfg::kR;
     prm.ks = L.ks;
@@ -504,8 +567,7 @@ static cudaError_t ck_launch(CkParams& prm, const uint16_t* x, const void* const
     attrs[na].val.clusterDim.y = 1;
     attrs[na].val.clusterDim.z = 1;
     ++na;
-    // spread a launch's CTAs over distinct SMs (two of one launch on an SM
-    // would finish last)
+    // spread a launch's clusters over the GPCs
     attrs[na].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
     attrs[na].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicySpread;
     ++na;
@@ -519,18 +581,34 @@ static cudaError_t ck_launch(CkParams& prm, const uint16_t* x, const void* const
     return cudaLaunchKernelEx(&cfg, kern, static_cast<const CkParams&>(prm));
 }
 
-// Warp split by batch (eight warps; sixteen measured no faster): M <= 8 one
-// m-tile per warp and no k split; M <= 16 two m-tiles, the stage's groups
-// split 2 ways; M <= 32 (int4) four m-tiles split 4 ways, so each x
-// fragment serves 64 rows (int8 stages hold only two groups: two m-tiles,
-// 2 ways).
+// Warp split by batch (eight warps; sixteen measured no faster), for row
+// blocks of 128 or 64 rows: M <= 8 one m-tile per warp (64 rows: the stage's
+// groups split 2 ways); M <= 16 two m-tiles, groups split 2 (4) ways; M <= 32
+// (int4) four m-tiles, groups split 4 ways (64 rows: each warp takes whole
+// groups of a piece, 8 ways), so each x fragment serves 64 rows; int8 stages
+// hold two groups: two m-tiles, 2 (4) ways.  The plan with the lower
+// estimate runs.
+template <int BITS, int MTW, int NT, int WK, int MTW2, int WK2>
+static cudaError_t ck_pick(CkParams& prm, const uint16_t* x, const void* const* codes, int nmat,
+                           cudaStream_t s) {
+    CkPlan a, b;
+    cudaError_t ea = cudaSuccess, eb = cudaSuccess;
+    const bool fa = ck_plan<BITS, MTW, NT, WK, 8>(prm, nmat, &a, &ea);
+    const bool fb = ck_plan<BITS, MTW2, NT, WK2, 8>(prm, nmat, &b, &eb);
+    if (ea != cudaSuccess) return ea;
+    if (eb != cudaSuccess) return eb;
+    if (fb && (!fa || b.est < a.est)) return ck_launch<BITS, MTW2, NT, WK2, 8>(prm, x, codes, nmat, s, b);
+    if (fa) return ck_launch<BITS, MTW, NT, WK, 8>(prm, x, codes, nmat, s, a);
+    return cudaErrorInvalidValue;
+}
+
 template <int BITS>
 static cudaError_t ck_dispatch(CkParams& prm, const uint16_t* x, const void* const* codes,
                                int nmat, cudaStream_t s) {
-    if (prm.M <= 8) return ck_launch<BITS, 1, 1, 1, 8>(prm, x, codes, nmat, s);
-    if (prm.M <= 16) return ck_launch<BITS, 2, 2, 2, 8>(prm, x, codes, nmat, s);
-    if constexpr (BITS == 4) return ck_launch<BITS, 4, 4, 4, 8>(prm, x, codes, nmat, s);
-    else return ck_launch<BITS, 2, 4, 2, 8>(prm, x, codes, nmat, s);
+    if (prm.M <= 8) return ck_pick<BITS, 1, 1, 1, 1, 2>(prm, x, codes, nmat, s);
+    if (prm.M <= 16) return ck_pick<BITS, 2, 2, 2, 2, 4>(prm, x, codes, nmat, s);
+    if constexpr (BITS == 4) return ck_pick<BITS, 4, 4, 4, 4, 8>(prm, x, codes, nmat, s);
+    else return ck_pick<BITS, 2, 4, 2, 2, 4>(prm, x, codes, nmat, s);
 }
 
 template <int BITS, int MTW, int NT, int WK, int NW>
@@ -545,10 +623,11 @@ static bool ck_fits_cfg(int M, int K) {
 
 template <int BITS>
 static bool ck_fits(int M, int K) {
-    if (M <= 8) return ck_fits_cfg<BITS, 1, 1, 1, 8>(M, K);
-    if (M <= 16) return ck_fits_cfg<BITS, 2, 2, 2, 8>(M, K);
-    if constexpr (BITS == 4) return ck_fits_cfg<BITS, 4, 4, 4, 8>(M, K);
-    else return ck_fits_cfg<BITS, 2, 4, 2, 8>(M, K);
+    if (M <= 8) return ck_fits_cfg<BITS, 1, 1, 1, 8>(M, K) || ck_fits_cfg<BITS, 1, 1, 2, 8>(M, K);
+    if (M <= 16) return ck_fits_cfg<BITS, 2, 2, 2, 8>(M, K) || ck_fits_cfg<BITS, 2, 2, 4, 8>(M, K);
+    if constexpr (BITS == 4)
+        return ck_fits_cfg<BITS, 4, 4, 4, 8>(M, K) || ck_fits_cfg<BITS, 4, 4, 8, 8>(M, K);
+    else return ck_fits_cfg<BITS, 2, 4, 2, 8>(M, K) || ck_fits_cfg<BITS, 2, 4, 4, 8>(M, K);
 }
 
 bool gemv_cluster_fits(int64_t M, int64_t K, int bits) {
