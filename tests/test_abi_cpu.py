@@ -88,6 +88,14 @@ def test_control_calls(L):
     assert L.rq_set_wait_limit_ns(0) == rq.ERR_RANGE
     assert L.rq_set_wait_limit_ns(10**9) == rq.OK
     assert L.rq_set_pdl(0) == rq.OK
+    # decode kernel selection: 0 automatic, 1 row tiles, 2 cluster split-K
+    for bad in (-1, 3, 1 << 20):
+        assert L.rq_set_decode_kernel(bad) == rq.ERR_RANGE
+    for kind, code in rq.DECODE_KERNELS.items():
+        assert L.rq_set_decode_kernel(code) == rq.OK
+        with rq.decode_kernel(kind):
+            pass
+    assert L.rq_set_decode_kernel(0) == rq.OK
     assert L.rq_selftest_bounded_wait(0, None) == rq.ERR_RANGE
     assert L.rq_read_device_status(None, 0) == rq.ERR_NULL
     for s in range(9):

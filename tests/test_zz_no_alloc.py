@@ -33,22 +33,24 @@ def _oracle(x, codes, scales, bits):
                          scales.cpu().numpy().view(np.uint16), bits)
 
 
+@pytest.mark.parametrize("kernel", ["auto", "rowtile", "cluster"])
 @pytest.mark.parametrize("N,K,M,bits", [(4096, 4096, 1, 4), (2048, 8192, 8, 4),
                                         (300, 640, 17, 4), (2560, 2560, 32, 8),
                                         (129, 128, 3, 8), (4096, 2048, 32, 4)])
-def test_noalloc_matches_gemv_two_calls(N, K, M, bits):
+def test_noalloc_matches_gemv_two_calls(N, K, M, bits, kernel):
     W = synth.weights(N, K, seed=71 + N + M, device="cuda")
     codes, scales = rq.quantize_g64(W, bits)
     x = synth.activations(M, K, seed=71 + M, device="cuda")
-    y_ref = rq.gemv_wq(x, codes, scales, N, bits)
     y1 = torch.full((M, N), float("nan"), device="cuda")
     y2 = torch.full((M, N), float("nan"), device="cuda")
     L = rq.lib()
     s = torch.cuda.current_stream().cuda_stream
-    for y in (y1, y2):
-        st = L.rq_gemv_wq_noalloc(x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(), N,
-                                  bits, y.data_ptr(), s)
-        assert st == rq.OK, rq.STATUS[st]
+    with rq.decode_kernel(kernel):
+        y_ref = rq.gemv_wq(x, codes, scales, N, bits)
+        for y in (y1, y2):
+            st = L.rq_gemv_wq_noalloc(x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(), N,
+                                      bits, y.data_ptr(), s)
+            assert st == rq.OK, rq.STATUS[st]
     torch.cuda.synchronize()
     y_or, bound = _oracle(x, codes, scales, bits)
     ref = y_ref.cpu().numpy().astype(np.float64)
