@@ -8,24 +8,33 @@
 // launch of the "RWKV-7 Quantization Toolkit" "Key Design"), decomposed for
 // batches where the activations are no longer small next to the weights.
 //
-// Decomposition.  A row block is R = 128 consecutive rows of one matrix (the
-// NMAT matrices of a fused call are stacked).  Each row block belongs to one
-// cluster of C CTAs; CTA rank c of the cluster takes the 128-byte code stages
-// [c*S/C, (c+1)*S/C) of every row (S stages per row), so the cluster splits K
-// and one row block's codes are read exactly once.  Each CTA loads the x
-// columns of its stages ONCE (one TMA box of its groups x all M tokens) and
-// keeps them in shared memory; only codes and scales stream, through a ring of
-// pieces (ks stages of the row block, one TMA box each; the first ones are
-// issued before the kernel waits on the previous grid).
-// Eight compute warps split the row block into WR = 8 / WK row strips of
-// 16 * MTW rows, and, when WK > 1, split each stage's groups WK ways; a warp
-// keeps MTW m-tiles so every x fragment it loads serves MTW * 16 rows.
+// Decomposition.  A row block is R = 128 or 64 consecutive rows of one
+// matrix (the NMAT matrices of a fused call are stacked).  Each row block
+// belongs to one cluster of C CTAs (C = 1: no split); CTA rank c of the
+// cluster takes the 128-byte code stages [c*S/C, (c+1)*S/C) of every row (S
+// stages per row), so the cluster splits K and one row block's codes are
+// read exactly once.  The host picks (R, C) per launch from an estimate of
+// the per-CTA streaming and MMA time, the waves and the reduction bytes, and
+// keeps one CTA per SM.
 //
-// Reduction.  Each warp leaves its fp32 sums for its rows and tokens in
-// shared memory; the CTA adds its WK k-warps' sums; after a cluster barrier,
-// CTA c adds, for rows [c*share, (c+1)*share) of the row block, the C CTAs'
-// sums in rank order through distributed shared memory and stores y.  The
-// order of every addition is fixed, so results are deterministic; nothing goes
+// Data path.  A piece is ks <= 2 stages of the row block: their codes (one
+// 3D TMA box), scales (one box) and the x of their groups for all M tokens
+// (one 3D box), in one ring slot on one mbarrier.  Thread 0 issues the codes
+// and scales of the first slots before the kernel waits on the previous grid
+// (they never depend on it), x after; later pieces are issued by the warp
+// whose turn it is once every warp has released the slot.  Eight warps, all
+// computing, split the row block into WR = 8 / WK row strips of 16 * MTW
+// rows; WK > 1 k-warps split each stage's groups (or, with more k-warps than
+// a stage has groups, take whole groups of a piece); a warp keeps MTW
+// m-tiles, so every x fragment it loads serves MTW * 16 rows.
+//
+// Reduction.  Each warp leaves its fp32 sums in shared memory; the CTA adds
+// its k-warps' sums row by row.  With C = 1 it stores y from there.
+// Otherwise the sum of row r goes, by plain distributed-shared-memory stores,
+// to the CTA of the cluster that owns r (rows [c*share, (c+1)*share) belong
+// to rank c); one release/acquire cluster barrier makes the stores visible;
+// each rank adds the C sums of its rows in rank order and stores y.  Every
+// addition has a fixed order, so results are deterministic; nothing goes
 // through global memory but x, codes, scales and y, and no counters or
 // workspace are needed.
 //
