@@ -230,13 +230,23 @@ def capture(fn):
 
 # ---------------------------------------------------------- CPU baseline --
 
-def cpu_oracle_rate(wl, budget_s=12.0, layer_rows=16):
+def oracle_threads(rows):
+    """OpenMP threads the oracle runs with: one per host core, but no more than
+    the rows it parallelises over (set before the oracle library loads)."""
+    threads = max(1, min(os.cpu_count() or 1, rows))
+    os.environ["OMP_NUM_THREADS"] = str(threads)
+    return threads
+
+
+def cpu_oracle_rate(wl, budget_s=12.0, layer_rows=None):
     """The oracle, as it stands, on a bounded sample of the decode workload:
-    `layer_rows` rows of every projection of layer 0 at every M, repeated
-    until `budget_s` of wall time; returns (weight GB/s, cores, sample)."""
+    `layer_rows` rows (default: one per host core, at least 16) of every
+    projection of layer 0 at every M, repeated until `budget_s` of wall time;
+    returns (weight GB/s, threads used, sample)."""
+    if layer_rows is None:
+        layer_rows = max(16, os.cpu_count() or 1)
+    cores = oracle_threads(layer_rows)
     import oracle
-    cores = os.cpu_count() or 1
-    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
     oracle.build()
     jobs = []
     for pi, pj in enumerate(wl.projs):
@@ -264,10 +274,10 @@ def reference_arm(args, wl, rank, world):
     """`--impl reference`: the oracle timed on the host cores, rank 0 only."""
     if rank != 0:
         return
+    rows = max(4, os.cpu_count() or 1)   # the oracle parallelises over rows
+    cores = oracle_threads(rows)
     import oracle
     oracle.build()
-    cores = os.cpu_count() or 1
-    rows = 4
     jobs = []
     for pi, pj in enumerate(wl.projs):
         W = synth.weights(rows, pj.K, seed=synth.seed_for(wl.index, 0, pi))
