@@ -187,6 +187,18 @@ rq_status rq_set_pdl(int enable);
 rq_status rq_set_decode_kernel(int kernel);
 
 /*
+ * rq_decode_kernel_for -- which decode kernel (RQ_DECODE_ROWTILE or
+ * RQ_DECODE_CLUSTER) a decode product of this shape would run on under the
+ * current rq_set_decode_kernel selection; nmat is 1 (rq_gemv_wq) or 3
+ * (rq_rkv_fused).  Host-only: launches nothing and needs no GPU.  The same
+ * argument checks as the products (RQ_ERR_BITS, RQ_ERR_SHAPE); kernel NULL
+ * gives RQ_ERR_NULL; a forced cluster kernel that cannot hold the shape gives
+ * RQ_ERR_SHAPE, as the product would.
+ */
+rq_status rq_decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat,
+                               int *kernel);
+
+/*
  * rq_set_wait_limit_ns -- time limit of every bounded on-chip wait of the
  * library's kernels (default 1 s).  A kernel whose wait exceeds it stops its
  * work, sets the device status word to RQ_ERR_TIMEOUT and exits; its outputs

@@ -103,6 +103,41 @@ def test_control_calls(L):
     assert L.rq_version() == b"0.1.0"
 
 
+def test_decode_kernel_choice(L):
+    """The automatic choice between the decode kernels (host logic, no GPU):
+    row tiles for M <= 8; the cluster kernel for M > 16; for 9 <= M <= 16
+    the cluster kernel on launches of >= 6144 rows with K <= 4096 (the fused
+    R/K/V and channel-mix key of the 1.5B-shaped layer), row tiles otherwise."""
+    D = 2048
+    layer = {"rkv": (D, D, 3), "o": (D, D, 1), "key": (4 * D, D, 1), "value": (D, 4 * D, 1)}
+    for M in (1, 4, 8):
+        for name, (N, K, nmat) in layer.items():
+            assert rq.decode_kernel_for(M, K, N, 4, nmat) == "rowtile", (M, name)
+    for M in (17, 24, 32):
+        for name, (N, K, nmat) in layer.items():
+            assert rq.decode_kernel_for(M, K, N, 4, nmat) == "cluster", (M, name)
+    for M in (9, 16):
+        assert rq.decode_kernel_for(M, D, D, 4, 3) == "cluster"
+        assert rq.decode_kernel_for(M, D, 4 * D, 4, 1) == "cluster"
+        assert rq.decode_kernel_for(M, D, D, 4, 1) == "rowtile"
+        assert rq.decode_kernel_for(M, 4 * D, D, 4, 1) == "rowtile"
+        assert rq.decode_kernel_for(M, 16384, 16384, 4, 1) == "rowtile"   # K > 4096
+    # a selection overrides the automatic choice
+    for kind in ("rowtile", "cluster"):
+        with rq.decode_kernel(kind):
+            for M in (1, 16, 32):
+                assert rq.decode_kernel_for(M, D, D, 8, 1) == kind
+    assert rq.decode_kernel_for(1, D, D, 4, 1) == "rowtile"
+    # argument checks
+    out = ctypes.c_int()
+    assert L.rq_decode_kernel_for(0, D, D, 4, 1, ctypes.byref(out)) == rq.ERR_SHAPE
+    assert L.rq_decode_kernel_for(33, D, D, 4, 1, ctypes.byref(out)) == rq.ERR_SHAPE
+    assert L.rq_decode_kernel_for(1, 100, D, 4, 1, ctypes.byref(out)) == rq.ERR_SHAPE
+    assert L.rq_decode_kernel_for(1, D, D, 4, 2, ctypes.byref(out)) == rq.ERR_SHAPE
+    assert L.rq_decode_kernel_for(1, D, D, 5, 1, ctypes.byref(out)) == rq.ERR_BITS
+    assert L.rq_decode_kernel_for(1, D, D, 4, 1, None) == rq.ERR_NULL
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(rq, "_lib", None)
     monkeypatch.setattr(rq, "LIB_PATH", str(tmp_path / "missing.so"))

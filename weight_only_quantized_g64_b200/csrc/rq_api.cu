@@ -285,6 +285,17 @@ rq_status rq_set_decode_kernel(int kernel) {
     return RQ_OK;
 }
 
+rq_status rq_decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat, int* kernel) {
+    rq_status st = check_weight_shape(N, K, bits);
+    if (st != RQ_OK) return st;
+    if (M < 1 || M > RQ_MAX_DECODE_M || (nmat != 1 && nmat != 3)) return RQ_ERR_SHAPE;
+    if (kernel == nullptr) return RQ_ERR_NULL;
+    const int which = decode_kernel_for(M, K, N, bits, nmat);
+    if (which < 0) return RQ_ERR_SHAPE;
+    *kernel = which;
+    return RQ_OK;
+}
+
 rq_status rq_set_wait_limit_ns(uint64_t limit_ns) {
     if (limit_ns == 0) return RQ_ERR_RANGE;
     g_wait_limit_ns = limit_ns;

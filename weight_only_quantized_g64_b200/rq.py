@@ -64,6 +64,8 @@ def lib():
     L.rq_set_pdl.restype = i32
     L.rq_set_decode_kernel.argtypes = [i32]
     L.rq_set_decode_kernel.restype = i32
+    L.rq_decode_kernel_for.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_int)]
+    L.rq_decode_kernel_for.restype = i32
     L.rq_set_wait_limit_ns.argtypes = [u64]
     L.rq_set_wait_limit_ns.restype = i32
     L.rq_read_device_status.argtypes = [ctypes.POINTER(ctypes.c_int), i32]
@@ -176,6 +178,13 @@ def set_pdl(enable: bool):
 def set_decode_kernel(kind: str):
     """Decode kernel for later products: "auto", "rowtile" or "cluster"."""
     _check(lib().rq_set_decode_kernel(DECODE_KERNELS[kind]), "rq_set_decode_kernel")
+
+
+def decode_kernel_for(M: int, K: int, N: int, bits: int, nmat: int = 1) -> str:
+    """The decode kernel ("rowtile" or "cluster") a product of this shape runs on."""
+    out = ctypes.c_int(-1)
+    _check(lib().rq_decode_kernel_for(M, K, N, bits, nmat, ctypes.byref(out)), "rq_decode_kernel_for")
+    return {v: k for k, v in DECODE_KERNELS.items()}[out.value]
 
 
 class decode_kernel:
