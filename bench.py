@@ -100,11 +100,20 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """The largest of every rank's v (device times are taken as the max over
+    ranks); the reduction runs where the process group's backend does."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cpu" if torch.distributed.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_gbs(world, bytes_per_rank_step, steps, max_ms):
+    """Whole-job weight GB/s: the bytes every rank streamed over the slowest
+    rank's time (each rank runs its own copy of the stack: weak scaling)."""
+    return world * bytes_per_rank_step * steps / (max_ms / 1e3) / 1e9
 
 
 # ---------------------------------------------------------------- clocks --
@@ -450,7 +459,7 @@ def main():
     bytes_per_step = stack.bytes_per_pass * len(wl.Ms)
     launches_per_step = stack.launches_per_pass * len(wl.Ms)
     ms_per_step = elapsed_ms / args.steps
-    value = world * bytes_per_step * args.steps / (elapsed_ms / 1e3) / 1e9
+    value = job_gbs(world, bytes_per_step, args.steps, elapsed_ms)
     per_rank_gbs = bytes_per_step / (ms_per_step / 1e3) / 1e9
     per_m = {str(M): {"us_per_pass": per_m_ms[M] / n_split * 1e3,
                       "gbs": stack.bytes_per_pass / (per_m_ms[M] / n_split / 1e3) / 1e9,
@@ -481,7 +490,7 @@ def main():
         e1.record(s)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-        e2e = {"value": world * bytes_per_step * e2e_steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+        e2e = {"value": job_gbs(world, bytes_per_step, e2e_steps, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / e2e_steps,
                "how": "pinned host x -> device, replay of the captured rq_* calls, "
