@@ -68,6 +68,8 @@ def _load():
     lib.rqo_f16_to_f64.restype = ctypes.c_double
     lib.rqo_quantize_g64.argtypes = [vp, i64, i64, ctypes.c_int, vp, vp]
     lib.rqo_quantize_g64.restype = ctypes.c_int
+    lib.rqo_quantize_g64_ex2.argtypes = [vp, i64, i64, ctypes.c_int, vp, vp, ctypes.c_int, vp, vp, vp]
+    lib.rqo_quantize_g64_ex2.restype = ctypes.c_int
     lib.rqo_matmul.argtypes = [vp, i64, i64, vp, vp, i64, ctypes.c_int, vp, vp]
     lib.rqo_matmul.restype = None
     lib.rqo_matmul_sampled.argtypes = [vp, i64, i64, vp, vp, i64, ctypes.c_int,
@@ -110,6 +112,28 @@ def quantize_g64(W: np.ndarray, bits: int):
     scales = np.zeros((N, K // GROUP), dtype=np.uint16)
     st = _load().rqo_quantize_g64(_ptr(W), N, K, bits, _ptr(codes), _ptr(scales))
     return codes, scales, int(st)
+
+
+def quantize_g64_ex2(W: np.ndarray, e2: np.ndarray, bits: int, factors):
+    """E[x^2]-weighted scale search on the symmetric group-64 grid: per group,
+    the candidate scale fp16(fp32(amax * f) / qmax), f in `factors`, whose
+    codes minimise sum_k e2[k] * (w_k - c_k * s16)^2 (fp32, k order; the
+    earlier candidate wins ties).  e2 [K] float32 >= 0, one value per input
+    channel.  Returns (codes, scales, chosen int32 [N, K/64], status)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    if bits not in (4, 8) or K % GROUP:
+        raise ValueError("bits must be 4 or 8 and K a multiple of 64")
+    e2 = np.ascontiguousarray(e2, dtype=np.float32)
+    f = np.ascontiguousarray(factors, dtype=np.float32)
+    if e2.shape != (K,) or f.ndim != 1 or f.size < 1:
+        raise ValueError("e2 must have K values and factors at least one")
+    codes = np.zeros((N, K * bits // 8), dtype=np.uint8)
+    scales = np.zeros((N, K // GROUP), dtype=np.uint16)
+    chosen = np.zeros((N, K // GROUP), dtype=np.int32)
+    st = _load().rqo_quantize_g64_ex2(_ptr(W), N, K, bits, _ptr(e2), _ptr(f), int(f.size),
+                                      _ptr(codes), _ptr(scales), _ptr(chosen))
+    return codes, scales, chosen, int(st)
 
 
 def matmul(x_f16: np.ndarray, codes: np.ndarray, scales: np.ndarray, bits: int,

@@ -211,6 +211,108 @@ int rqo_quantize_g64(const float *W, int64_t N, int64_t K, int bits,
     return status;
 }
 
+/* --------------------------------------------- E[x^2]-weighted search --- */
+/*
+ * "rwkv-quant: uma matriz em bf16 elimina 39% das perdas na quantização do
+ * RWKV-7 2.9B", section "Dois presets e seis tamanhos": in both presets the
+ * groups' scale (and, for the asymmetric layout, offset) is chosen by a
+ * search weighted by E[x^2], the mean square of the input channel's
+ * activation.  Here, on the symmetric g64 grid of rqo_quantize_g64, with the
+ * readings the page leaves open:
+ *   - candidates: scale factors f[0..nf) given by the caller; candidate j
+ *     uses s32 = fp32(amax * f[j]) / qmax (one fp32 multiply, one fp32
+ *     division), s16 = fp16_rn(s32), and codes c = clamp(rint(w / s16))
+ *     exactly as RTN does (f = 1 is RTN);
+ *   - criterion: err_j = sum over the group's 64 k, in k order, of
+ *     e2[k] * (d * d) with d = w - c * s16, every operation one fp32
+ *     rounding (t = c * s16, d = w - t, q = d * d, p = e2 * q, err = err + p);
+ *   - the candidate with the smallest err_j wins; on equal err_j the earlier
+ *     candidate wins; a candidate whose s16 overflows is never chosen;
+ *   - e2 is the caller's vector of E[x^2] per input channel (length K,
+ *     finite, >= 0); non-finite weights and an overflow of every candidate
+ *     give the statuses and outputs of RTN.
+ */
+static int quantize_group_ex2(const float *w, const float *e2, int bits, const float *f, int nf,
+                              uint16_t *scale_out, int *c_out, int *chosen_out)
+{
+    const int qmax = qmax_of(bits);
+    int i, j;
+    *chosen_out = 0;
+    for (i = 0; i < RQO_GROUP; i++)
+        if (!isfinite(w[i])) return quantize_group(w, bits, scale_out, c_out);
+    float amax = 0.0f;
+    for (i = 0; i < RQO_GROUP; i++) {
+        float a = fabsf(w[i]);
+        if (a > amax) amax = a;
+    }
+    int best = -1;
+    float best_err = 0.0f;
+    int cj[RQO_GROUP];
+    for (j = 0; j < nf; j++) {
+        volatile float a32 = amax * f[j];              /* fp32 multiply */
+        volatile float s32 = a32 / (float)qmax;        /* fp32 division */
+        uint16_t s16 = rqo_f32_to_f16(s32);
+        if (s16 == 0x7C00u) continue;                  /* overflow: never chosen */
+        float sf = (float)rqo_f16_to_f64(s16);
+        volatile float err = 0.0f;
+        for (i = 0; i < RQO_GROUP; i++) {
+            int c = 0;
+            if (sf != 0.0f) {
+                volatile float t0 = w[i] / sf;
+                float r = rintf(t0);
+                if (r > (float)qmax) r = (float)qmax;
+                if (r < (float)-qmax) r = (float)-qmax;
+                c = (int)r;
+            }
+            cj[i] = c;
+            volatile float t = (float)c * sf;
+            volatile float d = w[i] - t;
+            volatile float q = d * d;
+            volatile float pr = e2[i] * q;
+            err = err + pr;
+        }
+        if (best < 0 || err < best_err) {
+            best = j;
+            best_err = err;
+            *scale_out = s16;
+            for (i = 0; i < RQO_GROUP; i++) c_out[i] = cj[i];
+        }
+    }
+    if (best < 0) return quantize_group(w, bits, scale_out, c_out);   /* every candidate overflows */
+    *chosen_out = best;
+    return RQO_OK;
+}
+
+/* E[x^2]-weighted scale search over W[N, K] (layouts, statuses and packing
+ * as rqo_quantize_g64); e2[K], factors f[nf]; chosen (nullable) receives the
+ * winning candidate of each group, [N, K/64]. */
+int rqo_quantize_g64_ex2(const float *W, int64_t N, int64_t K, int bits, const float *e2,
+                         const float *f, int nf, uint8_t *codes, uint16_t *scales, int32_t *chosen)
+{
+    const int64_t G = K / RQO_GROUP;
+    int status = RQO_OK;
+    int64_t n;
+#pragma omp parallel for schedule(static) reduction(max : status)
+    for (n = 0; n < N; n++) {
+        int c[RQO_GROUP];
+        int64_t g;
+        for (g = 0; g < G; g++) {
+            int ch = 0;
+            int st = quantize_group_ex2(&W[n * K + g * RQO_GROUP], &e2[g * RQO_GROUP], bits, f, nf,
+                                        &scales[n * G + g], c, &ch);
+            int64_t i;
+            for (i = 0; i < RQO_GROUP; i++) put_code(codes, K, bits, n, g * RQO_GROUP + i, c[i]);
+            if (chosen) chosen[n * G + g] = ch;
+            if (st > status) status = st;
+        }
+    }
+    if (status != RQO_OK) {
+        int64_t i, total = N * G;
+        for (i = 0; i < total; i++) if (scales[i] == 0x7E00u) return RQO_ERR_NONFINITE;
+    }
+    return status;
+}
+
 /* ------------------------------------------------------------ products --- */
 
 /* Dequantised weight (n, k) = c * s16, exact in fp64. */

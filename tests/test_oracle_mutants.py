@@ -2,7 +2,8 @@
 
 Each case plants one mistake in a copy of the oracle's C source (on the CPU,
 in a temporary directory), builds it, swaps it in for the real oracle, and
-checks that at least one pin in test_oracle_pins.py fails.  The real oracle is
+checks that at least one pin in test_oracle_pins.py or test_oracle_ex2.py
+fails.  The real oracle is
 restored afterwards.
 """
 import ctypes
@@ -14,6 +15,7 @@ import numpy as np
 import pytest
 
 import oracle
+from tests import test_oracle_ex2 as ex2
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "rqo.c")
@@ -44,6 +46,16 @@ MUTANTS = {
     # scale from amax / (qmax + 1)
     "qmax_plus_one": ("volatile float s32 = amax / (float)qmax;",
                       "volatile float s32 = amax / (float)(qmax + 1);"),
+    # E[x^2] search: a tie goes to the later candidate
+    "ex2_ties_last": ("if (best < 0 || err < best_err) {", "if (best < 0 || err <= best_err) {"),
+    # E[x^2] search: the error is not weighted by E[x^2]
+    "ex2_unweighted": ("volatile float pr = e2[i] * q;", "volatile float pr = q;"),
+    # E[x^2] search: the candidate factor is ignored
+    "ex2_no_factor": ("volatile float a32 = amax * f[j];", "volatile float a32 = amax;"),
+    # E[x^2] search: absolute instead of squared error
+    "ex2_abs_error": ("volatile float q = d * d;", "volatile float q = fabsf(d);"),
+    # E[x^2] search: every group weighted by the first group's channels
+    "ex2_channel_index": ("&e2[g * RQO_GROUP]", "&e2[0]"),
 }
 
 PIN_TESTS = [
@@ -57,6 +69,11 @@ PIN_TESTS = [
     lambda: pins.test_exact_reconstruction_on_grid(8),
     lambda: pins.test_products_match_numpy_fp64(4),
     pins.test_unit_vector_picks_column,
+    ex2.test_hand_worked_group,
+    lambda: ex2.test_zero_weights_tie_first_wins(4),
+    lambda: ex2.test_single_factor_one_is_rtn(4),
+    lambda: ex2.test_matches_numpy_restatement(4, (3, 192)),
+    lambda: ex2.test_matches_numpy_restatement(8, (2, 256)),
 ]
 
 
@@ -79,8 +96,8 @@ def test_pins_catch_mutant(name):
     with tempfile.TemporaryDirectory() as tmp:
         so = _build_mutant(name, old, new, tmp)
         lib = ctypes.CDLL(so)
-        for fn in ("rqo_f32_to_f16", "rqo_f16_to_f64", "rqo_quantize_g64", "rqo_matmul",
-                   "rqo_matmul_sampled", "rqo_get_code"):
+        for fn in ("rqo_f32_to_f16", "rqo_f16_to_f64", "rqo_quantize_g64", "rqo_quantize_g64_ex2",
+                   "rqo_matmul", "rqo_matmul_sampled", "rqo_get_code"):
             getattr(lib, fn).argtypes = getattr(real, fn).argtypes
             getattr(lib, fn).restype = getattr(real, fn).restype
         caught = False
