@@ -92,6 +92,33 @@ rq_status rq_quantize_g64(const float *W, int64_t N, int64_t K, int bits,
                           rq_stream_t stream);
 
 /*
+ * rq_quantize_g64_ex2 -- group-64 symmetric quantization with the scale of
+ * each group chosen by an E[x^2]-weighted search ("rwkv-quant: uma matriz em
+ * bf16 elimina 39% das perdas na quantização do RWKV-7 2.9B", "Dois presets e
+ * seis tamanhos": the groups' scale is chosen by a search weighted by the mean
+ * square of the input channel's activation).  Same stored format as
+ * rq_quantize_g64.  Per group, candidate j (0 <= j < nf) has scale
+ * s16_j = fp16_rn(fp32(amax * factors[j]) / qmax) and RTN codes against it;
+ * its error is sum_k e2[k] * (w_k - c_k * s16_j)^2 over the group's 64 k in k
+ * order, every operation one IEEE fp32 rounding; the smallest error wins, the
+ * earlier candidate on a tie; a candidate whose scale overflows fp16 is never
+ * chosen (if all do, the group is quantized by RTN).  factors[0] = 1 makes
+ * the result never worse than RTN by this measure; nf = 1 with factor 1 is
+ * exactly rq_quantize_g64.
+ *
+ * W: fp32 [N, K] device, 16-byte aligned.  e2: fp32 [K] device, 16-byte
+ * aligned, E[x^2] per input channel (finite, >= 0; the caller's estimate).
+ * factors: fp32 [nf] device, 1 <= nf <= 16 (else RQ_ERR_RANGE).  codes,
+ * scales: outputs as for rq_quantize_g64.  chosen: nullable int32 [N, K/64]
+ * device, receives each group's winning candidate (0 for groups RTN
+ * handled).  dev_status: as for rq_quantize_g64.  Other argument errors as
+ * rq_quantize_g64.  Asynchronous on `stream`.
+ */
+rq_status rq_quantize_g64_ex2(const float *W, int64_t N, int64_t K, int bits, const float *e2,
+                              const float *factors, int nf, void *codes, uint16_t *scales,
+                              int32_t *chosen, int *dev_status, rq_stream_t stream);
+
+/*
  * rq_gemv_wq -- decode product y[M, N] = x[M, K] * w_hat^T for 1 <= M <= 32.
  * Streams each code and scale byte from HBM once.
  * x: fp16 [M, K] device.  codes/scales: as produced by rq_quantize_g64.

@@ -138,6 +138,23 @@ def test_decode_kernel_choice(L):
     assert L.rq_decode_kernel_for(1, D, D, 4, 1, None) == rq.ERR_NULL
 
 
+def test_quantize_ex2_argument_errors(L):
+    """rq_quantize_g64_ex2 rejects bad arguments before any CUDA call."""
+    p = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced
+    q = rq.lib().rq_quantize_g64_ex2
+    assert q(p, 4, 128, 4, p, p, 0, p, p, None, None, None) == rq.ERR_RANGE     # nf = 0
+    assert q(p, 4, 128, 4, p, p, 17, p, p, None, None, None) == rq.ERR_RANGE    # nf > 16
+    assert q(p, 4, 128, 5, p, p, 4, p, p, None, None, None) == rq.ERR_BITS
+    assert q(p, 4, 100, 4, p, p, 4, p, p, None, None, None) == rq.ERR_SHAPE
+    assert q(p, 0, 128, 4, p, p, 4, p, p, None, None, None) == rq.ERR_SHAPE
+    assert q(None, 4, 128, 4, p, p, 4, p, p, None, None, None) == rq.ERR_NULL
+    assert q(p, 4, 128, 4, None, p, 4, p, p, None, None, None) == rq.ERR_NULL
+    assert q(p, 4, 128, 4, p, None, 4, p, p, None, None, None) == rq.ERR_NULL
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert q(p, 4, 128, 4, odd, p, 4, p, p, None, None, None) == rq.ERR_ALIGN   # e2 not 16-B
+    assert q(p, 4, 128, 4, p, ctypes.c_void_p((1 << 20) + 2), 4, p, p, None, None, None) == rq.ERR_ALIGN
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(rq, "_lib", None)
     monkeypatch.setattr(rq, "LIB_PATH", str(tmp_path / "missing.so"))

@@ -240,6 +240,22 @@ rq_status rq_quantize_g64(const float* W, int64_t N, int64_t K, int bits, void* 
     return e == cudaSuccess ? RQ_OK : cuda_fail(e);
 }
 
+rq_status rq_quantize_g64_ex2(const float* W, int64_t N, int64_t K, int bits, const float* e2,
+                              const float* factors, int nf, void* codes, uint16_t* scales,
+                              int32_t* chosen, int* dev_status, rq_stream_t stream) {
+    rq_status st = check_weight_shape(N, K, bits);
+    if (st != RQ_OK) return st;
+    if (nf < 1 || nf > 16) return RQ_ERR_RANGE;
+    if (W == nullptr || e2 == nullptr || factors == nullptr || codes == nullptr || scales == nullptr)
+        return RQ_ERR_NULL;
+    if (!aligned16(W) || !aligned16(e2) || !aligned16(codes) || !aligned16(scales)) return RQ_ERR_ALIGN;
+    const auto mis4 = [](const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u); };
+    if (mis4(factors) || mis4(chosen) || mis4(dev_status)) return RQ_ERR_ALIGN;
+    cudaError_t e = launch_quantize_ex2(W, N, K, bits, e2, factors, nf, codes, scales, chosen,
+                                        dev_status, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
 rq_status rq_gemv_wq(const uint16_t* x, int64_t M, int64_t K, const void* codes,
                      const uint16_t* scales, int64_t N, int bits, float* y, rq_stream_t stream) {
     rq_status st = check_product(x, M, K, N, bits, RQ_MAX_DECODE_M);

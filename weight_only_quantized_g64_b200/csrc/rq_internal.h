@@ -17,6 +17,11 @@ constexpr int kGroup = 64;
 cudaError_t launch_quantize(const float* W, int64_t n_groups, int bits, void* codes,
                             uint16_t* scales, int* dev_status, cudaStream_t s);
 
+// Quantizer with an E[x^2]-weighted scale search (nf <= 16 candidates).
+cudaError_t launch_quantize_ex2(const float* W, int64_t N, int64_t K, int bits, const float* e2,
+                                const float* factors, int nf, void* codes, uint16_t* scales,
+                                int32_t* chosen, int* dev_status, cudaStream_t s);
+
 // One weight operand of a product: its TMA descriptor (codes), scales, output.
 struct WOperand {
     const void* codes;

@@ -99,4 +99,143 @@ cudaError_t launch_quantize(const float* W, int64_t n_groups, int bits, void* co
     return cudaGetLastError();
 }
 
+
+// ------------------------------------------- E[x^2]-weighted scale search --
+//
+// "rwkv-quant: uma matriz em bf16 elimina 39% das perdas na quantização do
+// RWKV-7 2.9B", section "Dois presets e seis tamanhos": a group's scale is
+// chosen by a search weighted by E[x^2], the mean square of the input
+// channel's activation.  On the symmetric g64 grid: candidate j has scale
+// s16_j = fp16_rn(fp32(amax * f[j]) / qmax) and RTN codes against it; its
+// error is sum_k e2[k] * (w_k - c_k * s16_j)^2 over the group's 64 k, in k
+// order, each operation one IEEE fp32 rounding (explicit _rn intrinsics: no
+// contraction); the candidate with the smallest error wins, the earlier one
+// on a tie, and one whose scale overflows is never chosen (if every one
+// does, the group is quantized by RTN).
+//
+// Layout of the work: as the RTN kernel, 16 threads per group, one float4 of
+// weights and one of E[x^2] each.  Thread j evaluates candidate j (nf <= 16)
+// over all 64 weights, fetched by shuffles in k order, so its sum runs in the
+// same order as a scalar loop; lane 0 then scans the candidates in order
+// (the same comparisons as a sequential argmin, NaN included).
+template <int BITS>
+__global__ void __launch_bounds__(256) quantize_g64_ex2_kernel(
+    const float4* __restrict__ W, int64_t n_groups, int64_t groups_per_row,
+    const float4* __restrict__ e2, const float* __restrict__ factors, int nf,
+    uint8_t* __restrict__ codes, uint16_t* __restrict__ scales, int32_t* __restrict__ chosen,
+    int* __restrict__ dev_status) {
+    constexpr int kQmax = BITS == 4 ? 7 : 127;
+    const int lane16 = threadIdx.x & 15;
+    const int base = threadIdx.x & 16;                      // first lane of this half-warp
+    const unsigned half_mask = 0xFFFFu << base;
+    const int64_t first = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+    const int64_t step = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
+    const float fj = lane16 < nf ? factors[lane16] : 1.0f;
+
+    for (int64_t gid = first; gid < n_groups; gid += step) {
+        const float4 v = __ldcs(&W[gid * 16 + lane16]);
+        const float4 ev = __ldg(&e2[(gid % groups_per_row) * 16 + lane16]);
+        const bool finite = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+        float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(half_mask, a, off));
+        const bool all_finite = __all_sync(half_mask, finite);
+
+        // ---- candidate lane16: scale, then its error over the 64 weights
+        const float a32 = __fmul_rn(a, fj);
+        const __half s16j = __float2half_rn(__fdiv_rn(a32, static_cast<float>(kQmax)));
+        const float sfj = __half2float(s16j);
+        const bool valid = lane16 < nf && __half_as_ushort(s16j) != 0x7C00u;
+        const float wv[4] = {v.x, v.y, v.z, v.w};
+        const float evv[4] = {ev.x, ev.y, ev.z, ev.w};
+        float err = 0.0f;
+#pragma unroll 4
+        for (int k = 0; k < 64; ++k) {
+            const float wk = __shfl_sync(half_mask, wv[k & 3], base + (k >> 2));
+            const float ek = __shfl_sync(half_mask, evv[k & 3], base + (k >> 2));
+            int c = 0;
+            if (sfj != 0.0f) c = max(-kQmax, min(kQmax, __float2int_rn(__fdiv_rn(wk, sfj))));
+            const float t = __fmul_rn(static_cast<float>(c), sfj);
+            const float d = __fsub_rn(wk, t);
+            err = __fadd_rn(err, __fmul_rn(ek, __fmul_rn(d, d)));
+        }
+        // ---- lane 0 scans the candidates in order (a sequential argmin)
+        int best = -1;
+        float best_err = 0.0f;
+        for (int j = 0; j < nf; ++j) {
+            const float ej = __shfl_sync(half_mask, err, base + j);
+            const int vj = __shfl_sync(half_mask, valid ? 1 : 0, base + j);
+            if (vj && (best < 0 || ej < best_err)) {
+                best = j;
+                best_err = ej;
+            }
+        }
+        best = __shfl_sync(half_mask, best, base);
+
+        // ---- the chosen scale (or RTN when no candidate is valid) and codes
+        const float fb = best >= 0 ? __shfl_sync(half_mask, fj, base + best) : 1.0f;
+        const float s32 = best >= 0 ? __fdiv_rn(__fmul_rn(a, fb), static_cast<float>(kQmax))
+                                    : __fdiv_rn(a, static_cast<float>(kQmax));
+        const __half s16 = __float2half_rn(s32);
+        uint16_t s_bits = __half_as_ushort(s16);
+        const float sf = __half2float(s16);
+        int status = 0;
+        int c[4] = {0, 0, 0, 0};
+        if (!all_finite) {
+            s_bits = 0x7E00u;
+            status = 5;  // RQ_ERR_NONFINITE
+        } else if (s_bits == 0x7C00u) {
+            status = 6;  // RQ_ERR_RANGE
+        } else if (sf != 0.0f) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int q = __float2int_rn(__fdiv_rn(wv[i], sf));
+                c[i] = max(-kQmax, min(kQmax, q));
+            }
+        }
+        if (BITS == 4) {
+            const uint16_t packed = static_cast<uint16_t>((c[0] & 0xF) | ((c[1] & 0xF) << 4) |
+                                                          ((c[2] & 0xF) << 8) |
+                                                          ((c[3] & 0xF) << 12));
+            __stcs(reinterpret_cast<unsigned short*>(codes + gid * 32 + lane16 * 2), packed);
+        } else {
+            const uint32_t packed = (c[0] & 0xFF) | ((c[1] & 0xFF) << 8) | ((c[2] & 0xFF) << 16) |
+                                    (static_cast<uint32_t>(c[3] & 0xFF) << 24);
+            __stcs(reinterpret_cast<unsigned int*>(codes + gid * 64 + lane16 * 4), packed);
+        }
+        if (lane16 == 0) {
+            scales[gid] = s_bits;
+            if (chosen != nullptr) chosen[gid] = (all_finite && best >= 0) ? best : 0;
+            if (dev_status != nullptr) {
+                if (status == 5) atomicExch(dev_status, 5);
+                else if (status == 6) atomicCAS(dev_status, 0, 6);
+            }
+        }
+    }
+}
+
+cudaError_t launch_quantize_ex2(const float* W, int64_t N, int64_t K, int bits, const float* e2,
+                                const float* factors, int nf, void* codes, uint16_t* scales,
+                                int32_t* chosen, int* dev_status, cudaStream_t s) {
+    const int64_t groups_per_row = K / kGroup;
+    const int64_t n_groups = N * groups_per_row;
+    if (n_groups <= 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t groups_per_block = threads / 16;
+    int64_t blocks = (n_groups + groups_per_block - 1) / groups_per_block;
+    const int64_t cap = 148LL * 8 * 4;
+    if (blocks > cap) blocks = cap;
+    if (bits == 4)
+        quantize_g64_ex2_kernel<4><<<static_cast<unsigned>(blocks), threads, 0, s>>>(
+            reinterpret_cast<const float4*>(W), n_groups, groups_per_row,
+            reinterpret_cast<const float4*>(e2), factors, nf, static_cast<uint8_t*>(codes), scales,
+            chosen, dev_status);
+    else
+        quantize_g64_ex2_kernel<8><<<static_cast<unsigned>(blocks), threads, 0, s>>>(
+            reinterpret_cast<const float4*>(W), n_groups, groups_per_row,
+            reinterpret_cast<const float4*>(e2), factors, nf, static_cast<uint8_t*>(codes), scales,
+            chosen, dev_status);
+    return cudaGetLastError();
+}
+
 }  // namespace rq

@@ -52,6 +52,8 @@ def lib():
     L.rq_scales_bytes.restype = ctypes.c_size_t
     L.rq_quantize_g64.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
     L.rq_quantize_g64.restype = i32
+    L.rq_quantize_g64_ex2.argtypes = [vp, i64, i64, i32, vp, vp, i32, vp, vp, vp, vp, vp]
+    L.rq_quantize_g64_ex2.restype = i32
     L.rq_gemv_wq.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, vp]
     L.rq_gemv_wq.restype = i32
     L.rq_gemm_wq.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, vp]
@@ -127,6 +129,22 @@ def quantize_g64(W: torch.Tensor, bits: int, codes=None, scales=None, dev_status
     _check(lib().rq_quantize_g64(_p(W), N, K, bits, _p(codes), _p(scales), _p(dev_status),
                                  _stream(stream)), "rq_quantize_g64")
     return codes, scales
+
+
+def quantize_g64_ex2(W: torch.Tensor, e2: torch.Tensor, bits: int, factors: torch.Tensor,
+                     codes=None, scales=None, chosen=None, dev_status=None, stream=None):
+    """Group-64 quantization of fp32 W[N, K] with each group's scale chosen by
+    an E[x^2]-weighted search over `factors` (fp32 device, 1..16 values);
+    e2: fp32 [K] device.  Returns (codes, scales, chosen int32 [N, K/64])."""
+    N, K = W.shape
+    if codes is None:
+        codes, scales = empty_weights(N, K, bits, W.device)
+    if chosen is None:
+        chosen = torch.empty((N, K // GROUP), dtype=torch.int32, device=W.device)
+    _check(lib().rq_quantize_g64_ex2(_p(W), N, K, bits, _p(e2), _p(factors), int(factors.numel()),
+                                     _p(codes), _p(scales), _p(chosen), _p(dev_status),
+                                     _stream(stream)), "rq_quantize_g64_ex2")
+    return codes, scales, chosen
 
 
 def gemv_wq(x: torch.Tensor, codes, scales, N: int, bits: int, y=None, stream=None):
