@@ -48,7 +48,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # until a new capture is taken.
 DECODE_SOURCES = ("rq_api.cu", "rq_gemv.cu", "rq_gemv_ck.cu", "rq_gemv_unit.cuh", "rq_ptx.cuh",
                   "rq_internal.h")
-DECODE_TRAFFIC = {"code_sha256_16": "8058f31dc68f7887", "bytes_per_launch": 6823383}
+DECODE_TRAFFIC = {"code_sha256_16": "076aa3b7224c42d8", "bytes_per_launch": 6823383}
 
 
 def decode_code_hash():
