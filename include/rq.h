@@ -29,10 +29,12 @@
  * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  * stream).  Argument errors are found before any launch and returned
  * synchronously; nothing is launched then.  The library allocates no device
- * memory per call; pointers must stay valid until the stream reaches the
- * call.  Inputs and outputs must not overlap.  All pointers must be 16-byte
- * aligned.  A call that fails to launch returns RQ_ERR_CUDA (the CUDA error
- * string is available from rq_last_cuda_error()).
+ * memory per call, except the decode products' workspace, allocated the
+ * first time a shape needs it (see rq_gemv_wq); pointers must stay valid
+ * until the stream reaches the call.  Inputs and outputs must not overlap.
+ * Array pointers must be 16-byte aligned unless a call states otherwise.  A
+ * call that fails to launch returns RQ_ERR_CUDA (the CUDA error string is
+ * available from rq_last_cuda_error()).
  */
 #ifndef RQ_H_
 #define RQ_H_
@@ -108,10 +110,11 @@ rq_status rq_quantize_g64(const float *W, int64_t N, int64_t K, int bits,
  *
  * W: fp32 [N, K] device, 16-byte aligned.  e2: fp32 [K] device, 16-byte
  * aligned, E[x^2] per input channel (finite, >= 0; the caller's estimate).
- * factors: fp32 [nf] device, 1 <= nf <= 16 (else RQ_ERR_RANGE).  codes,
- * scales: outputs as for rq_quantize_g64.  chosen: nullable int32 [N, K/64]
- * device, receives each group's winning candidate (0 for groups RTN
- * handled).  dev_status: as for rq_quantize_g64.  Other argument errors as
+ * factors: fp32 [nf] device, 4-byte aligned, 1 <= nf <= 16 (else
+ * RQ_ERR_RANGE).  codes, scales: outputs as for rq_quantize_g64.  chosen:
+ * nullable int32 [N, K/64] device, 4-byte aligned, receives each group's
+ * winning candidate (0 for groups RTN handled).  dev_status: as for
+ * rq_quantize_g64.  Other argument errors as
  * rq_quantize_g64.  Asynchronous on `stream`.
  */
 rq_status rq_quantize_g64_ex2(const float *W, int64_t N, int64_t K, int bits, const float *e2,
@@ -123,6 +126,11 @@ rq_status rq_quantize_g64_ex2(const float *W, int64_t N, int64_t K, int bits, co
  * Streams each code and scale byte from HBM once.
  * x: fp16 [M, K] device.  codes/scales: as produced by rq_quantize_g64.
  * y: fp32 [M, N] device, fully overwritten.  Requires K % 64 == 0, N >= 1.
+ * Two kernels compute it (rq_set_decode_kernel, rq_decode_kernel_for): the
+ * row-tile kernel keeps the partial sums of row tiles shared by several
+ * blocks in a device workspace that the library allocates (and grows) the
+ * first time a shape needs it -- make that first call outside any stream
+ * capture, or use rq_gemv_wq_noalloc; the cluster kernel needs no workspace.
  */
 rq_status rq_gemv_wq(const uint16_t *x, int64_t M, int64_t K, const void *codes,
                      const uint16_t *scales, int64_t N, int bits, float *y,
