@@ -2,14 +2,21 @@
 """Benchmark: decode weight GB/s (and prefill TFLOP/s) of group-64 quantized
 RWKV-7 projections on B200, through librq's C ABI.
 
-Default workload: the RWKV-7 1.5B-shaped int4 g64 decode layer (D = 2048:
-fused R/K/V 3 x 2048^2, O 2048^2, channel-mix key 2048->8192 and value
-8192->2048), over the model's 24 layers, at every batch M in {1, 4, 8, 16, 32}.
-One step = one decode pass through the 24-layer projection stack at each M
-(5 x 24 x 4 kernel launches), replayed from CUDA graphs.  The weights
-(642 MB) are larger than L2, so every step streams them from HBM.
+Default workload: the 13.3B-shaped int4 g64 decode stack -- 61 RWKV-7 layers
+of width D = 4096, each with fused R/K/V (3 x 4096^2), O 4096^2, channel-mix
+key 4096->16384 and value 16384->4096 -- at every batch M in {1, 2, 4, 8, 16,
+32}.  One step = one decode pass through the 61-layer projection stack at each
+M (6 x 61 x 4 kernel launches), replayed from CUDA graphs.  The weights
+(6.52 GB of codes and scales per pass) are far larger than L2, so every step
+streams them from HBM.  `--workload 2` / `3` run the 1.5B-shaped int4 and the
+2.9B-shaped int8 stacks instead.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py --case gemv|rkv|gemm|quantize|quantize_ex2 --shape NxK --M m [--bits b]
+
+`--case` runs one product (or quantizer) call per repeat on a single weight
+copy with nothing timed: the launch a profiler captures (`ncu -k ... -s 1`
+skips the first, warm-up call).
 
 Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank decodes its
 own batch through its own copy of the stack (independent replicas, no
@@ -40,9 +47,8 @@ METRIC = "decode w4g64 GEMV weight GB/s (% of B200 HBM peak); prefill TFLOP/s; 1
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# DRAM traffic of the decode kernels, from one ncu launch list of a timed step
-# (dram__bytes_read.sum + dram__bytes_write.sum over the step's 480 launches,
-# averaged per launch; profiles/launches_decode_1p5b_int4_24layers.md).  It
+# DRAM traffic of the decode kernels per launch (dram__bytes_read.sum +
+# dram__bytes_write.sum from an ncu capture, see the profile summaries).  It
 # is valid only for the kernel code it was taken on: when the code's hash
 # (comments and whitespace ignored) differs, the bench reports traffic as null
 # until a new capture is taken.
@@ -325,7 +331,7 @@ def reference_arm(args, wl, rank, world):
 
 # ------------------------------------------------------ prefill, quantizer --
 
-def bench_prefill(hbm_peak, tf_peak, reps=5):
+def bench_prefill(hbm_peak, tf_peak, reps=50):
     wl = synth.WORKLOADS[4]
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")  # 256 MB
     weights = []
@@ -362,7 +368,7 @@ def bench_prefill(hbm_peak, tf_peak, reps=5):
     return out
 
 
-def bench_quantizer(hbm_peak, reps=5):
+def bench_quantizer(hbm_peak, reps=50):
     N, K = 16384, 4096
     W = synth.weights(N, K, seed=5, device="cuda")
     codes, scales = rq.empty_weights(N, K, 4)
@@ -384,19 +390,66 @@ def bench_quantizer(hbm_peak, reps=5):
             "frac": byts / ms / 1e6 / hbm_peak}
 
 
+# ------------------------------------------------------- profiling case --
+
+def run_case(args):
+    """One call per repeat of a single product or quantizer on one weight
+    copy, synchronised after each call; nothing is timed or printed but a
+    status line.  The launch a profiler captures."""
+    rq_build.build()
+    torch.cuda.set_device(0)
+    rq.lib()
+    N, K = (int(t) for t in args.shape.split("x"))
+    W = synth.weights(N, K, seed=5, device="cuda")
+    if args.case == "quantize":
+        for _ in range(args.repeat):
+            rq.quantize_g64(W, args.bits)
+            torch.cuda.synchronize()
+    elif args.case == "quantize_ex2":
+        e2 = synth.activations(64, K, seed=6, device="cuda").float().pow(2).mean(0)
+        factors = torch.tensor([1.0, 0.95, 0.9, 0.85, 0.8, 0.75, 0.7], device="cuda")
+        for _ in range(args.repeat):
+            rq.quantize_g64_ex2(W, e2, args.bits, factors)
+            torch.cuda.synchronize()
+    else:
+        w = rq.quantize_g64(W, args.bits)
+        del W
+        x = synth.activations(args.M, K, seed=7, device="cuda")
+        for _ in range(args.repeat):
+            if args.case == "gemv":
+                rq.gemv_wq(x, w[0], w[1], N, args.bits)
+            elif args.case == "rkv":
+                rq.rkv_fused(x, w, w, w, N, args.bits)
+            else:
+                rq.gemm_wq(x, w[0], w[1], N, args.bits)
+            torch.cuda.synchronize()
+    print(f"case {args.case} {args.shape} M={args.M} bits={args.bits} x{args.repeat}: ok "
+          f"(device status {rq.read_device_status(reset=True)})", flush=True)
+
+
 # ------------------------------------------------------------------ main --
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
+    ap.add_argument("--workload", type=int, default=5, choices=[2, 3, 5])
+    ap.add_argument("--case", default=None,
+                    choices=["gemv", "rkv", "gemm", "quantize", "quantize_ex2"],
+                    help="one call per repeat of a single product or quantizer (profiling target)")
+    ap.add_argument("--shape", default="4096x4096", help="NxK of --case")
+    ap.add_argument("--M", type=int, default=1, help="batch of --case")
+    ap.add_argument("--bits", type=int, default=4, choices=[4, 8], help="bits of --case")
+    ap.add_argument("--repeat", type=int, default=2, help="calls of --case")
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--skip-extras", action="store_true",
                     help="decode only (no prefill/quantizer/cpu baseline/e2e)")
     args = ap.parse_args()
+    if args.case is not None:
+        run_case(args)
+        return
     wl = synth.WORKLOADS[args.workload]
 
     if args.impl == "reference":

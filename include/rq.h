@@ -128,9 +128,16 @@ rq_status rq_quantize_g64_ex2(const float *W, int64_t N, int64_t K, int bits, co
  * y: fp32 [M, N] device, fully overwritten.  Requires K % 64 == 0, N >= 1.
  * Two kernels compute it (rq_set_decode_kernel, rq_decode_kernel_for): the
  * row-tile kernel keeps the partial sums of row tiles shared by several
- * blocks in a device workspace that the library allocates (and grows) the
- * first time a shape needs it -- make that first call outside any stream
- * capture, or use rq_gemv_wq_noalloc; the cluster kernel needs no workspace.
+ * blocks in a device workspace that the library allocates the first time a
+ * shape needs it (at least 32 MiB of slots and 2^18 counters per device) --
+ * make that first call outside any stream capture, or use
+ * rq_gemv_wq_noalloc; the cluster kernel needs no workspace.  When a later
+ * shape needs a larger workspace, a larger one is allocated and the old one
+ * is kept until the process exits, so CUDA graphs captured earlier stay valid.
+ * Workspace sharing: every rq_gemv_wq and rq_rkv_fused call on one device uses
+ * the same workspace, so two such calls that may run at the same time on the
+ * GPU (e.g. on two streams with no ordering between them) race on it and can
+ * give wrong results; order them on one stream or with events.
  */
 rq_status rq_gemv_wq(const uint16_t *x, int64_t M, int64_t K, const void *codes,
                      const uint16_t *scales, int64_t N, int bits, float *y,
@@ -141,7 +148,8 @@ rq_status rq_gemv_wq(const uint16_t *x, int64_t M, int64_t K, const void *codes,
  * time-mix block, sharing one input x, in ONE kernel launch:
  *   yR = x * w_hat_R^T,  yK = x * w_hat_K^T,  yV = x * w_hat_V^T.
  * All three weights are N x K with the same bits.  Same rules as rq_gemv_wq
- * (1 <= M <= 32).
+ * (1 <= M <= 32), including its workspace: calls of rq_gemv_wq and
+ * rq_rkv_fused that may overlap on the GPU race on it.
  */
 rq_status rq_rkv_fused(const uint16_t *x, int64_t M, int64_t K, int64_t N, int bits,
                        const void *codes_r, const uint16_t *scales_r,
@@ -184,9 +192,10 @@ rq_status rq_gemm_wq(const uint16_t *x, int64_t M, int64_t K, const void *codes,
  * A call that runs on the row-tile kernel (see rq_set_decode_kernel) clears
  * the counters it uses (an asynchronous memset on `stream`) and then launches
  * the product; one that runs on the cluster kernel needs no scratch and
- * launches only the product.  All calls share the one array: calls that
- * overlap on the GPU (different streams, or several devices' calls mixed
- * without ordering) race with each other and give wrong results.
+ * launches only the product.  Each device has its own copy of the array, and
+ * all calls on one device share it: calls that may overlap on the same device
+ * (e.g. on two streams with no ordering between them) race on it and give
+ * wrong results.
  */
 rq_status rq_gemv_wq_noalloc(const uint16_t *x, int64_t M, int64_t K, const void *codes,
                              const uint16_t *scales, int64_t N, int bits, float *y,

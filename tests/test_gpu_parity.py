@@ -150,6 +150,27 @@ def test_gemm_parity(bits, M):
     check_close(to_host(y), y_ref, bound, f"gemm bits={bits} M={M}")
 
 
+# Ragged shapes of the tensor-core product on full outputs: N not a multiple
+# of the 128-row MMA tile (1, 129, 257, 300), a single k-block (K = 64), three
+# (K = 192), a k-block count that no cluster split divides evenly (K = 64*37),
+# and token counts that leave a partial token tile (65, 130, 2047).
+GEMM_RAGGED = [
+    (65, 1, 64), (65, 129, 192), (64, 300, 64 * 37), (130, 300, 64), (2047, 129, 512),
+    (256, 129, 4096), (300, 257, 64 * 37), (1, 129, 192), (100, 1, 64 * 37), (2047, 1, 192),
+]
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,N,K", GEMM_RAGGED)
+def test_gemm_parity_ragged(bits, M, N, K):
+    x, codes, scales = product_case(N, K, bits, M, seed=3100 + M + N + K)
+    cd, sd = upload(codes, scales)
+    y = rq.gemm_wq(x, cd, sd, N, bits)
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.matmul(to_host(x), codes, scales, bits)
+    check_close(to_host(y), y_ref, bound, f"gemm ragged bits={bits} M={M} N={N} K={K}")
+
+
 def test_unit_vectors_pick_columns():
     """x = e_j returns column j of the dequantised weight (exact up to fp32)."""
     N, K, bits = 130, 192, 4

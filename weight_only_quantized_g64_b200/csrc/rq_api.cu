@@ -54,11 +54,18 @@ int decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat) {
 
 
 // ------------------------------------------------------------- workspace --
+// Per-device scratch of the row-tile decode kernel.  When a launch needs more
+// than the current buffers hold, larger ones are allocated and the old ones
+// are kept (never freed before the process exits): a CUDA graph captured
+// earlier may still hold their addresses, and replaying it must not touch
+// freed memory.  The old counters stay zero (every completed launch leaves
+// them so), and the old slots are only ever written by replays of such graphs.
 struct Workspace {
     float* ws = nullptr;
     size_t ws_bytes = 0;
     int* cnt = nullptr;
     size_t n_cnt = 0;
+    int retired = 0;   // buffers replaced by larger ones and kept alive
 };
 static Workspace g_ws[kMaxDevices];
 
@@ -72,32 +79,22 @@ cudaError_t workspace_get(size_t ws_bytes, size_t n_counters, float** ws, int** 
     if (w.ws_bytes < ws_bytes) {
         const size_t want = ws_bytes > (size_t{32} << 20) ? ws_bytes : (size_t{32} << 20);
         void* p = nullptr;
-        if (w.ws != nullptr) {
-            e = cudaFree(w.ws);
-            if (e != cudaSuccess) return e;
-            w.ws = nullptr;
-            w.ws_bytes = 0;
-        }
         e = cudaMalloc(&p, want);
         if (e != cudaSuccess) return e;
+        if (w.ws != nullptr) ++w.retired;
         w.ws = static_cast<float*>(p);
         w.ws_bytes = want;
     }
     if (w.n_cnt < n_counters) {
         const size_t want = n_counters > (size_t{1} << 18) ? n_counters : (size_t{1} << 18);
         void* p = nullptr;
-        if (w.cnt != nullptr) {
-            e = cudaFree(w.cnt);
-            if (e != cudaSuccess) return e;
-            w.cnt = nullptr;
-            w.n_cnt = 0;
-        }
         e = cudaMalloc(&p, want * sizeof(int));
         if (e != cudaSuccess) return e;
         e = cudaMemset(p, 0, want * sizeof(int));
         if (e != cudaSuccess) return e;
         e = cudaDeviceSynchronize();
         if (e != cudaSuccess) return e;
+        if (w.cnt != nullptr) ++w.retired;
         w.cnt = static_cast<int*>(p);
         w.n_cnt = want;
     }
