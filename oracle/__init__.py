@@ -77,6 +77,8 @@ def _load():
     lib.rqo_matmul_sampled.restype = None
     lib.rqo_get_code.argtypes = [vp, i64, ctypes.c_int, i64, i64]
     lib.rqo_get_code.restype = ctypes.c_int
+    lib.rqo_gptq_g64.argtypes = [vp, i64, i64, ctypes.c_int, vp, vp, vp, vp]
+    lib.rqo_gptq_g64.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -174,3 +176,53 @@ def matmul_sampled(x_f16: np.ndarray, codes: np.ndarray, scales: np.ndarray,
 def get_code(codes: np.ndarray, K: int, bits: int, n: int, k: int) -> int:
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     return int(_load().rqo_get_code(_ptr(codes), K, bits, n, k))
+
+
+# ------------------------------------------------------------------ GPTQ ---
+# GPTQ on the symmetric group-64 grid ("Hakureirm/rwkv7-sglang-w4gptq-1.5b"
+# model card, opening summary: GPTQ-calibrated, symmetric, group 64, same
+# format as RTN; "rwkv-quant: uma matriz em bf16 elimina 39% das perdas na
+# quantização do RWKV-7 2.9B", "Vazamento de calibração e medições honestas":
+# GPTQ on the preset's grid, format and kernels unchanged).  The method is
+# the published GPTQ (Frantar et al., arXiv:2210.17323).
+
+GPTQ_DAMP = 0.01
+
+
+def gptq_prepare(X_f16: np.ndarray, damp: float = GPTQ_DAMP):
+    """The inverse-Hessian factor of GPTQ for calibration inputs X (fp16
+    [T, K], T tokens), in fp64 with numpy, following the method's steps:
+    H = 2 X^T X / T; a column whose input is always zero (H[j, j] == 0) is
+    marked dead and gets H[j, j] = 1; H += damp * mean(diag H) * I; then
+    H^-1 through the Cholesky factor of H, and U = the upper Cholesky factor
+    of H^-1 (H^-1 = U^T U).  Returns (U float64 [K, K], dead uint8 [K])."""
+    X = np.ascontiguousarray(X_f16).astype(np.float64)
+    T, K = X.shape
+    H = (2.0 / T) * (X.T @ X)
+    dead = np.diag(H) == 0
+    H[dead, dead] = 1.0
+    H[np.diag_indices(K)] += damp * np.mean(np.diag(H))
+    L = np.linalg.cholesky(H)                       # H = L L^T
+    Linv = np.linalg.inv(L)
+    Hinv = Linv.T @ Linv                            # H^-1
+    U = np.linalg.cholesky(Hinv).T                  # H^-1 = U^T U, U upper
+    return np.ascontiguousarray(U), dead.astype(np.uint8)
+
+
+def gptq_g64(W: np.ndarray, bits: int, U: np.ndarray, dead=None):
+    """The GPTQ column loop on the group-64 grid (rqo.c, fp32): W fp32 [N, K],
+    U the upper factor (rounded to fp32 here), dead uint8 [K] or None.
+    Returns (codes, scales, W_compensated, status)."""
+    Wc = np.array(W, dtype=np.float32, order="C", copy=True)
+    N, K = Wc.shape
+    if bits not in (4, 8) or K % GROUP:
+        raise ValueError("bits must be 4 or 8 and K a multiple of 64")
+    U32 = np.ascontiguousarray(U, dtype=np.float32)
+    if U32.shape != (K, K):
+        raise ValueError("U must be K x K")
+    d = None if dead is None else np.ascontiguousarray(dead, dtype=np.uint8)
+    codes = np.zeros((N, K * bits // 8), dtype=np.uint8)
+    scales = np.zeros((N, K // GROUP), dtype=np.uint16)
+    st = _load().rqo_gptq_g64(_ptr(Wc), N, K, bits, _ptr(U32), _ptr(d) if d is not None else None,
+                              _ptr(codes), _ptr(scales))
+    return codes, scales, Wc, int(st)

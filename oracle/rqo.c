@@ -372,3 +372,116 @@ int rqo_quantize_rows(const float *Wrows, int64_t rows, int64_t K, int bits,
 {
     return rqo_quantize_g64(Wrows, rows, K, bits, codes, scales);
 }
+
+/* ------------------------------------------------------------------ GPTQ --- */
+/*
+ * GPTQ on the symmetric group-64 grid.  "Hakureirm/rwkv7-sglang-w4gptq-1.5b"
+ * model card, opening summary: the int4 checkpoint is GPTQ-calibrated,
+ * symmetric, group 64, in the same .qweight + .scale format as the
+ * calibration-free RTN it is compared with; "rwkv-quant: uma matriz em bf16
+ * elimina 39% das perdas na quantização do RWKV-7 2.9B", "Vazamento de
+ * calibração e medições honestas": GPTQ runs on the preset's grid without
+ * changing the format, the kernels or the file size.  The method is the
+ * published GPTQ (Frantar et al., arXiv:2210.17323, which the RWKVQuant page
+ * lists among the works it builds on): quantize the columns of W in order and
+ * spread each column's rounding error over the columns not yet quantized,
+ * weighted by the inverse Hessian H^-1 of the layer's input (H = 2 X^T X / T
+ * plus damping), through U, the upper Cholesky factor of H^-1 (H^-1 = U^T U).
+ *
+ * This function is the column loop, given U (fp32, row-major [K, K], upper
+ * triangle read) and the dead-input mask (columns whose input never varies:
+ * their weights are zeroed first).  Readings where the pages are silent:
+ *   - the group's scale is found when the loop reaches the group's first
+ *     column, from the CURRENT (already error-compensated) weights of the
+ *     group's 64 columns, exactly as RTN finds it (fp32 amax / qmax, fp16
+ *     round to nearest even); each column's code is then RTN against that
+ *     stored scale: c_j = clamp(rint(w_j / s16), -qmax, qmax);
+ *   - every operation is one fp32 rounding, in this order:
+ *       d   = w_j - c_j * s16          (the product is exact in fp32)
+ *       e_j = d / U[j][j]
+ *       w_k = fmaf(-e_j, U[j][k], w_k)  for k = j+1 .. K-1, j ascending;
+ *   - a group whose scale is unusable (a non-finite weight: scale 0x7E00,
+ *     status NONFINITE; fp16 overflow: scale 0x7C00, status RANGE) gets codes
+ *     0 and spreads no error (e_j = 0) from its columns;
+ *   - a scale of zero (the group's weights are all zero when it starts) gives
+ *     codes 0 with the error spread as usual.
+ * W is overwritten with the compensated weights.  Returns the status, as
+ * rqo_quantize_g64 does (NONFINITE over RANGE over OK).
+ */
+static int gptq_row(float *w, int64_t K, int bits, const float *U, const uint8_t *dead,
+                    uint8_t *codes_row_base, int64_t n, uint16_t *scales_row)
+{
+    const int qmax = qmax_of(bits);
+    int status = RQO_OK;
+    int64_t j, k;
+    if (dead)
+        for (j = 0; j < K; j++) if (dead[j]) w[j] = 0.0f;
+    float sf = 0.0f;
+    int usable = 1;
+    for (j = 0; j < K; j++) {
+        if (j % RQO_GROUP == 0) {
+            /* the group's scale, from its current weights */
+            int i, finite = 1;
+            float amax = 0.0f;
+            for (i = 0; i < RQO_GROUP; i++) {
+                float v = w[j + i];
+                if (!isfinite(v)) finite = 0;
+                float a = fabsf(v);
+                if (a > amax) amax = a;
+            }
+            uint16_t s16;
+            if (!finite) {
+                s16 = 0x7E00u;
+                usable = 0;
+                status = RQO_ERR_NONFINITE;
+            } else {
+                volatile float s32 = amax / (float)qmax;
+                s16 = rqo_f32_to_f16(s32);
+                usable = s16 != 0x7C00u;
+                if (!usable && status == RQO_OK) status = RQO_ERR_RANGE;
+            }
+            scales_row[j / RQO_GROUP] = s16;
+            sf = usable ? (float)rqo_f16_to_f64(s16) : 0.0f;
+        }
+        int c = 0;
+        float e = 0.0f;
+        if (usable) {
+            if (sf != 0.0f) {
+                volatile float t = w[j] / sf;
+                float r = rintf(t);
+                if (r > (float)qmax) r = (float)qmax;
+                if (r < (float)-qmax) r = (float)-qmax;
+                c = (int)r;
+            }
+            volatile float dq = (float)c * sf;
+            volatile float d = w[j] - dq;
+            volatile float ev = d / U[j * K + j];
+            e = ev;
+        }
+        put_code(codes_row_base, K, bits, n, j, c);
+        if (e != 0.0f)
+            for (k = j + 1; k < K; k++) w[k] = fmaf(-e, U[j * K + k], w[k]);
+    }
+    return status;
+}
+
+/* GPTQ over W[N, K] (fp32, overwritten with the compensated weights); codes,
+ * scales and status as rqo_quantize_g64.  U: fp32 [K, K], the upper Cholesky
+ * factor of the damped inverse Hessian; dead: nullable uint8 [K]. */
+int rqo_gptq_g64(float *W, int64_t N, int64_t K, int bits, const float *U, const uint8_t *dead,
+                 uint8_t *codes, uint16_t *scales)
+{
+    const int64_t G = K / RQO_GROUP;
+    int status = RQO_OK;
+    int64_t n;
+#pragma omp parallel for schedule(dynamic, 1) reduction(max : status)
+    for (n = 0; n < N; n++) {
+        int st = gptq_row(&W[n * K], K, bits, U, dead, codes, n, &scales[n * G]);
+        if (st > status) status = st;
+    }
+    if (status != RQO_OK) {
+        int64_t i, total = N * G;
+        for (i = 0; i < total; i++) if (scales[i] == 0x7E00u) return RQO_ERR_NONFINITE;
+    }
+    return status;
+}

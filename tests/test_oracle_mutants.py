@@ -16,6 +16,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_ex2 as ex2
+from tests import test_oracle_gptq as gptq
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "rqo.c")
@@ -56,6 +57,16 @@ MUTANTS = {
     "ex2_abs_error": ("volatile float q = d * d;", "volatile float q = fabsf(d);"),
     # E[x^2] search: every group weighted by the first group's channels
     "ex2_channel_index": ("&e2[g * RQO_GROUP]", "&e2[0]"),
+    # GPTQ: the rounding error is not spread (RTN)
+    "gptq_no_spread": ("w[k] = fmaf(-e, U[j * K + k], w[k]);", "w[k] = w[k];"),
+    # GPTQ: the error spread along a column of U instead of its row
+    "gptq_u_transposed": ("w[k] = fmaf(-e, U[j * K + k], w[k]);", "w[k] = fmaf(-e, U[k * K + j], w[k]);"),
+    # GPTQ: the error is not divided by the diagonal of U
+    "gptq_no_diag_divide": ("volatile float ev = d / U[j * K + j];", "volatile float ev = d;"),
+    # GPTQ: the error spread with the wrong sign
+    "gptq_sign": ("w[k] = fmaf(-e, U[j * K + k], w[k]);", "w[k] = fmaf(e, U[j * K + k], w[k]);"),
+    # GPTQ: every group keeps the first group's scale
+    "gptq_scale_once": ("if (j % RQO_GROUP == 0) {\n            /* the group's scale", "if (j == 0) {\n            /* the group's scale"),
 }
 
 PIN_TESTS = [
@@ -74,6 +85,10 @@ PIN_TESTS = [
     lambda: ex2.test_single_factor_one_is_rtn(4),
     lambda: ex2.test_matches_numpy_restatement(4, (3, 192)),
     lambda: ex2.test_matches_numpy_restatement(8, (2, 256)),
+    lambda: gptq.test_diagonal_hessian_is_rtn(4),
+    lambda: gptq.test_matches_sequential_obs(4),
+    gptq.test_hand_worked_rows,
+    lambda: gptq.test_layer_error_below_rtn(8),
 ]
 
 
@@ -97,7 +112,7 @@ def test_pins_catch_mutant(name):
         so = _build_mutant(name, old, new, tmp)
         lib = ctypes.CDLL(so)
         for fn in ("rqo_f32_to_f16", "rqo_f16_to_f64", "rqo_quantize_g64", "rqo_quantize_g64_ex2",
-                   "rqo_matmul", "rqo_matmul_sampled", "rqo_get_code"):
+                   "rqo_matmul", "rqo_matmul_sampled", "rqo_get_code", "rqo_gptq_g64"):
             getattr(lib, fn).argtypes = getattr(real, fn).argtypes
             getattr(lib, fn).restype = getattr(real, fn).restype
         caught = False
