@@ -390,6 +390,38 @@ def bench_quantizer(hbm_peak, reps=50):
             "frac": byts / ms / 1e6 / hbm_peak}
 
 
+def bench_gptq(reps=3):
+    """GPTQ on one 4096 x 4096 projection (int4 g64) with 512 synthetic
+    calibration tokens: device time of each step (hessian, factor, column
+    loop), median of `reps` runs.  Offline work: reported, not a headline."""
+    N = K = 4096
+    T = 512
+    g = torch.Generator(device="cuda")
+    g.manual_seed(17)
+    X = torch.randn((T, K), generator=g, device="cuda").to(torch.float16)
+    W0 = synth.weights(N, K, seed=18, device="cuda")
+    s = torch.cuda.current_stream()
+    out = {"hessian": [], "factor": [], "loop": []}
+    for _ in range(reps):
+        W = W0.clone()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(s)
+        H = rq.gptq_hessian(X)
+        ev[1].record(s)
+        U, dead = rq.gptq_factor(H)
+        ev[2].record(s)
+        rq.gptq_g64(W, 4, U, dead)
+        ev[3].record(s)
+        ev[3].synchronize()
+        for i, k in enumerate(("hessian", "factor", "loop")):
+            out[k].append(ev[i].elapsed_time(ev[i + 1]))
+        del H, U, dead, W
+    res = {k: statistics.median(v) for k, v in out.items()}
+    res.update({"shape": [N, K], "tokens": T, "bits": 4, "unit": "ms",
+                "loop_tflops": N * K * K / (res["loop"] / 1e3) / 1e12})
+    return res
+
+
 # ------------------------------------------------------- profiling case --
 
 def run_case(args):
@@ -405,6 +437,12 @@ def run_case(args):
         for _ in range(args.repeat):
             rq.quantize_g64(W, args.bits)
             torch.cuda.synchronize()
+    elif args.case == "gptq":
+        X = synth.activations(512, K, seed=8, device="cuda")
+        for _ in range(args.repeat):
+            U, dead = rq.gptq_factor(rq.gptq_hessian(X))
+            rq.gptq_g64(W.clone(), args.bits, U, dead)
+            torch.cuda.synchronize()
     elif args.case == "quantize_ex2":
         e2 = synth.activations(64, K, seed=6, device="cuda").float().pow(2).mean(0)
         factors = torch.tensor([1.0, 0.95, 0.9, 0.85, 0.8, 0.75, 0.7], device="cuda")
@@ -415,6 +453,7 @@ def run_case(args):
         w = rq.quantize_g64(W, args.bits)
         del W
         x = synth.activations(args.M, K, seed=7, device="cuda")
+        rq.set_decode_kernel(args.decode_kernel)
         for _ in range(args.repeat):
             if args.case == "gemv":
                 rq.gemv_wq(x, w[0], w[1], N, args.bits)
@@ -437,12 +476,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", type=int, default=5, choices=[2, 3, 5])
     ap.add_argument("--case", default=None,
-                    choices=["gemv", "rkv", "gemm", "quantize", "quantize_ex2"],
+                    choices=["gemv", "rkv", "gemm", "quantize", "quantize_ex2", "gptq"],
                     help="one call per repeat of a single product or quantizer (profiling target)")
     ap.add_argument("--shape", default="4096x4096", help="NxK of --case")
     ap.add_argument("--M", type=int, default=1, help="batch of --case")
     ap.add_argument("--bits", type=int, default=4, choices=[4, 8], help="bits of --case")
     ap.add_argument("--repeat", type=int, default=2, help="calls of --case")
+    ap.add_argument("--decode-kernel", default="auto", choices=["auto", "rowtile", "cluster", "rowblock"],
+                    help="decode kernel of --case gemv/rkv")
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--skip-extras", action="store_true",
                     help="decode only (no prefill/quantizer/cpu baseline/e2e)")
@@ -549,10 +590,11 @@ def main():
                "how": "pinned host x -> device, replay of the captured rq_* calls, "
                       "every output -> pinned host, per step"}
 
-    prefill = quant = cpu = None
+    prefill = quant = cpu = gptq = None
     if not args.skip_extras:
         prefill = bench_prefill(hbm_peak, tf_peak)
         quant = bench_quantizer(hbm_peak)
+        gptq = bench_gptq()
         if rank == 0 and world == 1:
             g, cores, sample = cpu_oracle_rate(wl)
             cpu = {"value": g, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample}
@@ -586,6 +628,7 @@ def main():
             "prefill": prefill,
             "prefill_peak": {"tflops": tf_peak, "kind": peak_kind + " bf16 (fp16 same nominal rate)"},
             "quantizer": quant,
+            "gptq": gptq,
         }
         print(json.dumps(line), flush=True)
 

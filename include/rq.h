@@ -122,6 +122,56 @@ rq_status rq_quantize_g64_ex2(const float *W, int64_t N, int64_t K, int bits, co
                               int32_t *chosen, int *dev_status, rq_stream_t stream);
 
 /*
+ * GPTQ on the same group-64 grid -- the "GPTQ-calibrated, symmetric, group
+ * 64" int4 of the "Hakureirm/rwkv7-sglang-w4gptq-1.5b" model card (opening
+ * summary), run "on the preset's grid without changing the format or the
+ * kernels" ("rwkv-quant: uma matriz em bf16 elimina 39% das perdas na
+ * quantização do RWKV-7 2.9B", "Vazamento de calibração e medições
+ * honestas").  The method is the published GPTQ (Frantar et al.,
+ * arXiv:2210.17323): columns of W are quantized in order, each column's
+ * rounding error spread over the later columns through U, the upper Cholesky
+ * factor of the damped inverse Hessian of the layer input.  Three calls, on
+ * one stream in this order; the stored codes and scales are the format of
+ * rq_quantize_g64 and feed the same products.
+ *
+ * rq_gptq_hessian -- H = (2/T) X^T X in fp64.  X: fp16 [T, K] device (the
+ * calibration inputs of the layer, one row per token), 16-byte aligned.
+ * H: fp64 [K, K] device, fully overwritten.  64 <= K <= 65536, K % 64 == 0,
+ * 1 <= T < 2^31, else RQ_ERR_SHAPE.
+ *
+ * rq_gptq_factor -- from H (consumed: overwritten): every input j whose
+ * H[j][j] is 0 is dead (dead[j] = 1, H[j][j] = 1); H += damp * mean(diag H) * I;
+ * U = the upper Cholesky factor of H^-1 (H^-1 = U^T U), fp64 arithmetic, U
+ * written as fp32 [K, K] (zeros below the diagonal).  dead: uint8 [K] device.
+ * work: fp64, K*K + K values, device, 16-byte aligned.  damp: the relative
+ * damping (GPTQ's usual 0.01), 0 <= damp < 1e6 else RQ_ERR_RANGE.  The
+ * factorisation is right-looking with one kernel launch per column (K
+ * launches): offline cost, about K^3 / 3 fp64 operations.
+ *
+ * rq_gptq_g64 -- the column loop.  W: fp32 [N, K] device, overwritten with the
+ * error-compensated weights each column was quantized from (dead inputs'
+ * columns start at 0).  U, dead: from rq_gptq_factor (dead may be NULL: no
+ * dead inputs).  codes, scales: outputs in the layout of rq_quantize_g64.
+ * work: fp32 [N, 128] device.  Per row, for j = 0 .. K-1: at a group's first
+ * column its scale s16 = fp16_rn(fp32 amax / qmax) is found from the group's
+ * CURRENT weights; code c_j = clamp(rint(w_j / s16), +-qmax) (IEEE fp32
+ * division, ties to even); e_j = (w_j - c_j s16) / U[j][j]; w_k =
+ * fmaf(-e_j, U[j][k], w_k) for every k > j in ascending j.  Every operation
+ * is one fp32 rounding in that order, so the result is reproducible bit for
+ * bit.  A group with a non-finite weight gets scale 0x7E00 and codes 0, one
+ * whose scale overflows fp16 gets 0x7C00 and codes 0; neither spreads error;
+ * dev_status (optional, caller-zeroed device int) receives RQ_ERR_NONFINITE /
+ * RQ_ERR_RANGE as for rq_quantize_g64.  K <= 65536.
+ */
+rq_status rq_gptq_hessian(const uint16_t *X, int64_t T, int64_t K, double *H,
+                          rq_stream_t stream);
+rq_status rq_gptq_factor(double *H, int64_t K, double damp, float *U, uint8_t *dead,
+                         double *work, rq_stream_t stream);
+rq_status rq_gptq_g64(float *W, int64_t N, int64_t K, int bits, const float *U,
+                      const uint8_t *dead, void *codes, uint16_t *scales, float *work,
+                      int *dev_status, rq_stream_t stream);
+
+/*
  * rq_gemv_wq -- decode product y[M, N] = x[M, K] * w_hat^T for 1 <= M <= 32.
  * Streams each code and scale byte from HBM once.
  * x: fp16 [M, K] device.  codes/scales: as produced by rq_quantize_g64.
@@ -156,6 +206,46 @@ rq_status rq_rkv_fused(const uint16_t *x, int64_t M, int64_t K, int64_t N, int b
                        const void *codes_k, const uint16_t *scales_k,
                        const void *codes_v, const uint16_t *scales_v,
                        float *y_r, float *y_k, float *y_v, rq_stream_t stream);
+
+/*
+ * rq_gemv_wq_ex -- the decode product with a choice of output type and a
+ * fused epilogue ("fp16-output / fused-epilogue" decode variants).  Same
+ * product as rq_gemv_wq (1 <= M <= 32), on the row-block decode kernel, then,
+ * per output, before it is stored:
+ *   epilogue RQ_EPI_NONE     y
+ *   epilogue RQ_EPI_RELU_SQ  max(y, 0)^2 in fp32 -- the squared-ReLU that
+ *            follows the channel-mix key projection of an RWKV-7 block, so the
+ *            key output can feed the value projection directly;
+ *   out_dtype RQ_OUT_F32: y fp32 [M, N]; RQ_OUT_F16: y fp16 [M, N] (fp16 bit
+ *            patterns, round to nearest even; values beyond fp16 become inf).
+ * Other values of out_dtype / epilogue: RQ_ERR_RANGE.  y: device, 16-byte
+ * aligned, fully overwritten.  Needs no workspace.
+ */
+#define RQ_OUT_F32 0
+#define RQ_OUT_F16 1
+#define RQ_EPI_NONE 0
+#define RQ_EPI_RELU_SQ 1
+rq_status rq_gemv_wq_ex(const uint16_t *x, int64_t M, int64_t K, const void *codes,
+                        const uint16_t *scales, int64_t N, int bits, void *y, int out_dtype,
+                        int epilogue, rq_stream_t stream);
+
+/*
+ * rq_rkv_fused3 -- the receptance/key/value projections in ONE launch, each
+ * with its OWN input (RWKV-7 mixes a token-shifted copy of the block input
+ * into each of r, k and v with its own coefficients, so the three inputs
+ * differ): yR = xR * w_hat_R^T, yK = xK * w_hat_K^T, yV = xV * w_hat_V^T.
+ * The "RWKV-7 Quantization Toolkit" ("Key Design") runs R/K/V in a single
+ * launch; rq_rkv_fused is the shared-input form.  x_*: fp16 [M, K] device,
+ * 16-byte aligned.  Outputs fp32 or (out_dtype RQ_OUT_F16) fp16 [M, N].
+ * Same rules otherwise as rq_rkv_fused (1 <= M <= 32); row-block kernel, no
+ * workspace.
+ */
+rq_status rq_rkv_fused3(const uint16_t *x_r, const uint16_t *x_k, const uint16_t *x_v,
+                        int64_t M, int64_t K, int64_t N, int bits,
+                        const void *codes_r, const uint16_t *scales_r,
+                        const void *codes_k, const uint16_t *scales_k,
+                        const void *codes_v, const uint16_t *scales_v,
+                        void *y_r, void *y_k, void *y_v, int out_dtype, rq_stream_t stream);
 
 /*
  * rq_gemm_wq -- prefill product y[M, N] = x[M, K] * w_hat^T on the tcgen05
@@ -222,21 +312,24 @@ rq_status rq_set_pdl(int enable);
  *                          tiles summed through a workspace;
  *   RQ_DECODE_CLUSTER  (2) K split over the CTAs of a thread-block cluster,
  *                          each CTA's x held in shared memory, partial sums
- *                          added through distributed shared memory.
+ *                          added through distributed shared memory;
+ *   RQ_DECODE_ROWBLOCK (3) blocks of rows over the full K range, each output
+ *                          finished inside one CTA; needs no workspace.
  * Any other value is rejected with RQ_ERR_RANGE.  Not thread-safe.
  */
 #define RQ_DECODE_AUTO 0
 #define RQ_DECODE_ROWTILE 1
 #define RQ_DECODE_CLUSTER 2
+#define RQ_DECODE_ROWBLOCK 3
 rq_status rq_set_decode_kernel(int kernel);
 
 /*
- * rq_decode_kernel_for -- which decode kernel (RQ_DECODE_ROWTILE or
- * RQ_DECODE_CLUSTER) a decode product of this shape would run on under the
+ * rq_decode_kernel_for -- which decode kernel (RQ_DECODE_ROWTILE,
+ * RQ_DECODE_CLUSTER or RQ_DECODE_ROWBLOCK) a decode product of this shape would run on under the
  * current rq_set_decode_kernel selection; nmat is 1 (rq_gemv_wq) or 3
  * (rq_rkv_fused).  Host-only: launches nothing and needs no GPU.  The same
  * argument checks as the products (RQ_ERR_BITS, RQ_ERR_SHAPE); kernel NULL
- * gives RQ_ERR_NULL; a forced cluster kernel that cannot hold the shape gives
+ * gives RQ_ERR_NULL; a forced kernel that cannot take the shape gives
  * RQ_ERR_SHAPE, as the product would.
  */
 rq_status rq_decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat,

@@ -226,3 +226,19 @@ def gptq_g64(W: np.ndarray, bits: int, U: np.ndarray, dead=None):
     st = _load().rqo_gptq_g64(_ptr(Wc), N, K, bits, _ptr(U32), _ptr(d) if d is not None else None,
                               _ptr(codes), _ptr(scales))
     return codes, scales, Wc, int(st)
+
+
+# ------------------------------------------------ decode epilogues (fused) --
+# The squared ReLU that follows the channel-mix key projection of an RWKV-7
+# block (k = relu(key(x))^2; the value projection then reads k).
+
+def relu_sq(y: np.ndarray) -> np.ndarray:
+    """max(y, 0)^2 in fp64."""
+    r = np.maximum(np.asarray(y, dtype=np.float64), 0.0)
+    return r * r
+
+
+def relu_sq_budget(y_ref: np.ndarray, delta: np.ndarray) -> np.ndarray:
+    """Error budget of relu(a)^2 when |a - y_ref| <= delta:
+    |relu(a)^2 - relu(b)^2| <= |a - b| (relu(a) + relu(b)) <= delta (2 relu(b) + delta)."""
+    return delta * (2.0 * np.maximum(y_ref, 0.0) + delta)

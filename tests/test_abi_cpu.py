@@ -88,8 +88,8 @@ def test_control_calls(L):
     assert L.rq_set_wait_limit_ns(0) == rq.ERR_RANGE
     assert L.rq_set_wait_limit_ns(10**9) == rq.OK
     assert L.rq_set_pdl(0) == rq.OK
-    # decode kernel selection: 0 automatic, 1 row tiles, 2 cluster split-K
-    for bad in (-1, 3, 1 << 20):
+    # decode kernel selection: 0 automatic, 1 row tiles, 2 cluster split-K, 3 row blocks
+    for bad in (-1, 4, 1 << 20):
         assert L.rq_set_decode_kernel(bad) == rq.ERR_RANGE
     for kind, code in rq.DECODE_KERNELS.items():
         assert L.rq_set_decode_kernel(code) == rq.OK
@@ -128,6 +128,10 @@ def test_decode_kernel_choice(L):
             for M in (1, 16, 32):
                 assert rq.decode_kernel_for(M, D, D, 8, 1) == kind
     assert rq.decode_kernel_for(1, D, D, 4, 1) == "rowtile"
+    # a forced row-block selection takes every decode batch size
+    with rq.decode_kernel("rowblock"):
+        for M in (1, 9, 16, 17, 32):
+            assert rq.decode_kernel_for(M, D, D, 4, 3) == "rowblock"
     # argument checks
     out = ctypes.c_int()
     assert L.rq_decode_kernel_for(0, D, D, 4, 1, ctypes.byref(out)) == rq.ERR_SHAPE
@@ -160,3 +164,40 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(rq, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         rq.lib()
+
+
+def test_decode_variant_argument_errors(L):
+    """rq_gemv_wq_ex and rq_rkv_fused3 reject bad arguments before any launch."""
+    p = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    g = L.rq_gemv_wq_ex
+    assert g(p, 1, 128, p, p, 64, 4, p, 2, 0, None) == rq.ERR_RANGE        # out dtype
+    assert g(p, 1, 128, p, p, 64, 4, p, 0, 7, None) == rq.ERR_RANGE        # epilogue
+    assert g(p, 33, 128, p, p, 64, 4, p, 0, 0, None) == rq.ERR_SHAPE       # M > 32
+    assert g(p, 1, 100, p, p, 64, 4, p, 0, 0, None) == rq.ERR_SHAPE
+    assert g(p, 1, 128, p, p, 64, 5, p, 0, 0, None) == rq.ERR_BITS
+    assert g(None, 1, 128, p, p, 64, 4, p, 0, 0, None) == rq.ERR_NULL
+    assert g(p, 1, 128, p, p, 64, 4, None, 0, 0, None) == rq.ERR_NULL
+    assert g(p, 1, 128, p, p, 64, 4, odd, 1, 1, None) == rq.ERR_ALIGN
+    f = L.rq_rkv_fused3
+    assert f(p, p, p, 1, 128, 64, 4, p, p, p, p, p, p, p, p, p, 3, None) == rq.ERR_RANGE
+    assert f(p, None, p, 1, 128, 64, 4, p, p, p, p, p, p, p, p, p, 0, None) == rq.ERR_NULL
+    assert f(p, p, odd, 1, 128, 64, 4, p, p, p, p, p, p, p, p, p, 0, None) == rq.ERR_ALIGN
+    assert f(p, p, p, 0, 128, 64, 4, p, p, p, p, p, p, p, p, p, 0, None) == rq.ERR_SHAPE
+    assert f(p, p, p, 1, 128, 64, 4, p, p, p, p, p, None, p, p, p, 0, None) == rq.ERR_NULL
+
+
+def test_gptq_argument_errors(L):
+    p = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert L.rq_gptq_hessian(p, 10, 100, p, None) == rq.ERR_SHAPE
+    assert L.rq_gptq_hessian(p, 0, 128, p, None) == rq.ERR_SHAPE
+    assert L.rq_gptq_hessian(None, 10, 128, p, None) == rq.ERR_NULL
+    assert L.rq_gptq_hessian(odd, 10, 128, p, None) == rq.ERR_ALIGN
+    assert L.rq_gptq_factor(p, 128, -1.0, p, p, p, None) == rq.ERR_RANGE
+    assert L.rq_gptq_factor(p, 100, 0.01, p, p, p, None) == rq.ERR_SHAPE
+    assert L.rq_gptq_factor(p, 128, 0.01, p, None, p, None) == rq.ERR_NULL
+    assert L.rq_gptq_g64(p, 4, 128, 5, p, None, p, p, p, None, None) == rq.ERR_BITS
+    assert L.rq_gptq_g64(p, 4, 100, 4, p, None, p, p, p, None, None) == rq.ERR_SHAPE
+    assert L.rq_gptq_g64(p, 4, 128, 4, None, None, p, p, p, None, None) == rq.ERR_NULL
+    assert L.rq_gptq_g64(p, 4, 128, 4, p, None, p, p, odd, None, None) == rq.ERR_ALIGN

@@ -105,7 +105,12 @@ def product_case(N, K, bits, M, seed, massive=None):
     return x, codes, scales
 
 
-DECODE_KERNELS = ["rowtile", "cluster"]
+DECODE_KERNELS = ["rowtile", "cluster", "rowblock"]
+
+
+def takes(kernel, M):
+    """Whether a decode kernel takes batch M (all take 1 <= M <= 32)."""
+    return 1 <= M <= 32
 
 
 @pytest.mark.parametrize("kernel", DECODE_KERNELS)
@@ -113,6 +118,8 @@ DECODE_KERNELS = ["rowtile", "cluster"]
 @pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16, 17, 31, 32])
 @pytest.mark.parametrize("N,K", [(300, 640), (1, 64), (129, 128), (256, 2048), (390, 1792), (256, 16384)])
 def test_gemv_parity(kernel, bits, M, N, K):
+    if not takes(kernel, M):
+        pytest.skip("the row-block kernel takes M <= 16")
     x, codes, scales = product_case(N, K, bits, M, seed=1000 + M + N + K)
     cd, sd = upload(codes, scales)
     with rq.decode_kernel(kernel):
@@ -127,6 +134,8 @@ def test_gemv_parity(kernel, bits, M, N, K):
 @pytest.mark.parametrize("M", [1, 8, 13, 32])
 @pytest.mark.parametrize("N,K", [(200, 512), (256, 2048)])
 def test_rkv_fused_parity(kernel, bits, M, N, K):
+    if not takes(kernel, M):
+        pytest.skip("the row-block kernel takes M <= 16")
     cases = [product_case(N, K, bits, M, seed=2000 + i) for i in range(3)]
     x = cases[0][0]
     ws = [upload(c[1], c[2]) for c in cases]
@@ -247,6 +256,8 @@ def test_decode_workload_shapes(kernel, wl):
         codes, scales = quantize_checked(W, w.bits, seed=pi)
         del W
         for M in w.Ms:
+            if not takes(kernel, M):
+                continue
             x = synth.activations(M, pj.K, seed=synth.seed_for(wl, 0, pi) + M, device="cuda",
                                   massive_channel=w.massive_channel)
             with rq.decode_kernel(kernel):
@@ -266,6 +277,8 @@ def test_decode_workload_rkv_fused(kernel):
             ws.append(rq.quantize_g64(W, w.bits))
             del W
         for M in (w.Ms[0], w.Ms[-1]):
+            if not takes(kernel, M):
+                M = 16
             x = synth.activations(M, D, seed=M, device="cuda", massive_channel=w.massive_channel)
             with rq.decode_kernel(kernel):
                 ys = rq.rkv_fused(x, ws[0], ws[1], ws[2], D, w.bits)
@@ -306,7 +319,8 @@ def test_bounded_wait_times_out_cleanly():
     assert rq.read_device_status() == rq.OK
 
 
-@pytest.mark.parametrize("kernel,M", [("rowtile", 4), ("cluster", 4), ("cluster", 24)])
+@pytest.mark.parametrize("kernel,M", [("rowtile", 4), ("cluster", 4), ("cluster", 24),
+                                      ("rowblock", 4), ("rowblock", 13)])
 def test_pdl_chain_matches(kernel, M):
     """With programmatic dependent launch on, a chain of dependent products
     (each reading the previous output as its input) still matches."""
@@ -338,16 +352,20 @@ def test_pdl_chain_matches(kernel, M):
 
 # ------------------------------------------------------------ repeatability ---
 
-@pytest.mark.parametrize("path", ["gemv", "gemv-cluster", "gemv-cluster-m32", "gemm"])
+@pytest.mark.parametrize("path", ["gemv", "gemv-cluster", "gemv-cluster-m32", "gemv-rowblock",
+                                  "gemv-rowblock-m16", "gemm"])
 def test_repeat_runs_bit_identical(path):
-    """Both kernels sum in a fixed order, so repeated runs must agree bit for
+    """Every kernel sums in a fixed order, so repeated runs must agree bit for
     bit; a pipeline race (a stage read before or after its data) shows up here
     even when it stays within tolerance."""
-    kernel = "cluster" if path.startswith("gemv-cluster") else "rowtile"
+    kernel = ("cluster" if path.startswith("gemv-cluster") else
+              "rowblock" if path.startswith("gemv-rowblock") else "rowtile")
     if path == "gemm":
         N, K, M, bits = 1024, 8192, 512, 4
     elif path == "gemv-cluster-m32":
         N, K, M, bits = 2048, 8192, 32, 4
+    elif path == "gemv-rowblock-m16":
+        N, K, M, bits = 16384, 4096, 16, 4
     else:
         N, K, M, bits = 4096, 4096, 5, 4
     W = synth.weights(N, K, seed=31, device="cuda")

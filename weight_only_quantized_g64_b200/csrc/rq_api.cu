@@ -43,6 +43,8 @@ int decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat) {
     const bool fits = gemv_cluster_fits(M, K, bits);
     if (g_decode_kernel == RQ_DECODE_CLUSTER) return fits ? RQ_DECODE_CLUSTER : -1;
     if (g_decode_kernel == RQ_DECODE_ROWTILE) return RQ_DECODE_ROWTILE;
+    if (g_decode_kernel == RQ_DECODE_ROWBLOCK)
+        return gemv_rowblock_fits(M, K, N, bits, nmat) ? RQ_DECODE_ROWBLOCK : -1;
     // measured on B200 (graph-replayed chains, int4): the cluster kernel is
     // ahead for M > 16 on every projection shape, and for M 9..16 on tall
     // ones (>= 6144 rows per launch, K <= 4096); the row-tile kernel
@@ -208,8 +210,10 @@ static rq_status launch_decode(const uint16_t* x, int64_t M, int64_t K, int64_t 
                                const WOperand* w, int nmat, cudaStream_t s) {
     const int which = decode_kernel_for(M, K, N, bits, nmat);
     if (which < 0) return RQ_ERR_SHAPE;
-    const cudaError_t e = which == RQ_DECODE_CLUSTER ? launch_gemv_cluster(x, M, K, N, bits, w, nmat, s)
-                                                     : launch_gemv_product(x, M, K, N, bits, w, nmat, s);
+    const cudaError_t e =
+        which == RQ_DECODE_CLUSTER    ? launch_gemv_cluster(x, M, K, N, bits, w, nmat, s)
+        : which == RQ_DECODE_ROWBLOCK ? launch_gemv_rowblock(x, M, K, N, bits, w, nmat, s)
+                                      : launch_gemv_product(x, M, K, N, bits, w, nmat, s);
     return e == cudaSuccess ? RQ_OK : cuda_fail(e);
 }
 
@@ -253,6 +257,41 @@ rq_status rq_quantize_g64_ex2(const float* W, int64_t N, int64_t K, int bits, co
     return e == cudaSuccess ? RQ_OK : cuda_fail(e);
 }
 
+rq_status rq_gptq_hessian(const uint16_t* X, int64_t T, int64_t K, double* H, rq_stream_t stream) {
+    if (K < kGroup || K % kGroup != 0 || K > (int64_t{1} << 16) || T < 1 || T > (int64_t{1} << 31))
+        return RQ_ERR_SHAPE;
+    if (X == nullptr || H == nullptr) return RQ_ERR_NULL;
+    if (!aligned16(X) || !aligned16(H)) return RQ_ERR_ALIGN;
+    const cudaError_t e = launch_gptq_hessian(X, T, K, H, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+rq_status rq_gptq_factor(double* H, int64_t K, double damp, float* U, uint8_t* dead, double* work,
+                         rq_stream_t stream) {
+    if (K < kGroup || K % kGroup != 0 || K > (int64_t{1} << 16)) return RQ_ERR_SHAPE;
+    if (!(damp >= 0.0) || !(damp < 1e6)) return RQ_ERR_RANGE;
+    if (H == nullptr || U == nullptr || dead == nullptr || work == nullptr) return RQ_ERR_NULL;
+    if (!aligned16(H) || !aligned16(U) || !aligned16(work)) return RQ_ERR_ALIGN;
+    const cudaError_t e = launch_gptq_factor(H, K, damp, U, dead, work,
+                                             reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+rq_status rq_gptq_g64(float* W, int64_t N, int64_t K, int bits, const float* U, const uint8_t* dead,
+                      void* codes, uint16_t* scales, float* work, int* dev_status, rq_stream_t stream) {
+    rq_status st = check_weight_shape(N, K, bits);
+    if (st != RQ_OK) return st;
+    if (K > (int64_t{1} << 16)) return RQ_ERR_SHAPE;
+    if (W == nullptr || U == nullptr || codes == nullptr || scales == nullptr || work == nullptr)
+        return RQ_ERR_NULL;
+    if (!aligned16(W) || !aligned16(U) || !aligned16(codes) || !aligned16(scales) || !aligned16(work))
+        return RQ_ERR_ALIGN;
+    if (dev_status != nullptr && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return RQ_ERR_ALIGN;
+    const cudaError_t e = launch_gptq_quantize(W, N, K, bits, U, dead, codes, scales, work, dev_status,
+                                               reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
 rq_status rq_gemv_wq(const uint16_t* x, int64_t M, int64_t K, const void* codes,
                      const uint16_t* scales, int64_t N, int bits, float* y, rq_stream_t stream) {
     rq_status st = check_product(x, M, K, N, bits, RQ_MAX_DECODE_M);
@@ -275,6 +314,45 @@ rq_status rq_rkv_fused(const uint16_t* x, int64_t M, int64_t K, int64_t N, int b
     return launch_decode(x, M, K, N, bits, w, 3, reinterpret_cast<cudaStream_t>(stream));
 }
 
+rq_status rq_gemv_wq_ex(const uint16_t* x, int64_t M, int64_t K, const void* codes,
+                        const uint16_t* scales, int64_t N, int bits, void* y, int out_dtype,
+                        int epilogue, rq_stream_t stream) {
+    rq_status st = check_product(x, M, K, N, bits, RQ_MAX_DECODE_M);
+    if (st != RQ_OK) return st;
+    if (out_dtype != RQ_OUT_F32 && out_dtype != RQ_OUT_F16) return RQ_ERR_RANGE;
+    if (epilogue != RQ_EPI_NONE && epilogue != RQ_EPI_RELU_SQ) return RQ_ERR_RANGE;
+    if ((st = check_operand(codes, scales, static_cast<const float*>(y))) != RQ_OK) return st;
+    if (!gemv_rowblock_fits(M, K, N, bits, 1)) return RQ_ERR_SHAPE;
+    WOperand w = {codes, scales, static_cast<float*>(y)};
+    const uint16_t* xs[1] = {x};
+    const cudaError_t e = launch_gemv_rowblock_ex(xs, 1, M, K, N, bits, &w, 1, out_dtype == RQ_OUT_F16,
+                                                  epilogue, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+rq_status rq_rkv_fused3(const uint16_t* x_r, const uint16_t* x_k, const uint16_t* x_v, int64_t M,
+                        int64_t K, int64_t N, int bits, const void* codes_r, const uint16_t* scales_r,
+                        const void* codes_k, const uint16_t* scales_k, const void* codes_v,
+                        const uint16_t* scales_v, void* y_r, void* y_k, void* y_v, int out_dtype,
+                        rq_stream_t stream) {
+    rq_status st = check_product(x_r, M, K, N, bits, RQ_MAX_DECODE_M);
+    if (st != RQ_OK) return st;
+    if (x_k == nullptr || x_v == nullptr) return RQ_ERR_NULL;
+    if (!aligned16(x_k) || !aligned16(x_v)) return RQ_ERR_ALIGN;
+    if (out_dtype != RQ_OUT_F32 && out_dtype != RQ_OUT_F16) return RQ_ERR_RANGE;
+    if ((st = check_operand(codes_r, scales_r, static_cast<const float*>(y_r))) != RQ_OK) return st;
+    if ((st = check_operand(codes_k, scales_k, static_cast<const float*>(y_k))) != RQ_OK) return st;
+    if ((st = check_operand(codes_v, scales_v, static_cast<const float*>(y_v))) != RQ_OK) return st;
+    if (!gemv_rowblock_fits(M, K, N, bits, 3)) return RQ_ERR_SHAPE;
+    WOperand w[3] = {{codes_r, scales_r, static_cast<float*>(y_r)},
+                     {codes_k, scales_k, static_cast<float*>(y_k)},
+                     {codes_v, scales_v, static_cast<float*>(y_v)}};
+    const uint16_t* xs[3] = {x_r, x_k, x_v};
+    const cudaError_t e = launch_gemv_rowblock_ex(xs, 3, M, K, N, bits, w, 3, out_dtype == RQ_OUT_F16,
+                                                  RQ_EPI_NONE, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
 rq_status rq_gemm_wq(const uint16_t* x, int64_t M, int64_t K, const void* codes,
                      const uint16_t* scales, int64_t N, int bits, float* y, rq_stream_t stream) {
     rq_status st = check_product(x, M, K, N, bits, (int64_t{1} << 31) - 1);
@@ -292,7 +370,8 @@ rq_status rq_set_pdl(int enable) {
 }
 
 rq_status rq_set_decode_kernel(int kernel) {
-    if (kernel != RQ_DECODE_AUTO && kernel != RQ_DECODE_ROWTILE && kernel != RQ_DECODE_CLUSTER)
+    if (kernel != RQ_DECODE_AUTO && kernel != RQ_DECODE_ROWTILE && kernel != RQ_DECODE_CLUSTER &&
+        kernel != RQ_DECODE_ROWBLOCK)
         return RQ_ERR_RANGE;
     g_decode_kernel = kernel;
     return RQ_OK;

@@ -1,0 +1,705 @@
+// rq_gemv_rb.cu -- decode product (1 <= M <= 32) on group-64 quantized
+// weights, row blocks over full K: the row-block decode kernel.
+//
+//   y[m, n] = sum_g s16[n, g] * sum_{k in g} x[m, k] * code[n, k]
+//
+// The "Hakureirm/rwkv7-sglang-w4gptq-1.5b" model card (opening summary)
+// credits its decode speed-up to a hand-written int4 GEMV / small-M kernel
+// family streaming the g64 codes; the "RWKV-7 Quantization Toolkit"
+// (rwkv-quant-nv 1.2.1), "Key Design", keeps weights quantized on the path and
+// runs R/K/V in one launch.  This is the B200 form of that decode step.
+//
+// Work decomposition.  The rows of each matrix are cut into 16-row m-tiles
+// and the m-tiles into blocks of TC consecutive m-tiles (TC = the m-tiles
+// per SM, rounded up); a CTA owns whole blocks over the FULL K range, so
+// every output is finished inside one CTA: no partial sums leave the SM, no
+// workspace, no counters.  (An SM that owns fewer m-tiles than another simply
+// finishes early; one CTA can pull well above its share of HBM bandwidth, so
+// the busiest SMs set the pace only when their share exceeds what one SM can
+// stream.)  Fused R/K/V: the three matrices' blocks are concatenated; a block
+// never straddles two matrices.
+//
+// Data path.  A ring of slots in shared memory; a slot holds, for the
+// block's rows, S consecutive 128-byte code stages (one 3-D TMA box
+// {128 B, 16*TC rows, S stages}, 128-byte swizzled), their fp16 scales (one
+// 2-D box) and the x of their groups (one 3-D box {64 k, M tokens, groups}).
+// Codes and scales of the first slots are requested by thread 0 before the
+// kernel waits on the previous grid (they never depend on it); x after.  The
+// last warp to finish with a slot refills it (an arrival counter in shared
+// memory), so no warp waits to refill.  The 8 warps, all computing, split a
+// slot's group columns (warp w takes columns w, w+8, ...) and
+// each takes every m-tile of the block for its columns, so an x fragment is
+// loaded once per warp and column and used TC times.  At the end of a block
+// the warps' partial sums meet in shared memory (the ring, reused) and are
+// added in warp order, so the result is deterministic.
+//
+// Math.  Thread (g = lane/4, t = lane%4) owns, per group of 64 k, the 16 k
+// [16t, 16t+16) of rows g and g+8 of each m-tile (a k-permutation inside the
+// group, the same on the A and B side, so the sum over k is unchanged).  Codes
+// are turned into BIASED fp16 values with one lop3 per pair (the bit placement
+// of Kim et al., arXiv:2211.10017, without the exact bias subtraction): int4
+// low nibbles become 1032 + c (exponent of [1024, 2048)), high nibbles
+// 72 + c (exponent of [64, 128), the nibble at mantissa bits 4..7); int8
+// bytes 1152 + c.  mma.sync.m16n8k16 sums x * (code + bias) in fp32, starting
+// from -sum_k bias_k x_k of the group, which one chain of MMAs with a
+// constant A operand (-bias) computes once per group and 8-token tile and
+// every m-tile reuses.  The group's scale is applied in fp32
+// (acc = fma(part, s16, acc)).  Products x * (code + bias) are exact in fp32
+// (11 x 11 significant bits), so the bias costs only the fp32 rounding of
+// sums of magnitude ~1000 |x|: about 1e-4 of the error budget
+// 2e-3 * sum |x||w_hat| per output.
+#include <cuda_fp16.h>
+
+#include <cstring>
+
+#include "rq_internal.h"
+#include "rq_ptx.cuh"
+#include "rq_gemv_unit.cuh"
+
+namespace rq {
+
+struct RbParams {
+    CUtensorMap tm_w[3];  // codes: 3-D {128 B, N rows, stages} box {128, RB, S}, or (rows not whole
+                          // stages) 2-D {row bytes, N} box {128, RB}; SWIZZLE_128B
+    CUtensorMap tm_s[3];  // scales [N, groups] fp16: box {SROW, RB} (when ssc)
+    CUtensorMap tm_x[3];  // x of each matrix as 3-D {64, M, groups}: box {64, M, J}, SWIZZLE_128B
+    const uint16_t* scales[3];
+    void* y[3];           // fp32 or (yh) fp16 [M, N]
+    int M, N, K;
+    int groups;           // K / 64
+    int stages;           // 128-byte code stages per row
+    int tc;               // m-tiles per block (TC)
+    int bpm;              // blocks per matrix
+    int nblocks;          // blocks in all matrices
+    int S;                // stages per slot
+    int J;                // group columns per slot (S * groups per stage)
+    int slots;            // slots per block: ceil(stages / S)
+    int sg;               // ring depth (slots)
+    int three_d;          // codes through the 3-D map
+    int ssc;              // scales staged by TMA
+    int srow;             // scale row length in a slot (fp16, 16-byte multiple)
+    int slot_bytes, s_off, x_off, bar_off, red_stride;
+    int nx;               // distinct inputs: 1 (shared x) or 3 (one per matrix)
+    int yh;               // y stored as fp16 (round to nearest even)
+    int epi;              // epilogue: 0 none, 1 relu(y)^2
+    int* status;
+    uint64_t timeout_ns;
+};
+
+constexpr int kRbWarps = 8;                     // warps, all computing
+constexpr int kRbThreads = kRbWarps * 32;
+constexpr int kRbMaxSG = 8;
+
+struct RbBars {
+    uint64_t full[kRbMaxSG];   // the slot holds its codes, scales and x
+    int done[kRbMaxSG];        // warps finished with the slot's current round
+    int issued_hi[kRbMaxSG];   // last slot index issued into each ring slot
+    int abort;
+};
+
+// D = A * B + C (fp16 inputs, fp32 accumulate), C and D distinct.
+__device__ __forceinline__ void mma16816_c(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                           uint32_t b1, const float (&c)[4]) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%11,%12,%13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]),
+          "f"(c[2]), "f"(c[3]));
+}
+
+// int4, permuted pair order, biased: one code word (positions 0..7 of a row,
+// position 2i in the low nibble of byte i) -> pairs (p0,p4) and (p2,p6) as
+// 1032 + c, pairs (p1,p5) and (p3,p7) as 72 + c.  5 instructions per 8 codes.
+__device__ __forceinline__ void i4_word_biased(uint32_t w, uint32_t (&P)[4]) {
+    const uint32_t w8 = w >> 8;
+    P[0] = lop3_bmux(w, 0x000F000Fu, 0x64086408u);    // 0x6400 | (nibble ^ 8)       = 1032 + c
+    P[1] = lop3_bmux(w, 0x00F000F0u, 0x54805480u);    // 0x5400 | (nibble ^ 8) << 4  = 72 + c
+    P[2] = lop3_bmux(w8, 0x000F000Fu, 0x64086408u);
+    P[3] = lop3_bmux(w8, 0x00F000F0u, 0x54805480u);
+}
+
+// int8, biased: one 32-bit word (positions 0..3) -> pairs (p0,p1), (p2,p3) as
+// 1152 + c.  3 instructions per 4 codes.
+__device__ __forceinline__ void i8_word_biased(uint32_t w, uint32_t (&Q)[2]) {
+    w ^= 0x80808080u;
+    Q[0] = __byte_perm(w, 0x64646464u, 0x5140u);
+    Q[1] = __byte_perm(w, 0x64646464u, 0x5342u);
+}
+
+// Group columns of one warp (NC of them, processed together for independent
+// dependency chains): every m-tile of the block (MT of them) times the x of
+// the column's group, for NT 8-token tiles.  Per column c:
+//   cw0[c] codes of the column's stage, m-tile 0, this thread's physical row
+//          and chunk (rows 16i + prow and +8 of m-tile i are 16*128*i and
+//          8*128 further)
+//   sp[c]  scales: (row 16i + 8h + prow, this group) at sp[c][(16i + 8h) * srow]
+//   xg[c]  x of the group: token rows of 128 B (swizzled); xl[c][nt] the row
+//          of token nt*8+g
+//   grp[c] the group (for scales read from global memory when !ssc)
+// The four MMA steps of a group run as two independent 2-step chains and the
+// bias term as a third chain; the three are added before the scale, in a
+// fixed order.
+template <int BITS, int MT, int NT, int NC>
+__device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
+                                           const uint16_t* const (&sp)[NC], int srow,
+                                           const uint8_t* const (&xg)[NC], const int (&xl)[NC][NT],
+                                           int t, float (&acc)[MT][NT][4], bool ssc,
+                                           const uint16_t* gscales, int64_t grow0, int groups,
+                                           const int (&grp)[NC], int N) {
+    constexpr int CW = BITS == 4 ? 2 : 4;   // code words per row and group
+    // ---- x fragments: token nt*8+g, positions 16t .. 16t+15 of the group
+    uint32_t b[NC][NT][4][2];
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int line = xl[c][nt];
+            const uint8_t* xr = xg[c] + line * 128;
+            const int ph = line & 7;
+            const uint4 v0 = lds128(xr + (((2 * t) ^ ph) << 4));
+            const uint4 v1 = lds128(xr + (((2 * t + 1) ^ ph) << 4));
+            const uint32_t X[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                if constexpr (BITS == 4) {
+                    // step jj pairs (p0,p4),(p1,p5) or (p2,p6),(p3,p7) of word jj/2
+                    const int wb = (jj >> 1) * 4 + (jj & 1);
+                    b[c][nt][jj][0] = __byte_perm(X[wb], X[wb + 2], 0x5410);
+                    b[c][nt][jj][1] = __byte_perm(X[wb], X[wb + 2], 0x7632);
+                } else {
+                    b[c][nt][jj][0] = X[2 * jj];
+                    b[c][nt][jj][1] = X[2 * jj + 1];
+                }
+            }
+        }
+    // ---- -sum_k bias_k x_k of each column's group, per token tile (the same
+    // for every row): two 2-step chains
+    float negc[NC][NT][4];
+    {
+        uint32_t an[4];
+        if constexpr (BITS == 4) {
+            an[0] = an[1] = 0xE408E408u;   // -1032 (slots 2t, 2t+1: low-nibble pairs)
+            an[2] = an[3] = 0xD480D480u;   // -72   (slots 2t+8, 2t+9: high-nibble pairs)
+        } else {
+            an[0] = an[1] = an[2] = an[3] = 0xE480E480u;   // -1152
+        }
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float h0[4], h1[4];
+                mma16816(h0, an, b[c][nt][0][0], b[c][nt][0][1], true);
+                mma16816(h1, an, b[c][nt][2][0], b[c][nt][2][1], true);
+                mma16816(h0, an, b[c][nt][1][0], b[c][nt][1][1], false);
+                mma16816(h1, an, b[c][nt][3][0], b[c][nt][3][1], false);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) negc[c][nt][e] = h0[e] + h1[e];
+            }
+    }
+    // ---- every m-tile
+#pragma unroll
+    for (int i = 0; i < MT; ++i) {
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            uint32_t cw[2][CW];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint8_t* cp = cw0[c] + (16 * i + 8 * h) * 128;
+                if constexpr (BITS == 4) {
+                    const uint2 v = lds64(cp);
+                    cw[h][0] = v.x;
+                    cw[h][1] = v.y;
+                } else {
+                    const uint4 v = lds128(cp);
+                    cw[h][0] = v.x; cw[h][1] = v.y; cw[h][2] = v.z; cw[h][3] = v.w;
+                }
+            }
+            float sv[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint16_t s16;
+                if (ssc) {
+                    s16 = sp[c][(16 * i + 8 * h) * srow];
+                } else {
+                    const int64_t n = grow0 + 16 * i + 8 * h;
+                    s16 = (n < N && grp[c] < groups) ? __ldg(gscales + n * groups + grp[c])
+                                                     : static_cast<uint16_t>(0);
+                }
+                sv[h] = __half2float(__ushort_as_half(s16));
+            }
+            uint32_t A[4][4];   // [step][a-reg]
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if constexpr (BITS == 4) {
+                    uint32_t P0[4], P1[4];
+                    i4_word_biased(cw[h][0], P0);
+                    i4_word_biased(cw[h][1], P1);
+                    A[0][h] = P0[0]; A[0][h + 2] = P0[1];
+                    A[1][h] = P0[2]; A[1][h + 2] = P0[3];
+                    A[2][h] = P1[0]; A[2][h + 2] = P1[1];
+                    A[3][h] = P1[2]; A[3][h + 2] = P1[3];
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        uint32_t Q[2];
+                        i8_word_biased(cw[h][jj], Q);
+                        A[jj][h] = Q[0];
+                        A[jj][h + 2] = Q[1];
+                    }
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float p0[4], p1[4];
+                mma16816(p0, A[0], b[c][nt][0][0], b[c][nt][0][1], true);
+                mma16816(p1, A[2], b[c][nt][2][0], b[c][nt][2][1], true);
+                mma16816(p0, A[1], b[c][nt][1][0], b[c][nt][1][1], false);
+                mma16816(p1, A[3], b[c][nt][3][0], b[c][nt][3][1], false);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc[i][nt][e] = fmaf((p0[e] + p1[e]) + negc[c][nt][e], sv[e >> 1], acc[i][nt][e]);
+            }
+        }
+    }
+}
+
+template <int BITS, int MT, int NT>
+__global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_constant__ RbParams p) {
+    constexpr int GPS = BITS == 4 ? 4 : 2;      // groups per 128-byte stage
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* ring = smem;
+    RbBars* bars = reinterpret_cast<RbBars*>(smem + p.bar_off);
+    volatile int* abort_flag = &bars->abort;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int SG = p.sg;
+    const int RB = 16 * MT;                     // rows of a block (== 16 * p.tc)
+    const int cbytes = RB * 128 * p.S;          // code bytes of a slot
+    const uint32_t x_bytes = static_cast<uint32_t>(p.J * p.M * 128);
+    const uint32_t s_bytes = p.ssc ? static_cast<uint32_t>(RB * p.srow * 2) : 0u;
+
+    // Loads of the CTA's slot i (block blk, slot sl of the block) into ring slot r.
+    auto issue_w = [&](int r, int blk, int sl) {
+        uint8_t* dst = ring + r * p.slot_bytes;
+        const int m = blk / p.bpm;
+        const int row0 = (blk - m * p.bpm) * RB;
+        const int st0 = sl * p.S;
+        const uint64_t pol = l2_policy_evict_first();
+        mbar_arrive_expect_tx(&bars->full[r], static_cast<uint32_t>(cbytes) + s_bytes + x_bytes);
+        if (p.three_d) {
+            tma_load_3d(dst, &p.tm_w[m], &bars->full[r], 0, row0, st0, pol);
+        } else {
+            for (int s = 0; s < p.S; ++s)
+                tma_load_2d(dst + s * RB * 128, &p.tm_w[m], &bars->full[r], (st0 + s) * 128, row0, pol);
+        }
+        if (p.ssc)
+            tma_load_2d(dst + p.s_off, &p.tm_s[m], &bars->full[r], (st0 * GPS) & ~7, row0, pol);
+    };
+    auto issue_x = [&](int r, int blk, int sl) {
+        const int m = p.nx > 1 ? blk / p.bpm : 0;
+        tma_load_3d(ring + r * p.slot_bytes + p.x_off, &p.tm_x[m], &bars->full[r], 0, 0, sl * p.J,
+                    l2_policy_evict_last());
+    };
+
+    if (threadIdx.x == 0) {
+        for (int r = 0; r < SG; ++r) {
+            mbar_init(&bars->full[r], 1);
+            bars->done[r] = 0;
+            bars->issued_hi[r] = -1;
+        }
+        bars->abort = 0;
+        fence_mbar_init();
+        for (int m = 0; m < 3; ++m) {
+            if (p.y[m] == nullptr) break;
+            if (m < p.nx) tma_prefetch_desc(&p.tm_x[m]);
+            tma_prefetch_desc(&p.tm_w[m]);
+            if (p.ssc) tma_prefetch_desc(&p.tm_s[m]);
+        }
+        // codes and scales of the first block's first slots: they never
+        // depend on the previous grid, so they go out before waiting on it
+        const int n_pre = min(SG, p.slots);
+        for (int r = 0; r < n_pre; ++r) {
+            bars->issued_hi[r] = r;
+            issue_w(r, blockIdx.x, r);
+        }
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+    pdl_wait();   // x (and y) may be used by the previous kernel
+    if (threadIdx.x == 0) {
+        const int n_pre = min(SG, p.slots);
+        for (int r = 0; r < n_pre; ++r) issue_x(r, blockIdx.x, r);
+    }
+
+    const int g = lane >> 2;
+    const int t = lane & 3;
+    const int prow = phys_row<BITS>(g);
+    int gi = 0;                 // the CTA's slot index (over all its blocks)
+    bool dead = false;
+    int kb = 0;                 // blocks done by this CTA
+    for (int blk = blockIdx.x; blk < p.nblocks; blk += gridDim.x, ++kb) {
+        const int m = blk / p.bpm;
+        const int row0 = (blk - m * p.bpm) * RB;
+        if (kb > 0 && threadIdx.x == 0) {
+            // a later block: the ring was the previous block's reduction
+            // buffer, so its first slots go out only now
+            const int n_pre = min(SG, p.slots);
+            for (int q = 0; q < n_pre; ++q) {
+                const int r = (gi + q) % SG;
+                bars->issued_hi[r] = gi + q;
+                issue_w(r, blk, q);
+                issue_x(r, blk, q);
+            }
+        }
+        float acc[MT][NT][4];
+#pragma unroll
+        for (int i = 0; i < MT; ++i)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[i][nt][e] = 0.0f;
+        for (int sl = 0; sl < p.slots; ++sl, ++gi) {
+            const int r = gi % SG;
+            if (!dead && !mbar_wait(&bars->full[r], static_cast<uint32_t>(gi / SG) & 1, abort_flag,
+                                    p.timeout_ns, p.status))
+                dead = true;
+            const int grp0 = sl * p.J;                  // first group of the slot
+            int jn = p.groups - grp0;                   // group columns holding data
+            if (jn > p.J) jn = p.J;
+            if (!dead) {
+                const uint8_t* base = ring + r * p.slot_bytes;
+                // this warp's columns j = warp, warp + 8, ...: two at a time
+                auto col = [&](int j, const uint8_t*& cw0, const uint16_t*& sp, int (&xl)[NT]) {
+                    const int s = j / GPS;
+                    const int q = j - s * GPS;
+                    int coff;
+                    if constexpr (BITS == 4)
+                        coff = prow * 128 + (((2 * q + (t >> 1)) ^ (prow & 7)) << 4) + ((t & 1) << 3);
+                    else
+                        coff = prow * 128 + (((4 * q + t) ^ (prow & 7)) << 4);
+                    cw0 = base + s * RB * 128 + coff;
+                    sp = reinterpret_cast<const uint16_t*>(base + p.s_off) + prow * p.srow +
+                         ((grp0 & 7) + j);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) xl[nt] = j * p.M + min(nt * 8 + g, p.M - 1);
+                };
+                int j = warp;
+                // (pairs only for one token tile: larger M takes one column
+                // per warp and slot, and the registers go to its tiles)
+                if constexpr (NT == 1)
+                for (; j + kRbWarps < jn; j += 2 * kRbWarps) {
+                    const uint8_t* cw0[2];
+                    const uint16_t* sp[2];
+                    int xl[2][NT];
+                    col(j, cw0[0], sp[0], xl[0]);
+                    col(j + kRbWarps, cw0[1], sp[1], xl[1]);
+                    const uint8_t* xg[2] = {base + p.x_off, base + p.x_off};
+                    const int gr[2] = {grp0 + j, grp0 + j + kRbWarps};
+                    rb_columns<BITS, MT, NT, 2>(cw0, sp, p.srow, xg, xl, t, acc, p.ssc != 0,
+                                                p.scales[m], row0 + prow, p.groups, gr, p.N);
+                }
+                for (; j < jn; j += kRbWarps) {
+                    const uint8_t* cw0[1];
+                    const uint16_t* sp[1];
+                    int xl[1][NT];
+                    col(j, cw0[0], sp[0], xl[0]);
+                    const uint8_t* xg[1] = {base + p.x_off};
+                    const int gr[1] = {grp0 + j};
+                    rb_columns<BITS, MT, NT, 1>(cw0, sp, p.srow, xg, xl, t, acc, p.ssc != 0,
+                                                p.scales[m], row0 + prow, p.groups, gr, p.N);
+                }
+            }
+            // ---- release the slot; the last warp out refills it with the
+            // block's slot sl + SG (later blocks refill after their reduction)
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence_block();
+                const int prev = atomicAdd(&bars->done[r], 1);
+                if (prev == kRbWarps - 1) {
+                    __threadfence_block();
+                    bars->done[r] = 0;
+                    const int nsl = sl + SG;
+                    if (nsl < p.slots && !dead && *abort_flag == 0) {
+                        bars->issued_hi[r] = gi + SG;
+                        // order every warp's generic reads of the slot before
+                        // the asynchronous writes into it
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        issue_w(r, blk, nsl);
+                        issue_x(r, blk, nsl);
+                    }
+                }
+            }
+        }
+        // ---- the block's sums: warps deposit, then add in warp order
+        __syncthreads();   // every warp is done reading the ring
+        float* red = reinterpret_cast<float*>(ring);
+        const int RS = p.red_stride;                   // floats per (warp, token)
+        for (int nt0 = 0; nt0 < NT; ++nt0) {
+            // round nt0: tokens [8 nt0, 8 nt0 + 8)
+#pragma unroll
+            for (int i = 0; i < MT; ++i)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int tl = 2 * t + (e & 1);
+                    const int rr = 16 * i + 8 * (e >> 1) + prow;
+                    float v = 0.0f;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        if (nt == nt0) v = acc[i][nt][e];
+                    red[(warp * 8 + tl) * RS + rr] = v;
+                }
+            __syncthreads();
+            const int ntok = min(8, p.M - 8 * nt0);
+            for (int o = threadIdx.x; o < ntok * RB; o += kRbThreads) {
+                const int tl = o / RB;
+                const int rr = o - tl * RB;
+                float v = 0.0f;
+#pragma unroll
+                for (int w = 0; w < kRbWarps; ++w) v += red[(w * 8 + tl) * RS + rr];
+                if (p.epi == 1) {
+                    v = fmaxf(v, 0.0f);
+                    v = v * v;
+                }
+                const int n = row0 + rr;
+                if (n < p.N && !dead && *abort_flag == 0) {
+                    const int64_t at = static_cast<int64_t>(8 * nt0 + tl) * p.N + n;
+                    if (p.yh)
+                        static_cast<__half*>(p.y[m])[at] = __float2half_rn(v);
+                    else
+                        static_cast<float*>(p.y[m])[at] = v;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    // After a timeout some issued copies may never have been waited for:
+    // wait (bounded) for the last one of every slot before the CTA exits.
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag) {
+        int dummy_abort = 0;
+        for (int r = 0; r < SG; ++r) {
+            const int il = bars->issued_hi[r];
+            if (il >= 0)
+                mbar_wait(&bars->full[r], static_cast<uint32_t>(il / SG) & 1, &dummy_abort,
+                          p.timeout_ns, p.status);
+        }
+    }
+}
+
+// ------------------------------------------------------------- launcher --
+
+static int rb_num_sms() {
+    static int sms[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (sms[dev] == 0) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        sms[dev] = v > 0 ? v : 148;
+    }
+    return sms[dev];
+}
+
+#ifndef RQ_RB_SMEM_BUDGET
+#define RQ_RB_SMEM_BUDGET (227 * 1024)
+#endif
+constexpr int kRbMaxTC = 8;                       // m-tiles per block at most
+
+static int rb_align(int v, int a) { return (v + a - 1) / a * a; }
+
+// How a decode product of this shape is cut for the row-block kernel.
+struct RbPlan {
+    int tc, bpm, nblocks, grid, stages, S, J, slots, sg, srow;
+    int slot_bytes, s_off, x_off, bar_off, red_stride, smem;
+    bool three_d;
+};
+
+static bool rb_plan(int64_t M, int64_t K, int64_t N, int bits, int nmat, RbPlan* P) {
+    const int GPS = bits == 4 ? 4 : 2;
+    const int sms = rb_num_sms();
+    const int64_t tm = (N + 15) / 16;                 // m-tiles per matrix
+    const int64_t T = tm * nmat;
+    int64_t tc = (T + sms - 1) / sms;
+    if (tc > kRbMaxTC) tc = kRbMaxTC;
+    if (tc < 1) tc = 1;
+    P->tc = static_cast<int>(tc);
+    P->bpm = static_cast<int>((tm + tc - 1) / tc);
+    P->nblocks = P->bpm * nmat;
+    P->grid = P->nblocks < sms ? P->nblocks : sms;
+    const int RB = 16 * P->tc;
+    const int64_t row_bytes = K * bits / 8;
+    P->stages = static_cast<int>((row_bytes + 127) / 128);
+    P->three_d = row_bytes % 128 == 0;
+    // stages per slot: about 16 KB of codes, at least 16 group columns (two
+    // per warp, processed together) for M <= 8 and 8 otherwise, when the row
+    // has them, and at most 16 KB of x (32 KB for M > 16)
+    const int smin = (M <= 8 ? 16 : 8) / GPS;
+    const int64_t x_cap = M > 16 ? 32768 : 16384;
+    int S = 1;
+    while (S * 2 * RB * 128 <= 16384 && S < 16) S *= 2;
+    if (S < smin) S = smin;
+    while (S > smin && static_cast<int64_t>(S) * GPS * M * 128 > x_cap) S /= 2;
+    if (S > P->stages) S = P->stages;
+    P->S = S;
+    P->J = S * GPS;
+    P->slots = (P->stages + S - 1) / S;
+    P->srow = rb_align(P->J + 8, 8);
+    const int cbytes = RB * 128 * S;
+    P->s_off = cbytes;
+    P->x_off = rb_align(P->s_off + RB * P->srow * 2, 1024);
+    P->slot_bytes = rb_align(P->x_off + P->J * static_cast<int>(M) * 128, 1024);
+    P->red_stride = RB + 4;
+    const int red_bytes = kRbWarps * 8 * P->red_stride * 4;
+    const int per_cta = (P->nblocks + P->grid - 1) / P->grid;
+    int want = P->slots * per_cta;
+    if (want > kRbMaxSG) want = kRbMaxSG;
+    for (int sg = want; sg >= 1; --sg) {
+        const int ring = sg * P->slot_bytes > red_bytes ? sg * P->slot_bytes : rb_align(red_bytes, 1024);
+        const int bar_off = ring;
+        const int smem = 1024 + bar_off + static_cast<int>(sizeof(RbBars));
+        if (smem <= RQ_RB_SMEM_BUDGET) {
+            P->sg = sg;
+            P->bar_off = bar_off;
+            P->smem = smem;
+            return true;
+        }
+    }
+    return false;
+}
+
+bool gemv_rowblock_fits(int64_t M, int64_t K, int64_t N, int bits, int nmat) {
+    if (M < 1 || M > 32) return false;
+    RbPlan P;
+    return rb_plan(M, K, N, bits, nmat, &P);
+}
+
+template <int BITS, int MT, int NT>
+static cudaError_t rb_launch(RbParams& prm, const RbPlan& P, const uint16_t* const* xs,
+                             const void* const* codes, int nmat, cudaStream_t s) {
+    auto kern = gemv_rb_kernel<BITS, MT, NT>;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    const int RB = 16 * MT;
+    const uint64_t row_bytes = static_cast<uint64_t>(prm.K) * BITS / 8;
+    for (int i = 0; i < nmat; ++i) {
+        const bool okw =
+            P.three_d
+                ? make_tmap_3d(&prm.tm_w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, codes[i], 128,
+                               static_cast<uint64_t>(prm.N), static_cast<uint64_t>(P.stages),
+                               row_bytes, 128, 128, static_cast<uint32_t>(RB),
+                               static_cast<uint32_t>(P.S), CU_TENSOR_MAP_SWIZZLE_128B)
+                : make_tmap_2d(&prm.tm_w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, codes[i], row_bytes,
+                               static_cast<uint64_t>(prm.N), row_bytes, 128,
+                               static_cast<uint32_t>(RB), CU_TENSOR_MAP_SWIZZLE_128B);
+        if (!okw) return cudaErrorInvalidValue;
+        if (prm.ssc &&
+            !make_tmap_2d(&prm.tm_s[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, prm.scales[i],
+                          static_cast<uint64_t>(prm.groups), static_cast<uint64_t>(prm.N),
+                          static_cast<uint64_t>(prm.groups) * 2, static_cast<uint32_t>(P.srow),
+                          static_cast<uint32_t>(RB), CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    }
+    for (int i = 0; i < prm.nx; ++i)
+        if (!make_tmap_3d(&prm.tm_x[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs[i], 64,
+                          static_cast<uint64_t>(prm.M), static_cast<uint64_t>(prm.groups),
+                          static_cast<uint64_t>(prm.K) * 2, 128, 64, static_cast<uint32_t>(prm.M),
+                          static_cast<uint32_t>(P.J), CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(P.grid), 1, 1);
+    cfg.blockDim = dim3(kRbThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(P.smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attrs[1];
+    int na = 0;
+    if (pdl_enabled()) {
+        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attrs;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<const RbParams&>(prm));
+}
+
+template <int BITS, int NT>
+static cudaError_t rb_dispatch_mt(RbParams& prm, const RbPlan& P, const uint16_t* const* x,
+                                  const void* const* codes, int nmat, cudaStream_t s) {
+    switch (P.tc) {
+        case 1: return rb_launch<BITS, 1, NT>(prm, P, x, codes, nmat, s);
+        case 2: return rb_launch<BITS, 2, NT>(prm, P, x, codes, nmat, s);
+        case 3: return rb_launch<BITS, 3, NT>(prm, P, x, codes, nmat, s);
+        case 4: return rb_launch<BITS, 4, NT>(prm, P, x, codes, nmat, s);
+        case 5: return rb_launch<BITS, 5, NT>(prm, P, x, codes, nmat, s);
+        case 6: return rb_launch<BITS, 6, NT>(prm, P, x, codes, nmat, s);
+        case 7: return rb_launch<BITS, 7, NT>(prm, P, x, codes, nmat, s);
+        default: return rb_launch<BITS, 8, NT>(prm, P, x, codes, nmat, s);
+    }
+}
+
+cudaError_t launch_gemv_rowblock(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
+                                 const WOperand* w, int nmat, cudaStream_t s) {
+    const uint16_t* xs[1] = {x};
+    return launch_gemv_rowblock_ex(xs, 1, M, K, N, bits, w, nmat, false, 0, s);
+}
+
+cudaError_t launch_gemv_rowblock_ex(const uint16_t* const* xs, int nx, int64_t M, int64_t K,
+                                    int64_t N, int bits, const WOperand* w, int nmat, bool y_half,
+                                    int epilogue, cudaStream_t s) {
+    RbPlan P;
+    const uint16_t* const* x = xs;
+    if (M < 1 || M > 32 || !rb_plan(M, K, N, bits, nmat, &P)) return cudaErrorInvalidValue;
+    RbParams prm;
+    memset(&prm, 0, sizeof(prm));
+    prm.M = static_cast<int>(M);
+    prm.N = static_cast<int>(N);
+    prm.K = static_cast<int>(K);
+    prm.groups = static_cast<int>(K / kGroup);
+    prm.stages = P.stages;
+    prm.tc = P.tc;
+    prm.bpm = P.bpm;
+    prm.nblocks = P.nblocks;
+    prm.S = P.S;
+    prm.J = P.J;
+    prm.slots = P.slots;
+    prm.sg = P.sg;
+    prm.three_d = P.three_d ? 1 : 0;
+    prm.ssc = (prm.groups * 2) % 16 == 0 ? 1 : 0;
+    prm.srow = P.srow;
+    prm.slot_bytes = P.slot_bytes;
+    prm.s_off = P.s_off;
+    prm.x_off = P.x_off;
+    prm.bar_off = P.bar_off;
+    prm.red_stride = P.red_stride;
+    prm.nx = nx;
+    prm.yh = y_half ? 1 : 0;
+    prm.epi = epilogue;
+    prm.status = device_status_ptr();
+    prm.timeout_ns = wait_limit_ns();
+    const void* codes[3] = {nullptr, nullptr, nullptr};
+    for (int i = 0; i < nmat; ++i) {
+        codes[i] = w[i].codes;
+        prm.scales[i] = w[i].scales;
+        prm.y[i] = w[i].y;
+    }
+    if (bits == 4)
+        return M <= 8    ? rb_dispatch_mt<4, 1>(prm, P, x, codes, nmat, s)
+               : M <= 16 ? rb_dispatch_mt<4, 2>(prm, P, x, codes, nmat, s)
+                         : rb_dispatch_mt<4, 4>(prm, P, x, codes, nmat, s);
+    return M <= 8    ? rb_dispatch_mt<8, 1>(prm, P, x, codes, nmat, s)
+           : M <= 16 ? rb_dispatch_mt<8, 2>(prm, P, x, codes, nmat, s)
+                     : rb_dispatch_mt<8, 4>(prm, P, x, codes, nmat, s);
+}
+
+}  // namespace rq

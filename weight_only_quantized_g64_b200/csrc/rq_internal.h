@@ -48,9 +48,25 @@ cudaError_t launch_gemv_cluster(const uint16_t* x, int64_t M, int64_t K, int64_t
 // K (each CTA keeps the x of its K range on chip).
 bool gemv_cluster_fits(int64_t M, int64_t K, int bits);
 
-// The decode kernel a product of this shape runs on: RQ_DECODE_ROWTILE or
-// RQ_DECODE_CLUSTER (the selection of rq_set_decode_kernel, or the automatic
-// choice), or -1 when the selected cluster kernel cannot take the shape.
+// Decode product (M <= 16), row blocks over the full K range: every output is
+// finished inside one CTA.  Needs no workspace.
+cudaError_t launch_gemv_rowblock(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
+                                 const WOperand* w, int nmat, cudaStream_t s);
+
+// The row-block kernel with nx inputs (1 shared, or one per matrix), y as
+// fp16 when y_half (WOperand::y then points to fp16), and an epilogue
+// (0 none, 1 relu(y)^2) applied before the store.
+cudaError_t launch_gemv_rowblock_ex(const uint16_t* const* xs, int nx, int64_t M, int64_t K,
+                                    int64_t N, int bits, const WOperand* w, int nmat, bool y_half,
+                                    int epilogue, cudaStream_t s);
+
+// Whether the row-block kernel takes a product of this shape.
+bool gemv_rowblock_fits(int64_t M, int64_t K, int64_t N, int bits, int nmat);
+
+// The decode kernel a product of this shape runs on: RQ_DECODE_ROWTILE,
+// RQ_DECODE_CLUSTER or RQ_DECODE_ROWBLOCK (the selection of
+// rq_set_decode_kernel, or the automatic choice), or -1 when the selected
+// kernel cannot take the shape.
 int decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat);
 
 // Caller-provided scratch for the decode product instead of the library's
@@ -67,6 +83,16 @@ struct GemvScratch {
 cudaError_t launch_gemv_product_scratch(const uint16_t* x, int64_t M, int64_t K, int64_t N,
                                         int bits, const WOperand* w, int nmat, cudaStream_t s,
                                         const GemvScratch* scratch);
+
+// GPTQ on the group-64 grid: H = (2/T) X^T X (fp64); the damped inverse-
+// Hessian factor U (fp32 upper, H^-1 = U^T U) and the dead-input mask (work:
+// K*K + K doubles, H consumed); the column loop (W in/out, work: N*128 fp32).
+cudaError_t launch_gptq_hessian(const uint16_t* X, int64_t T, int64_t K, double* H, cudaStream_t s);
+cudaError_t launch_gptq_factor(double* H, int64_t K, double damp, float* U, uint8_t* dead,
+                               double* work, cudaStream_t s);
+cudaError_t launch_gptq_quantize(float* W, int64_t N, int64_t K, int bits, const float* U,
+                                 const uint8_t* dead, void* codes, uint16_t* scales, float* work,
+                                 int* dev_status, cudaStream_t s);
 
 // Bounded-wait self test: a kernel waits on an mbarrier nothing completes.
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s);

@@ -20,82 +20,144 @@
 
 namespace rq {
 
+// rint(w / sf) with the quotient an IEEE fp32 division (ties to even), as
+// __float2int_rn(__fdiv_rn(w, sf)), but dividing only where it can matter.
+// t = w * r with r = 1/sf rounded to nearest lies within |q| * 2^-23 (1 + 2^-25)
+// of the exact quotient q, and the rounded quotient fl(q) within |q| * 2^-24
+// of it; when t is more than |t| * 2^-21 away from every half-integer, no
+// half-integer separates t from fl(q) and both round to the same integer.
+// Otherwise (ties and near-ties, e.g. weights on the grid) the exact division
+// decides.  sf must be finite and non-zero; |t| stays far below 2^22 here, so
+// t - floor(t) is exact.
+__device__ __forceinline__ int rint_quotient(float w, float sf, float r) {
+    const float t = __fmul_rn(w, r);
+    const float f = __fsub_rn(t, floorf(t));
+    if (fabsf(__fsub_rn(f, 0.5f)) > fabsf(t) * 4.76837158203125e-7f)   // 2^-21
+        return __float2int_rn(t);
+    return __float2int_rn(__fdiv_rn(w, sf));
+}
+
+// One group held by a half-warp, four weights per lane: scale bits, codes,
+// status (0, 5 = NONFINITE, 6 = RANGE).
+template <int BITS>
+__device__ __forceinline__ void quantize_group16(const float4 v, unsigned half_mask,
+                                                 uint16_t& s_bits, int (&c)[4], int& status) {
+    constexpr int kQmax = BITS == 4 ? 7 : 127;
+    const bool finite = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+    float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(half_mask, a, off));
+    const bool all_finite = __all_sync(half_mask, finite);
+
+    const float s32 = __fdiv_rn(a, static_cast<float>(kQmax));
+    const __half s16 = __float2half_rn(s32);
+    s_bits = __half_as_ushort(s16);
+    const float sf = __half2float(s16);
+    status = 0;
+    c[0] = c[1] = c[2] = c[3] = 0;
+    if (!all_finite) {
+        s_bits = 0x7E00u;
+        status = 5;  // RQ_ERR_NONFINITE
+    } else if (s_bits == 0x7C00u) {
+        status = 6;  // RQ_ERR_RANGE
+    } else if (sf != 0.0f) {
+        const float r = __frcp_rn(sf);
+        const float w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c[i] = max(-kQmax, min(kQmax, rint_quotient(w[i], sf, r)));
+    }
+}
+
+template <int BITS>
+__device__ __forceinline__ void store_group16(int64_t gid, int lane16, uint16_t s_bits,
+                                              const int (&c)[4], uint8_t* __restrict__ codes,
+                                              uint16_t* __restrict__ scales) {
+    if (BITS == 4) {
+        const uint16_t packed = static_cast<uint16_t>((c[0] & 0xF) | ((c[1] & 0xF) << 4) |
+                                                      ((c[2] & 0xF) << 8) | ((c[3] & 0xF) << 12));
+        __stcs(reinterpret_cast<unsigned short*>(codes + gid * 32 + lane16 * 2), packed);
+    } else {
+        const uint32_t packed = (c[0] & 0xFF) | ((c[1] & 0xFF) << 8) | ((c[2] & 0xFF) << 16) |
+                                (static_cast<uint32_t>(c[3] & 0xFF) << 24);
+        __stcs(reinterpret_cast<unsigned int*>(codes + gid * 64 + lane16 * 4), packed);
+    }
+    if (lane16 == 0) scales[gid] = s_bits;
+}
+
+// NONFINITE overrides everything; RANGE only replaces OK.
+__device__ __forceinline__ void raise_status(int* dev_status, int status) {
+    if (dev_status == nullptr) return;
+    if (status == 5) atomicExch(dev_status, 5);
+    else if (status == 6) atomicCAS(dev_status, 0, 6);
+}
+
+// Half-warp h takes groups h + H*(kQU*i + j), j < kQU, for i = 0, 1, ...
+// (H = half-warps in the grid): the kQU groups' loads are issued together.
+constexpr int kQU = 4;
+
 template <int BITS>
 __global__ void __launch_bounds__(256) quantize_g64_kernel(const float4* __restrict__ W,
                                                            int64_t n_groups,
                                                            uint8_t* __restrict__ codes,
                                                            uint16_t* __restrict__ scales,
                                                            int* __restrict__ dev_status) {
-    constexpr int kQmax = BITS == 4 ? 7 : 127;
     const int lane16 = threadIdx.x & 15;
     const unsigned half_mask = 0xFFFFu << (threadIdx.x & 16);
     const int64_t first = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
     const int64_t step = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
 
-    for (int64_t gid = first; gid < n_groups; gid += step) {
-        const float4 v = __ldcs(&W[gid * 16 + lane16]);
-        const bool finite = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
-        float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    for (int64_t g0 = first; g0 < n_groups; g0 += kQU * step) {
+        float4 v[kQU];
 #pragma unroll
-        for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(half_mask, a, off));
-        const bool all_finite = __all_sync(half_mask, finite);
-
-        const float s32 = __fdiv_rn(a, static_cast<float>(kQmax));
-        const __half s16 = __float2half_rn(s32);
-        uint16_t s_bits = __half_as_ushort(s16);
-        const float sf = __half2float(s16);
-        int status = 0;
-        int c[4] = {0, 0, 0, 0};
-        if (!all_finite) {
-            s_bits = 0x7E00u;
-            status = 5;  // RQ_ERR_NONFINITE
-        } else if (s_bits == 0x7C00u) {
-            status = 6;  // RQ_ERR_RANGE
-        } else if (sf != 0.0f) {
-            const float w[4] = {v.x, v.y, v.z, v.w};
+        for (int j = 0; j < kQU; ++j) {
+            const int64_t gid = g0 + j * step;
+            v[j] = gid < n_groups ? __ldcs(&W[gid * 16 + lane16]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        int status_any = 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                int q = __float2int_rn(__fdiv_rn(w[i], sf));
-                c[i] = max(-kQmax, min(kQmax, q));
-            }
+        for (int j = 0; j < kQU; ++j) {
+            const int64_t gid = g0 + j * step;
+            if (gid >= n_groups) break;   // uniform over the half-warp
+            uint16_t s_bits;
+            int c[4], status;
+            quantize_group16<BITS>(v[j], half_mask, s_bits, c, status);
+            store_group16<BITS>(gid, lane16, s_bits, c, codes, scales);
+            if (status == 5 || (status == 6 && status_any == 0)) status_any = status;
         }
-        if (BITS == 4) {
-            const uint16_t packed = static_cast<uint16_t>((c[0] & 0xF) | ((c[1] & 0xF) << 4) |
-                                                          ((c[2] & 0xF) << 8) |
-                                                          ((c[3] & 0xF) << 12));
-            __stcs(reinterpret_cast<unsigned short*>(codes + gid * 32 + lane16 * 2), packed);
-        } else {
-            const uint32_t packed = (c[0] & 0xFF) | ((c[1] & 0xFF) << 8) | ((c[2] & 0xFF) << 16) |
-                                    (static_cast<uint32_t>(c[3] & 0xFF) << 24);
-            __stcs(reinterpret_cast<unsigned int*>(codes + gid * 64 + lane16 * 4), packed);
-        }
-        if (lane16 == 0) {
-            scales[gid] = s_bits;
-            // NONFINITE overrides everything; RANGE only replaces OK.
-            if (dev_status != nullptr) {
-                if (status == 5) atomicExch(dev_status, 5);
-                else if (status == 6) atomicCAS(dev_status, 0, 6);
-            }
-        }
+        if (lane16 == 0 && status_any != 0) raise_status(dev_status, status_any);
     }
+}
+
+// Blocks of 256 threads: as many as are resident on every SM at once (the
+// loop walks the rest), no more than the groups need.
+static int quantize_grid(int64_t n_groups, const void* kern) {
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        sms = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0) != cudaSuccess ||
+        per_sm <= 0)
+        per_sm = 1;
+    const int64_t need = (n_groups + 15) / 16;
+    const int64_t full = static_cast<int64_t>(sms) * per_sm;
+    return static_cast<int>(need < full ? need : full);
 }
 
 cudaError_t launch_quantize(const float* W, int64_t n_groups, int bits, void* codes,
                             uint16_t* scales, int* dev_status, cudaStream_t s) {
     if (n_groups <= 0) return cudaSuccess;
     const int threads = 256;
-    const int64_t groups_per_block = threads / 16;
-    int64_t blocks = (n_groups + groups_per_block - 1) / groups_per_block;
-    const int64_t cap = 148LL * 8 * 4;  // a few waves of fully resident blocks, then grid-stride
-    if (blocks > cap) blocks = cap;
-    if (bits == 4)
+    if (bits == 4) {
+        const int blocks = quantize_grid(n_groups, reinterpret_cast<const void*>(quantize_g64_kernel<4>));
         quantize_g64_kernel<4><<<static_cast<unsigned>(blocks), threads, 0, s>>>(
             reinterpret_cast<const float4*>(W), n_groups, static_cast<uint8_t*>(codes), scales,
             dev_status);
-    else
+    } else {
+        const int blocks = quantize_grid(n_groups, reinterpret_cast<const void*>(quantize_g64_kernel<8>));
         quantize_g64_kernel<8><<<static_cast<unsigned>(blocks), threads, 0, s>>>(
             reinterpret_cast<const float4*>(W), n_groups, static_cast<uint8_t*>(codes), scales,
             dev_status);
+    }
     return cudaGetLastError();
 }
 
@@ -146,6 +208,7 @@ __global__ void __launch_bounds__(256) quantize_g64_ex2_kernel(
         const __half s16j = __float2half_rn(__fdiv_rn(a32, static_cast<float>(kQmax)));
         const float sfj = __half2float(s16j);
         const bool valid = lane16 < nf && __half_as_ushort(s16j) != 0x7C00u;
+        const float rj = (sfj != 0.0f && valid) ? __frcp_rn(sfj) : 0.0f;
         const float wv[4] = {v.x, v.y, v.z, v.w};
         const float evv[4] = {ev.x, ev.y, ev.z, ev.w};
         float err = 0.0f;
@@ -154,7 +217,7 @@ __global__ void __launch_bounds__(256) quantize_g64_ex2_kernel(
             const float wk = __shfl_sync(half_mask, wv[k & 3], base + (k >> 2));
             const float ek = __shfl_sync(half_mask, evv[k & 3], base + (k >> 2));
             int c = 0;
-            if (sfj != 0.0f) c = max(-kQmax, min(kQmax, __float2int_rn(__fdiv_rn(wk, sfj))));
+            if (sfj != 0.0f) c = max(-kQmax, min(kQmax, rint_quotient(wk, sfj, rj)));
             const float t = __fmul_rn(static_cast<float>(c), sfj);
             const float d = __fsub_rn(wk, t);
             err = __fadd_rn(err, __fmul_rn(ek, __fmul_rn(d, d)));
@@ -187,11 +250,9 @@ __global__ void __launch_bounds__(256) quantize_g64_ex2_kernel(
         } else if (s_bits == 0x7C00u) {
             status = 6;  // RQ_ERR_RANGE
         } else if (sf != 0.0f) {
+            const float r = __frcp_rn(sf);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int q = __float2int_rn(__fdiv_rn(wv[i], sf));
-                c[i] = max(-kQmax, min(kQmax, q));
-            }
+            for (int i = 0; i < 4; ++i) c[i] = max(-kQmax, min(kQmax, rint_quotient(wv[i], sf, r)));
         }
         if (BITS == 4) {
             const uint16_t packed = static_cast<uint16_t>((c[0] & 0xF) | ((c[1] & 0xF) << 4) |
@@ -221,10 +282,9 @@ cudaError_t launch_quantize_ex2(const float* W, int64_t N, int64_t K, int bits, 
     const int64_t n_groups = N * groups_per_row;
     if (n_groups <= 0) return cudaSuccess;
     const int threads = 256;
-    const int64_t groups_per_block = threads / 16;
-    int64_t blocks = (n_groups + groups_per_block - 1) / groups_per_block;
-    const int64_t cap = 148LL * 8 * 4;
-    if (blocks > cap) blocks = cap;
+    const int blocks = quantize_grid(
+        n_groups, bits == 4 ? reinterpret_cast<const void*>(quantize_g64_ex2_kernel<4>)
+                            : reinterpret_cast<const void*>(quantize_g64_ex2_kernel<8>));
     if (bits == 4)
         quantize_g64_ex2_kernel<4><<<static_cast<unsigned>(blocks), threads, 0, s>>>(
             reinterpret_cast<const float4*>(W), n_groups, groups_per_row,

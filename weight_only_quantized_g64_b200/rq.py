@@ -22,7 +22,7 @@ MAX_DECODE_M = 32
 STATUS = {0: "RQ_OK", 1: "RQ_ERR_NULL", 2: "RQ_ERR_BITS", 3: "RQ_ERR_SHAPE", 4: "RQ_ERR_ALIGN",
           5: "RQ_ERR_NONFINITE", 6: "RQ_ERR_RANGE", 7: "RQ_ERR_TIMEOUT", 8: "RQ_ERR_CUDA"}
 OK, ERR_NULL, ERR_BITS, ERR_SHAPE, ERR_ALIGN, ERR_NONFINITE, ERR_RANGE, ERR_TIMEOUT, ERR_CUDA = range(9)
-DECODE_KERNELS = {"auto": 0, "rowtile": 1, "cluster": 2}
+DECODE_KERNELS = {"auto": 0, "rowtile": 1, "cluster": 2, "rowblock": 3}
 
 _lib = None
 
@@ -62,6 +62,16 @@ def lib():
     L.rq_gemv_wq_noalloc.restype = i32
     L.rq_rkv_fused.argtypes = [vp, i64, i64, i64, i32] + [vp] * 9 + [vp]
     L.rq_rkv_fused.restype = i32
+    L.rq_gptq_hessian.argtypes = [vp, i64, i64, vp, vp]
+    L.rq_gptq_hessian.restype = i32
+    L.rq_gptq_factor.argtypes = [vp, i64, ctypes.c_double, vp, vp, vp, vp]
+    L.rq_gptq_factor.restype = i32
+    L.rq_gptq_g64.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp]
+    L.rq_gptq_g64.restype = i32
+    L.rq_gemv_wq_ex.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, i32, i32, vp]
+    L.rq_gemv_wq_ex.restype = i32
+    L.rq_rkv_fused3.argtypes = [vp, vp, vp, i64, i64, i64, i32] + [vp] * 9 + [i32, vp]
+    L.rq_rkv_fused3.restype = i32
     L.rq_set_pdl.argtypes = [i32]
     L.rq_set_pdl.restype = i32
     L.rq_set_decode_kernel.argtypes = [i32]
@@ -147,6 +157,39 @@ def quantize_g64_ex2(W: torch.Tensor, e2: torch.Tensor, bits: int, factors: torc
     return codes, scales, chosen
 
 
+def gptq_hessian(X: torch.Tensor, H=None, stream=None):
+    """H = (2/T) X^T X (fp64 [K, K]) of calibration inputs X fp16 [T, K]."""
+    T, K = X.shape
+    if H is None:
+        H = torch.empty((K, K), dtype=torch.float64, device=X.device)
+    _check(lib().rq_gptq_hessian(_p(X), T, K, _p(H), _stream(stream)), "rq_gptq_hessian")
+    return H
+
+
+def gptq_factor(H: torch.Tensor, damp: float = 0.01, stream=None):
+    """(U fp32 [K, K], dead uint8 [K]) from H (consumed)."""
+    K = H.shape[0]
+    U = torch.empty((K, K), dtype=torch.float32, device=H.device)
+    dead = torch.empty((K,), dtype=torch.uint8, device=H.device)
+    work = torch.empty((K * K + K,), dtype=torch.float64, device=H.device)
+    _check(lib().rq_gptq_factor(_p(H), K, float(damp), _p(U), _p(dead), _p(work), _stream(stream)),
+           "rq_gptq_factor")
+    return U, dead
+
+
+def gptq_g64(W: torch.Tensor, bits: int, U: torch.Tensor, dead=None, codes=None, scales=None,
+             dev_status=None, stream=None):
+    """GPTQ column loop on the group-64 grid; W fp32 [N, K] is overwritten with
+    the compensated weights.  Returns (codes, scales)."""
+    N, K = W.shape
+    if codes is None:
+        codes, scales = empty_weights(N, K, bits, W.device)
+    work = torch.empty((N, 128), dtype=torch.float32, device=W.device)
+    _check(lib().rq_gptq_g64(_p(W), N, K, bits, _p(U), _p(dead), _p(codes), _p(scales), _p(work),
+                             _p(dev_status), _stream(stream)), "rq_gptq_g64")
+    return codes, scales
+
+
 def gemv_wq(x: torch.Tensor, codes, scales, N: int, bits: int, y=None, stream=None):
     """Decode product y[M, N] = x[M, K] @ w_hat^T, 1 <= M <= 32."""
     M, K = x.shape
@@ -166,6 +209,36 @@ def gemv_wq_noalloc(x: torch.Tensor, codes, scales, N: int, bits: int, y=None, s
     _check(lib().rq_gemv_wq_noalloc(_p(x), M, K, _p(codes), _p(scales), N, bits, _p(y),
                                     _stream(stream)), "rq_gemv_wq_noalloc")
     return y
+
+
+OUT_F32, OUT_F16 = 0, 1
+EPI_NONE, EPI_RELU_SQ = 0, 1
+
+
+def gemv_wq_ex(x: torch.Tensor, codes, scales, N: int, bits: int, out_dtype=torch.float32,
+               epilogue: int = EPI_NONE, y=None, stream=None):
+    """Decode product with the output stored as fp32 or fp16 and an optional
+    fused epilogue (EPI_RELU_SQ: max(y, 0)^2)."""
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    od = OUT_F16 if y.dtype == torch.float16 else OUT_F32
+    _check(lib().rq_gemv_wq_ex(_p(x), M, K, _p(codes), _p(scales), N, bits, _p(y), od, epilogue,
+                               _stream(stream)), "rq_gemv_wq_ex")
+    return y
+
+
+def rkv_fused3(xr: torch.Tensor, xk: torch.Tensor, xv: torch.Tensor, wr, wk, wv, N: int, bits: int,
+               out_dtype=torch.float32, ys=None, stream=None):
+    """R/K/V projections, each with its own input, in one launch."""
+    M, K = xr.shape
+    if ys is None:
+        ys = tuple(torch.empty((M, N), dtype=out_dtype, device=xr.device) for _ in range(3))
+    od = OUT_F16 if ys[0].dtype == torch.float16 else OUT_F32
+    _check(lib().rq_rkv_fused3(_p(xr), _p(xk), _p(xv), M, K, N, bits, _p(wr[0]), _p(wr[1]),
+                               _p(wk[0]), _p(wk[1]), _p(wv[0]), _p(wv[1]), _p(ys[0]), _p(ys[1]),
+                               _p(ys[2]), od, _stream(stream)), "rq_rkv_fused3")
+    return ys
 
 
 def gemm_wq(x: torch.Tensor, codes, scales, N: int, bits: int, y=None, stream=None):
@@ -194,12 +267,12 @@ def set_pdl(enable: bool):
 
 
 def set_decode_kernel(kind: str):
-    """Decode kernel for later products: "auto", "rowtile" or "cluster"."""
+    """Decode kernel for later products: "auto", "rowtile", "cluster" or "rowblock"."""
     _check(lib().rq_set_decode_kernel(DECODE_KERNELS[kind]), "rq_set_decode_kernel")
 
 
 def decode_kernel_for(M: int, K: int, N: int, bits: int, nmat: int = 1) -> str:
-    """The decode kernel ("rowtile" or "cluster") a product of this shape runs on."""
+    """The decode kernel ("rowtile", "cluster" or "rowblock") a product of this shape runs on."""
     out = ctypes.c_int(-1)
     _check(lib().rq_decode_kernel_for(M, K, N, bits, nmat, ctypes.byref(out)), "rq_decode_kernel_for")
     return {v: k for k, v in DECODE_KERNELS.items()}[out.value]
