@@ -79,6 +79,15 @@ def _load():
     lib.rqo_get_code.restype = ctypes.c_int
     lib.rqo_gptq_g64.argtypes = [vp, i64, i64, ctypes.c_int, vp, vp, vp, vp]
     lib.rqo_gptq_g64.restype = ctypes.c_int
+    lib.rqo_quantize_sym.argtypes = [vp, i64, i64, ctypes.c_int, ctypes.c_int, vp, vp, ctypes.c_int,
+                                     vp, vp, vp]
+    lib.rqo_quantize_sym.restype = ctypes.c_int
+    lib.rqo_quantize_p4a.argtypes = [vp, i64, i64, vp, vp, ctypes.c_int, vp, vp, vp, vp]
+    lib.rqo_quantize_p4a.restype = ctypes.c_int
+    lib.rqo_get_ucode4.argtypes = [vp, i64, i64, i64]
+    lib.rqo_get_ucode4.restype = ctypes.c_int
+    lib.rqo_matmul_fmt.argtypes = [ctypes.c_int, vp, i64, i64, vp, vp, vp, i64, i64, vp, vp, vp, vp]
+    lib.rqo_matmul_fmt.restype = None
     _lib = lib
     return lib
 
@@ -242,3 +251,85 @@ def relu_sq_budget(y_ref: np.ndarray, delta: np.ndarray) -> np.ndarray:
     """Error budget of relu(a)^2 when |a - y_ref| <= delta:
     |relu(a)^2 - relu(b)^2| <= |a - b| (relu(a) + relu(b)) <= delta (2 relu(b) + delta)."""
     return delta * (2.0 * np.maximum(y_ref, 0.0) + delta)
+
+
+# ------------------------------------------- preset formats ("rwkv-quant") --
+# "rwkv-quant: uma matriz em bf16 elimina 39% das perdas na quantização do
+# RWKV-7 2.9B", "Dois presets e seis tamanhos": REDUCTION projections in 8
+# bits, symmetric, groups of 16; COMPRESSION projections in 4 bits,
+# asymmetric, super-blocks, groups of 32; scales and offsets chosen by a
+# search weighted by E[x^2].  The readings are written at the top of the
+# preset section of rqo.c.
+
+
+def _search_args(e2, factors, K):
+    if e2 is None:
+        return None, np.ones(1, np.float32), 1
+    e2 = np.ascontiguousarray(e2, dtype=np.float32)
+    f = np.ascontiguousarray(factors if factors is not None else [1.0], dtype=np.float32)
+    if e2.shape != (K,) or f.ndim != 1 or f.size < 1:
+        raise ValueError("e2 must have K values and factors at least one")
+    return e2, f, int(f.size)
+
+
+def quantize_sym(W: np.ndarray, bits: int, G: int, e2=None, factors=None):
+    """Symmetric group-G quantization (RTN when e2 is None, else the
+    E[x^2]-weighted scale search over `factors`).  Returns (codes, scales
+    uint16 [N, K/G], chosen int32 [N, K/G], status)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    if bits not in (4, 8) or G not in (16, 32, 64) or K % G:
+        raise ValueError("bits 4/8, G in {16, 32, 64}, K a multiple of G")
+    e2a, f, nf = _search_args(e2, factors, K)
+    codes = np.zeros((N, K * bits // 8), dtype=np.uint8)
+    scales = np.zeros((N, K // G), dtype=np.uint16)
+    chosen = np.zeros((N, K // G), dtype=np.int32)
+    st = _load().rqo_quantize_sym(_ptr(W), N, K, bits, G, _ptr(e2a) if e2a is not None else None,
+                                  _ptr(f), nf, _ptr(codes), _ptr(scales), _ptr(chosen))
+    return codes, scales, chosen, int(st)
+
+
+def quantize_p4a(W: np.ndarray, e2=None, factors=None):
+    """Asymmetric int4, groups of 32 in super-blocks of 8 groups.  Returns
+    (codes uint8 [N, K/2], sub uint8 [N, K/32, 2] = (a, b), sup uint16
+    [N, K/256, 2] = (ds, dm) fp16 bits, chosen int32 [N, K/32], status)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    if K % 256:
+        raise ValueError("K must be a multiple of 256")
+    e2a, f, nf = _search_args(e2, factors, K)
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    sub = np.zeros((N, K // 32, 2), dtype=np.uint8)
+    sup = np.zeros((N, K // 256, 2), dtype=np.uint16)
+    chosen = np.zeros((N, K // 32), dtype=np.int32)
+    st = _load().rqo_quantize_p4a(_ptr(W), N, K, _ptr(e2a) if e2a is not None else None, _ptr(f), nf,
+                                  _ptr(codes), _ptr(sub), _ptr(sup), _ptr(chosen))
+    return codes, sub, sup, chosen, int(st)
+
+
+def matmul_fmt(fmt: int, x_f16: np.ndarray, codes, meta0, meta1=None, ms=None, ns=None):
+    """Products of the preset formats in fp64 with the budget sum |x||w_hat|:
+    fmt 8 = int8 g16 symmetric (meta0 = scales [N, K/16]); fmt 4 = int4 g32
+    asymmetric super-blocks (meta0 = sub, meta1 = sup).  Every output, or the
+    sampled pairs (ms[p], ns[p])."""
+    x = np.ascontiguousarray(x_f16).view(np.uint16)
+    M, K = x.shape
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    m0 = np.ascontiguousarray(meta0)
+    m1 = None if meta1 is None else np.ascontiguousarray(meta1)
+    N = m0.shape[0]
+    if ms is None:
+        P = M * N
+        y = np.zeros(P, np.float64)
+        b = np.zeros(P, np.float64)
+        _load().rqo_matmul_fmt(fmt, _ptr(x), M, K, _ptr(codes), _ptr(m0),
+                               _ptr(m1) if m1 is not None else None, N, P, None, None, _ptr(y), _ptr(b))
+        return y.reshape(M, N), b.reshape(M, N)
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    P = ms.shape[0]
+    y = np.zeros(P, np.float64)
+    b = np.zeros(P, np.float64)
+    _load().rqo_matmul_fmt(fmt, _ptr(x), M, K, _ptr(codes), _ptr(m0), _ptr(m1) if m1 is not None else None,
+                           N, P, _ptr(ms), _ptr(ns), _ptr(y), _ptr(b))
+    return y, b

@@ -485,3 +485,326 @@ int rqo_gptq_g64(float *W, int64_t N, int64_t K, int bits, const float *U, const
     }
     return status;
 }
+
+/* --------------------------------------------------- preset formats (f3) --- */
+/*
+ * The two presets of "rwkv-quant: uma matriz em bf16 elimina 39% das perdas na
+ * quantização do RWKV-7 2.9B", section "Dois presets e seis tamanhos":
+ * REDUCTION stores projections in 8 bits, symmetric, groups of 16 weights;
+ * COMPRESSION stores them in 4 bits, asymmetric, in super-blocks, groups of
+ * 32; in both, each group's scale (and offset) is chosen by a search weighted
+ * by E[x^2] of the input channel.  Readings where the page is silent:
+ *
+ * int8 g16 symmetric ("p8"): exactly the g64 steps of rqo_quantize_g64 /
+ *   rqo_quantize_g64_ex2 with groups of G = 16 (scale fp16_rn(fp32 amax * f /
+ *   127), RTN codes, the smallest sum e2 (w - c s)^2 wins, earlier on ties).
+ *   Written once for any G here; G = 64 reproduces the g64 functions.
+ *
+ * int4 g32 asymmetric in super-blocks of 8 groups ("p4a"), per row:
+ *   group g (32 weights): lo = min(0, min w), hi = max(0, max w);
+ *     candidate j: lo_j = fp32(lo * f_j), hi_j = fp32(hi * f_j),
+ *       s_j = fp32(fp32(hi_j - lo_j) / 15), o_j = lo_j,
+ *       q = clamp(rint(fp32(w - o_j) / s_j), 0, 15)  (q = 0 when s_j == 0),
+ *       err_j = sum_k e2[k] * (w - (q s_j + o_j))^2, one fp32 rounding per
+ *       operation in k order; the smallest err_j wins (earlier on ties);
+ *     without a search (e2 NULL) the single candidate f = 1;
+ *   super-block (8 groups): ds = fp16_rn(fp32(max_g s_g) / 63),
+ *     dm = fp16_rn(fp32(max_g -o_g) / 63);
+ *     a_g = clamp(rint(s_g / ds), 0, 63), b_g = clamp(rint(-o_g / dm), 0, 63)
+ *     (0 when ds / dm is 0);
+ *   stored scale and offset: S_g = ds * a_g, O_g = -(dm * b_g) (exact in fp32);
+ *   codes q = clamp(rint(fp32(w - O_g) / S_g), 0, 15) (q = 0 when S_g == 0);
+ *   w_hat = S_g * q + O_g.
+ *   Layout: codes uint8 [N, K/2] (q unsigned, k = 2j in the low nibble);
+ *   sub uint8 [N, K/32, 2] = {a_g, b_g}; sup fp16 [N, K/256, 2] = {ds, dm}.
+ *   K % 256 == 0.  A super-block holding a non-finite weight gets ds = dm =
+ *   0x7E00, sub-codes and codes 0, status NONFINITE; one whose ds or dm
+ *   overflows fp16 keeps the inf, sub-codes and codes 0, status RANGE.
+ */
+
+/* Symmetric group of G weights, optional E[x^2] search (e2 NULL: RTN). */
+static int quantize_sym_group(const float *w, int G, int bits, const float *e2, const float *f,
+                              int nf, uint16_t *scale_out, int *c_out, int *chosen_out)
+{
+    const int qmax = qmax_of(bits);
+    int i, j;
+    *chosen_out = 0;
+    for (i = 0; i < G; i++) {
+        if (!isfinite(w[i])) {
+            *scale_out = 0x7E00u;
+            for (i = 0; i < G; i++) c_out[i] = 0;
+            return RQO_ERR_NONFINITE;
+        }
+    }
+    float amax = 0.0f;
+    for (i = 0; i < G; i++) {
+        float a = fabsf(w[i]);
+        if (a > amax) amax = a;
+    }
+    const int ncand = e2 ? nf : 1;
+    int best = -1;
+    float best_err = 0.0f;
+    int cj[64];
+    for (j = 0; j < ncand; j++) {
+        volatile float a32 = e2 ? amax * f[j] : amax;
+        volatile float s32 = a32 / (float)qmax;
+        uint16_t s16 = rqo_f32_to_f16(s32);
+        if (s16 == 0x7C00u) continue;
+        float sf = (float)rqo_f16_to_f64(s16);
+        volatile float err = 0.0f;
+        for (i = 0; i < G; i++) {
+            int c = 0;
+            if (sf != 0.0f) {
+                volatile float t0 = w[i] / sf;
+                float r = rintf(t0);
+                if (r > (float)qmax) r = (float)qmax;
+                if (r < (float)-qmax) r = (float)-qmax;
+                c = (int)r;
+            }
+            cj[i] = c;
+            if (e2) {
+                volatile float t = (float)c * sf;
+                volatile float d = w[i] - t;
+                volatile float q = d * d;
+                volatile float pr = e2[i] * q;
+                err = err + pr;
+            }
+        }
+        if (best < 0 || err < best_err) {
+            best = j;
+            best_err = err;
+            *scale_out = s16;
+            for (i = 0; i < G; i++) c_out[i] = cj[i];
+        }
+    }
+    if (best < 0) {
+        /* every candidate's scale overflows: RTN decides (as the g64 search
+         * does); RTN's own overflow gives scale +inf, codes 0, RANGE */
+        if (e2) return quantize_sym_group(w, G, bits, 0, f, nf, scale_out, c_out, chosen_out);
+        *scale_out = 0x7C00u;
+        for (i = 0; i < G; i++) c_out[i] = 0;
+        return RQO_ERR_RANGE;
+    }
+    *chosen_out = best;
+    return RQO_OK;
+}
+
+/* Symmetric group-G quantization of W[N, K] (K % G == 0, G in {16, 32, 64}):
+ * codes as rqo_quantize_g64, scales fp16 [N, K/G], chosen (nullable) [N, K/G].
+ * e2 NULL: RTN. */
+int rqo_quantize_sym(const float *W, int64_t N, int64_t K, int bits, int G, const float *e2,
+                     const float *f, int nf, uint8_t *codes, uint16_t *scales, int32_t *chosen)
+{
+    const int64_t NG = K / G;
+    int status = RQO_OK;
+    int64_t n;
+#pragma omp parallel for schedule(static) reduction(max : status)
+    for (n = 0; n < N; n++) {
+        int c[64];
+        int64_t g;
+        for (g = 0; g < NG; g++) {
+            int ch = 0;
+            int st = quantize_sym_group(&W[n * K + g * G], G, bits, e2 ? &e2[g * G] : 0, f, nf,
+                                        &scales[n * NG + g], c, &ch);
+            int64_t i;
+            for (i = 0; i < G; i++) put_code(codes, K, bits, n, g * G + i, c[i]);
+            if (chosen) chosen[n * NG + g] = ch;
+            if (st > status) status = st;
+        }
+    }
+    if (status != RQO_OK) {
+        int64_t i, total = N * NG;
+        for (i = 0; i < total; i++) if (scales[i] == 0x7E00u) return RQO_ERR_NONFINITE;
+    }
+    return status;
+}
+
+/* Unsigned 4-bit code store / load (asymmetric format). */
+static void put_ucode4(uint8_t *codes, int64_t K, int64_t n, int64_t k, int q)
+{
+    uint8_t *b = &codes[n * (K / 2) + k / 2];
+    if (k % 2 == 0) *b = (uint8_t)((*b & 0xF0u) | (q & 0xF));
+    else            *b = (uint8_t)((*b & 0x0Fu) | ((q & 0xF) << 4));
+}
+
+int rqo_get_ucode4(const uint8_t *codes, int64_t K, int64_t n, int64_t k)
+{
+    uint8_t b = codes[n * (K / 2) + k / 2];
+    return (k % 2 == 0) ? (b & 0xF) : (b >> 4);
+}
+
+static int rint_clamp(float t, int lo, int hi)
+{
+    float r = rintf(t);
+    if (r > (float)hi) r = (float)hi;
+    if (r < (float)lo) r = (float)lo;
+    return (int)r;
+}
+
+/* One asymmetric group of 32: the chosen (s, o) in fp32. */
+static void p4a_group_choice(const float *w, const float *e2, const float *f, int nf, float *s_out,
+                             float *o_out, int *chosen_out)
+{
+    int i, j;
+    float lo = 0.0f, hi = 0.0f;
+    for (i = 0; i < 32; i++) {
+        if (w[i] < lo) lo = w[i];
+        if (w[i] > hi) hi = w[i];
+    }
+    const int ncand = e2 ? nf : 1;
+    int best = -1;
+    float best_err = 0.0f, bs = 0.0f, bo = 0.0f;
+    for (j = 0; j < ncand; j++) {
+        volatile float loj = e2 ? lo * f[j] : lo;
+        volatile float hij = e2 ? hi * f[j] : hi;
+        volatile float rng = hij - loj;
+        volatile float sj = rng / 15.0f;
+        volatile float err = 0.0f;
+        if (e2) {
+            for (i = 0; i < 32; i++) {
+                int q = 0;
+                if (sj != 0.0f) {
+                    volatile float dw = w[i] - loj;
+                    volatile float t = dw / sj;
+                    q = rint_clamp(t, 0, 15);
+                }
+                volatile float t1 = (float)q * sj;
+                volatile float u = t1 + loj;
+                volatile float d = w[i] - u;
+                volatile float qq = d * d;
+                volatile float pr = e2[i] * qq;
+                err = err + pr;
+            }
+        }
+        if (best < 0 || err < best_err) {
+            best = j;
+            best_err = err;
+            bs = sj;
+            bo = loj;
+        }
+    }
+    *s_out = bs;
+    *o_out = bo;
+    *chosen_out = best;
+}
+
+/* Asymmetric int4 g32 super-block quantization of W[N, K] (K % 256 == 0).
+ * codes uint8 [N, K/2]; sub uint8 [N, K/32, 2]; sup fp16 [N, K/256, 2];
+ * chosen (nullable) int32 [N, K/32]; e2 NULL: no search (factor 1). */
+int rqo_quantize_p4a(const float *W, int64_t N, int64_t K, const float *e2, const float *f, int nf,
+                     uint8_t *codes, uint8_t *sub, uint16_t *sup, int32_t *chosen)
+{
+    const int64_t NSB = K / 256, NG = K / 32;
+    int status = RQO_OK;
+    int64_t n;
+#pragma omp parallel for schedule(static) reduction(max : status)
+    for (n = 0; n < N; n++) {
+        int64_t sb;
+        for (sb = 0; sb < NSB; sb++) {
+            const float *w = &W[n * K + sb * 256];
+            int i, g;
+            int finite = 1;
+            for (i = 0; i < 256; i++) if (!isfinite(w[i])) finite = 0;
+            uint16_t *sp = &sup[(n * NSB + sb) * 2];
+            uint8_t *ab = &sub[(n * NG + sb * 8) * 2];
+            if (!finite) {
+                sp[0] = sp[1] = 0x7E00u;
+                for (g = 0; g < 16; g++) ab[g] = 0;
+                for (i = 0; i < 256; i++) put_ucode4(codes, K, n, sb * 256 + i, 0);
+                if (chosen) for (g = 0; g < 8; g++) chosen[n * NG + sb * 8 + g] = 0;
+                if (RQO_ERR_NONFINITE > status) status = RQO_ERR_NONFINITE;
+                continue;
+            }
+            float s[8], o[8];
+            float smax = 0.0f, omax = 0.0f;
+            for (g = 0; g < 8; g++) {
+                int ch = 0;
+                p4a_group_choice(&w[g * 32], e2 ? &e2[sb * 256 + g * 32] : 0, f, nf, &s[g], &o[g], &ch);
+                if (chosen) chosen[n * NG + sb * 8 + g] = ch;
+                if (s[g] > smax) smax = s[g];
+                if (-o[g] > omax) omax = -o[g];
+            }
+            volatile float ds32 = smax / 63.0f;
+            volatile float dm32 = omax / 63.0f;
+            uint16_t ds = rqo_f32_to_f16(ds32), dm = rqo_f32_to_f16(dm32);
+            sp[0] = ds;
+            sp[1] = dm;
+            if (ds == 0x7C00u || dm == 0x7C00u) {
+                for (g = 0; g < 16; g++) ab[g] = 0;
+                for (i = 0; i < 256; i++) put_ucode4(codes, K, n, sb * 256 + i, 0);
+                if (RQO_ERR_RANGE > status) status = RQO_ERR_RANGE;
+                continue;
+            }
+            const float dsf = (float)rqo_f16_to_f64(ds), dmf = (float)rqo_f16_to_f64(dm);
+            for (g = 0; g < 8; g++) {
+                int a = 0, b = 0;
+                if (dsf != 0.0f) {
+                    volatile float t = s[g] / dsf;
+                    a = rint_clamp(t, 0, 63);
+                }
+                if (dmf != 0.0f) {
+                    volatile float t = -o[g] / dmf;
+                    b = rint_clamp(t, 0, 63);
+                }
+                ab[2 * g] = (uint8_t)a;
+                ab[2 * g + 1] = (uint8_t)b;
+                volatile float S = dsf * (float)a;
+                volatile float O = -(dmf * (float)b);
+                for (i = 0; i < 32; i++) {
+                    int q = 0;
+                    if (S != 0.0f) {
+                        volatile float dw = w[g * 32 + i] - O;
+                        volatile float t = dw / S;
+                        q = rint_clamp(t, 0, 15);
+                    }
+                    put_ucode4(codes, K, n, sb * 256 + g * 32 + i, q);
+                }
+            }
+        }
+    }
+    return status;
+}
+
+/* Dequantised weight of the preset formats, exact in fp64.
+ * fmt 8: int8 g16 symmetric (meta0 = scales fp16 [N, K/16]);
+ * fmt 4: int4 g32 asymmetric super-blocks (meta0 = sub, meta1 = sup). */
+static double fmt_weight(int fmt, const uint8_t *codes, const void *meta0, const void *meta1,
+                         int64_t K, int64_t n, int64_t k)
+{
+    if (fmt == 8) {
+        const uint16_t *sc = (const uint16_t *)meta0;
+        return (double)(int)(int8_t)codes[n * K + k] * rqo_f16_to_f64(sc[n * (K / 16) + k / 16]);
+    }
+    const uint8_t *sub = (const uint8_t *)meta0;
+    const uint16_t *sup = (const uint16_t *)meta1;
+    const int64_t g = k / 32, sb = k / 256;
+    const double ds = rqo_f16_to_f64(sup[(n * (K / 256) + sb) * 2]);
+    const double dm = rqo_f16_to_f64(sup[(n * (K / 256) + sb) * 2 + 1]);
+    const double S = ds * (double)sub[(n * (K / 32) + g) * 2];
+    const double O = -(dm * (double)sub[(n * (K / 32) + g) * 2 + 1]);
+    return S * (double)rqo_get_ucode4(codes, K, n, k) + O;
+}
+
+/* y[m, n] = sum_k x[m, k] w_hat[n, k] (fp64) and the budget sum |x||w_hat|,
+ * for the P pairs (ms[p], ns[p]) (ms NULL: every output, row-major). */
+void rqo_matmul_fmt(int fmt, const uint16_t *x, int64_t M, int64_t K, const uint8_t *codes,
+                    const void *meta0, const void *meta1, int64_t N, int64_t P, const int64_t *ms,
+                    const int64_t *ns, double *y, double *bound)
+{
+    const int64_t total = ms ? P : M * N;
+    int64_t p;
+#pragma omp parallel for schedule(static)
+    for (p = 0; p < total; p++) {
+        const int64_t m = ms ? ms[p] : p / N, n = ms ? ns[p] : p % N;
+        double acc = 0.0, b = 0.0;
+        int64_t k;
+        for (k = 0; k < K; k++) {
+            double xv = rqo_f16_to_f64(x[m * K + k]);
+            double wv = fmt_weight(fmt, codes, meta0, meta1, K, n, k);
+            acc += xv * wv;
+            b += fabs(xv) * fabs(wv);
+        }
+        y[p] = acc;
+        if (bound) bound[p] = b;
+    }
+}

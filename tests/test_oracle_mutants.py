@@ -18,6 +18,7 @@ import oracle
 from tests import test_oracle_ex2 as ex2
 from tests import test_oracle_gptq as gptq
 from tests import test_oracle_pins as pins
+from tests import test_oracle_presets as presets
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "rqo.c")
 
@@ -65,6 +66,19 @@ MUTANTS = {
     "gptq_no_diag_divide": ("volatile float ev = d / U[j * K + j];", "volatile float ev = d;"),
     # GPTQ: the error spread with the wrong sign
     "gptq_sign": ("w[k] = fmaf(-e, U[j * K + k], w[k]);", "w[k] = fmaf(e, U[j * K + k], w[k]);"),
+    # presets, asymmetric: the group range not widened to include 0
+    "p4a_range_unclamped": ("    float lo = 0.0f, hi = 0.0f;\n    for (i = 0; i < 32; i++) {",
+                            "    float lo = w[0], hi = w[0];\n    for (i = 0; i < 32; i++) {"),
+    # presets, asymmetric: sub-codes truncated instead of rounded
+    "p4a_subcode_floor": ("                    a = rint_clamp(t, 0, 63);",
+                          "                    a = rint_clamp(floorf(t), 0, 63);"),
+    # presets, asymmetric: the offset's sign lost
+    "p4a_offset_sign": ("                volatile float O = -(dmf * (float)b);",
+                        "                volatile float O = (dmf * (float)b);"),
+    # presets, asymmetric: the offset super-scale over 64 steps
+    "p4a_dm_steps": ("            volatile float dm32 = omax / 63.0f;", "            volatile float dm32 = omax / 64.0f;"),
+    # presets, symmetric: every group searched with the first group's E[x^2]
+    "sym_e2_index": ("e2 ? &e2[g * G] : 0", "e2 ? &e2[0] : 0"),
     # GPTQ: every group keeps the first group's scale
     "gptq_scale_once": ("if (j % RQO_GROUP == 0) {\n            /* the group's scale", "if (j == 0) {\n            /* the group's scale"),
 }
@@ -88,6 +102,11 @@ PIN_TESTS = [
     lambda: gptq.test_diagonal_hessian_is_rtn(4),
     lambda: gptq.test_matches_sequential_obs(4),
     gptq.test_hand_worked_rows,
+    lambda: presets.test_sym_g16_matches_restatement(True),
+    lambda: presets.test_p4a_matches_restatement(False),
+    lambda: presets.test_p4a_matches_restatement(True),
+    presets.test_p4a_hand_built_superblock_reproduced,
+    lambda: presets.test_preset_products_match_numpy(4),
     lambda: gptq.test_layer_error_below_rtn(8),
 ]
 
@@ -112,7 +131,8 @@ def test_pins_catch_mutant(name):
         so = _build_mutant(name, old, new, tmp)
         lib = ctypes.CDLL(so)
         for fn in ("rqo_f32_to_f16", "rqo_f16_to_f64", "rqo_quantize_g64", "rqo_quantize_g64_ex2",
-                   "rqo_matmul", "rqo_matmul_sampled", "rqo_get_code", "rqo_gptq_g64"):
+                   "rqo_matmul", "rqo_matmul_sampled", "rqo_get_code", "rqo_gptq_g64",
+                   "rqo_quantize_sym", "rqo_quantize_p4a", "rqo_get_ucode4", "rqo_matmul_fmt"):
             getattr(lib, fn).argtypes = getattr(real, fn).argtypes
             getattr(lib, fn).restype = getattr(real, fn).restype
         caught = False
