@@ -122,6 +122,52 @@ rq_status rq_quantize_g64_ex2(const float *W, int64_t N, int64_t K, int bits, co
                               int32_t *chosen, int *dev_status, rq_stream_t stream);
 
 /*
+ * The two preset formats of "rwkv-quant: uma matriz em bf16 elimina 39% das
+ * perdas na quantização do RWKV-7 2.9B" ("Dois presets e seis tamanhos"):
+ * REDUCTION stores projections in 8 bits, symmetric, groups of 16 weights;
+ * COMPRESSION in 4 bits, asymmetric, in super-blocks, groups of 32; in both
+ * the groups' scale (and offset) is chosen by a search weighted by E[x^2].
+ * Where the article is silent, this library reads (and its oracle follows):
+ *
+ * rq_quantize_p8_g16 -- int8 symmetric, groups of 16 consecutive k: per group
+ *   amax; candidate j: s16 = fp16_rn(fp32(amax * factors[j]) / 127), codes
+ *   clamp(rint(w / s16), +-127) (IEEE fp32 division, ties to even), error
+ *   sum_k e2[k] (w - c s16)^2 in k order (each operation one fp32 rounding);
+ *   the smallest error wins, the earlier candidate on a tie; a candidate whose
+ *   scale overflows is never chosen (all overflow: RTN).  e2 NULL: RTN (one
+ *   candidate, factor 1).  codes int8 [N, K]; scales fp16 [N, K/16]; chosen
+ *   (nullable) int32 [N, K/16].
+ *
+ * rq_quantize_p4a_g32 -- int4 asymmetric, groups of 32 in super-blocks of 8
+ *   groups (256 k).  Per group: lo = min(0, min w), hi = max(0, max w);
+ *   candidate j: lo_j = lo f_j, hi_j = hi f_j, s_j = (hi_j - lo_j) / 15, codes
+ *   clamp(rint((w - lo_j) / s_j), 0, 15), error sum e2 (w - (q s_j + lo_j))^2;
+ *   the chosen group's (s, o = lo_j).  Per super-block: ds =
+ *   fp16_rn(max s / 63), dm = fp16_rn(max(-o) / 63); per group 6-bit
+ *   sub-codes a = clamp(rint(s / ds), 0, 63), b = clamp(rint(-o / dm), 0, 63);
+ *   stored scale S = ds a and offset O = -(dm b); codes q = clamp(rint((w - O) /
+ *   S), 0, 15); w_hat = S q + O.  Layout: codes uint8 [N, K/2], unsigned
+ *   nibbles, k = 2j in the low nibble of byte j; sub uint8 [N, K/32, 2] = (a,
+ *   b); sup fp16 [N, K/256, 2] = (ds, dm); chosen (nullable) int32 [N, K/32].
+ *   K % 256 == 0.  A super-block holding a non-finite weight: ds = dm =
+ *   0x7E00, sub-codes and codes 0; an overflowing ds or dm: kept (+inf),
+ *   sub-codes and codes 0.
+ *
+ * Both: W fp32 [N, K] device, 16-byte aligned; e2 fp32 [K] (E[x^2] per input
+ * channel, >= 0) or NULL; factors fp32 [nf], 1 <= nf <= 16 (else
+ * RQ_ERR_RANGE), read only with e2; dev_status as rq_quantize_g64
+ * (RQ_ERR_NONFINITE over RQ_ERR_RANGE).  Every operation is one IEEE fp32
+ * rounding in the order stated, so results are reproducible bit for bit.
+ */
+rq_status rq_quantize_p8_g16(const float *W, int64_t N, int64_t K, const float *e2,
+                             const float *factors, int nf, void *codes, uint16_t *scales,
+                             int32_t *chosen, int *dev_status, rq_stream_t stream);
+rq_status rq_quantize_p4a_g32(const float *W, int64_t N, int64_t K, const float *e2,
+                              const float *factors, int nf, void *codes, uint8_t *sub,
+                              uint16_t *sup, int32_t *chosen, int *dev_status,
+                              rq_stream_t stream);
+
+/*
  * GPTQ on the same group-64 grid -- the "GPTQ-calibrated, symmetric, group
  * 64" int4 of the "Hakureirm/rwkv7-sglang-w4gptq-1.5b" model card (opening
  * summary), run "on the preset's grid without changing the format or the

@@ -694,6 +694,7 @@ static void p4a_group_choice(const float *w, const float *e2, const float *f, in
 int rqo_quantize_p4a(const float *W, int64_t N, int64_t K, const float *e2, const float *f, int nf,
                      uint8_t *codes, uint8_t *sub, uint16_t *sup, int32_t *chosen)
 {
+    /* statuses as rqo_quantize_g64: NONFINITE over RANGE over OK */
     const int64_t NSB = K / 256, NG = K / 32;
     int status = RQO_OK;
     int64_t n;
@@ -761,6 +762,10 @@ int rqo_quantize_p4a(const float *W, int64_t N, int64_t K, const float *e2, cons
                 }
             }
         }
+    }
+    if (status != RQO_OK) {
+        int64_t i, total = N * NSB * 2;
+        for (i = 0; i < total; i++) if (sup[i] == 0x7E00u) return RQO_ERR_NONFINITE;
     }
     return status;
 }

@@ -257,6 +257,45 @@ rq_status rq_quantize_g64_ex2(const float* W, int64_t N, int64_t K, int bits, co
     return e == cudaSuccess ? RQ_OK : cuda_fail(e);
 }
 
+static rq_status check_search(const float* e2, const float* factors, int nf) {
+    if (e2 == nullptr) return RQ_OK;
+    if (nf < 1 || nf > 16) return RQ_ERR_RANGE;
+    if (factors == nullptr) return RQ_ERR_NULL;
+    if (!aligned16(e2) || (reinterpret_cast<uintptr_t>(factors) & 3u)) return RQ_ERR_ALIGN;
+    return RQ_OK;
+}
+
+rq_status rq_quantize_p8_g16(const float* W, int64_t N, int64_t K, const float* e2,
+                             const float* factors, int nf, void* codes, uint16_t* scales,
+                             int32_t* chosen, int* dev_status, rq_stream_t stream) {
+    rq_status st = check_weight_shape(N, K, 8);
+    if (st != RQ_OK) return st;
+    if ((st = check_search(e2, factors, nf)) != RQ_OK) return st;
+    if (W == nullptr || codes == nullptr || scales == nullptr) return RQ_ERR_NULL;
+    if (!aligned16(W) || !aligned16(codes) || !aligned16(scales)) return RQ_ERR_ALIGN;
+    const auto mis4 = [](const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u); };
+    if (mis4(chosen) || mis4(dev_status)) return RQ_ERR_ALIGN;
+    const cudaError_t e = launch_quantize_p8(W, N, K, e2, factors, nf, codes, scales, chosen, dev_status,
+                                             reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+rq_status rq_quantize_p4a_g32(const float* W, int64_t N, int64_t K, const float* e2,
+                              const float* factors, int nf, void* codes, uint8_t* sub, uint16_t* sup,
+                              int32_t* chosen, int* dev_status, rq_stream_t stream) {
+    rq_status st = check_weight_shape(N, K, 4);
+    if (st != RQ_OK) return st;
+    if (K % 256 != 0) return RQ_ERR_SHAPE;
+    if ((st = check_search(e2, factors, nf)) != RQ_OK) return st;
+    if (W == nullptr || codes == nullptr || sub == nullptr || sup == nullptr) return RQ_ERR_NULL;
+    if (!aligned16(W) || !aligned16(codes) || !aligned16(sub) || !aligned16(sup)) return RQ_ERR_ALIGN;
+    const auto mis4 = [](const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u); };
+    if (mis4(chosen) || mis4(dev_status)) return RQ_ERR_ALIGN;
+    const cudaError_t e = launch_quantize_p4a(W, N, K, e2, factors, nf, codes, sub, sup, chosen, dev_status,
+                                              reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
 rq_status rq_gptq_hessian(const uint16_t* X, int64_t T, int64_t K, double* H, rq_stream_t stream) {
     if (K < kGroup || K % kGroup != 0 || K > (int64_t{1} << 16) || T < 1 || T > (int64_t{1} << 31))
         return RQ_ERR_SHAPE;

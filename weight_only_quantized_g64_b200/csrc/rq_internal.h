@@ -94,6 +94,17 @@ cudaError_t launch_gptq_quantize(float* W, int64_t N, int64_t K, int bits, const
                                  const uint8_t* dead, void* codes, uint16_t* scales, float* work,
                                  int* dev_status, cudaStream_t s);
 
+// Quantizers of the rwkv-quant preset formats: symmetric int8 with groups of
+// 16 (scales fp16 [N, K/16]); asymmetric int4 with groups of 32 in
+// super-blocks of 8 (sub uint8 [N, K/32, 2], sup fp16 [N, K/256, 2]).
+// e2 NULL: no search (RTN).
+cudaError_t launch_quantize_p8(const float* W, int64_t N, int64_t K, const float* e2,
+                               const float* factors, int nf, void* codes, uint16_t* scales,
+                               int32_t* chosen, int* dev_status, cudaStream_t s);
+cudaError_t launch_quantize_p4a(const float* W, int64_t N, int64_t K, const float* e2,
+                                const float* factors, int nf, void* codes, uint8_t* sub, uint16_t* sup,
+                                int32_t* chosen, int* dev_status, cudaStream_t s);
+
 // Bounded-wait self test: a kernel waits on an mbarrier nothing completes.
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s);
 

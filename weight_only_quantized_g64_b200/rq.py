@@ -72,6 +72,10 @@ def lib():
     L.rq_gemv_wq_ex.restype = i32
     L.rq_rkv_fused3.argtypes = [vp, vp, vp, i64, i64, i64, i32] + [vp] * 9 + [i32, vp]
     L.rq_rkv_fused3.restype = i32
+    L.rq_quantize_p8_g16.argtypes = [vp, i64, i64, vp, vp, i32, vp, vp, vp, vp, vp]
+    L.rq_quantize_p8_g16.restype = i32
+    L.rq_quantize_p4a_g32.argtypes = [vp, i64, i64, vp, vp, i32, vp, vp, vp, vp, vp, vp]
+    L.rq_quantize_p4a_g32.restype = i32
     L.rq_set_pdl.argtypes = [i32]
     L.rq_set_pdl.restype = i32
     L.rq_set_decode_kernel.argtypes = [i32]
@@ -155,6 +159,33 @@ def quantize_g64_ex2(W: torch.Tensor, e2: torch.Tensor, bits: int, factors: torc
                                      _p(codes), _p(scales), _p(chosen), _p(dev_status),
                                      _stream(stream)), "rq_quantize_g64_ex2")
     return codes, scales, chosen
+
+
+def quantize_p8_g16(W: torch.Tensor, e2=None, factors=None, dev_status=None, stream=None):
+    """Preset int8 symmetric groups of 16 -> (codes int8-as-uint8 [N, K],
+    scales int16 [N, K/16], chosen int32 [N, K/16])."""
+    N, K = W.shape
+    codes = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N, K // 16), dtype=torch.int16, device=W.device)
+    chosen = torch.empty((N, K // 16), dtype=torch.int32, device=W.device)
+    nf = 0 if factors is None else int(factors.numel())
+    _check(lib().rq_quantize_p8_g16(_p(W), N, K, _p(e2), _p(factors), nf, _p(codes), _p(scales),
+                                    _p(chosen), _p(dev_status), _stream(stream)), "rq_quantize_p8_g16")
+    return codes, scales, chosen
+
+
+def quantize_p4a_g32(W: torch.Tensor, e2=None, factors=None, dev_status=None, stream=None):
+    """Preset int4 asymmetric groups of 32 in super-blocks -> (codes uint8
+    [N, K/2], sub uint8 [N, K/32, 2], sup int16 [N, K/256, 2], chosen int32 [N, K/32])."""
+    N, K = W.shape
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    sub = torch.empty((N, K // 32, 2), dtype=torch.uint8, device=W.device)
+    sup = torch.empty((N, K // 256, 2), dtype=torch.int16, device=W.device)
+    chosen = torch.empty((N, K // 32), dtype=torch.int32, device=W.device)
+    nf = 0 if factors is None else int(factors.numel())
+    _check(lib().rq_quantize_p4a_g32(_p(W), N, K, _p(e2), _p(factors), nf, _p(codes), _p(sub), _p(sup),
+                                     _p(chosen), _p(dev_status), _stream(stream)), "rq_quantize_p4a_g32")
+    return codes, sub, sup, chosen
 
 
 def gptq_hessian(X: torch.Tensor, H=None, stream=None):
