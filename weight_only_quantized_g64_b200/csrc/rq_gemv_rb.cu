@@ -86,6 +86,7 @@ struct RbParams {
     uint64_t timeout_ns;
 };
 
+constexpr int kRbSrow = 40;                     // fp16 scales per staged row (J <= 32, + slack)
 constexpr int kRbWarps = 8;                     // warps, all computing
 constexpr int kRbThreads = kRbWarps * 32;
 constexpr int kRbMaxSG = 8;
@@ -129,23 +130,21 @@ __device__ __forceinline__ void i8_word_biased(uint32_t w, uint32_t (&Q)[2]) {
 // Group columns of one warp (NC of them, processed together for independent
 // dependency chains): every m-tile of the block (MT of them) times the x of
 // the column's group, for NT 8-token tiles.  Per column c:
-//   cw0[c] codes of the column's stage, m-tile 0, this thread's physical row
-//          and chunk (rows 16i + prow and +8 of m-tile i are 16*128*i and
-//          8*128 further)
-//   sp[c]  scales: (row 16i + 8h + prow, this group) at sp[c][(16i + 8h) * srow]
-//   xg[c]  x of the group: token rows of 128 B (swizzled); xl[c][nt] the row
-//          of token nt*8+g
-//   grp[c] the group (for scales read from global memory when !ssc)
-// The four MMA steps of a group run as two independent 2-step chains and the
-// bias term as a third chain; the three are added before the scale, in a
-// fixed order.
-template <int BITS, int MT, int NT, int NC>
+//   cw0[c]  codes of the column's stage, m-tile 0, this thread's physical row
+//           and chunk (rows 16i + prow and +8 of m-tile i are 16*128*i and
+//           8*128 further)
+//   sp[c]   scales: (row 16i + 8h + prow, this group) at sp[c][(16i + 8h) * kRbSrow]
+//   xrow    byte offsets (from xbase) of the 128-byte x rows of the column's
+//           group for the tokens nt*8+g; xph[nt] their swizzle phase
+//   grp[c]  the group (for scales read from global memory when !SSC)
+// The group's four MMA steps run as one chain that starts from the bias term
+// (so no additions are needed), and the scale is applied with one fma.
+template <int BITS, int MT, int NT, int NC, bool SSC>
 __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
-                                           const uint16_t* const (&sp)[NC], int srow,
-                                           const uint8_t* const (&xg)[NC], const int (&xl)[NC][NT],
-                                           int t, float (&acc)[MT][NT][4], bool ssc,
-                                           const uint16_t* gscales, int64_t grow0, int groups,
-                                           const int (&grp)[NC], int N) {
+                                           const uint16_t* const (&sp)[NC], const uint8_t* xbase,
+                                           const int (&xrow)[NC][NT], const int (&xph)[NT], int t,
+                                           float (&acc)[MT][NT][4], const uint16_t* gscales,
+                                           int64_t grow0, int groups, const int (&grp)[NC], int N) {
     constexpr int CW = BITS == 4 ? 2 : 4;   // code words per row and group
     // ---- x fragments: token nt*8+g, positions 16t .. 16t+15 of the group
     uint32_t b[NC][NT][4][2];
@@ -153,11 +152,10 @@ __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
     for (int c = 0; c < NC; ++c)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const int line = xl[c][nt];
-            const uint8_t* xr = xg[c] + line * 128;
-            const int ph = line & 7;
-            const uint4 v0 = lds128(xr + (((2 * t) ^ ph) << 4));
-            const uint4 v1 = lds128(xr + (((2 * t + 1) ^ ph) << 4));
+            const uint8_t* xr = xbase + xrow[c][nt];
+            const int c0 = ((2 * t) ^ xph[nt]) << 4;
+            const uint4 v0 = lds128(xr + c0);
+            const uint4 v1 = lds128(xr + (c0 ^ 16));
             const uint32_t X[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
@@ -173,7 +171,7 @@ __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
             }
         }
     // ---- -sum_k bias_k x_k of each column's group, per token tile (the same
-    // for every row): two 2-step chains
+    // for every row)
     float negc[NC][NT][4];
     {
         uint32_t an[4];
@@ -187,13 +185,10 @@ __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
         for (int c = 0; c < NC; ++c)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                float h0[4], h1[4];
-                mma16816(h0, an, b[c][nt][0][0], b[c][nt][0][1], true);
-                mma16816(h1, an, b[c][nt][2][0], b[c][nt][2][1], true);
-                mma16816(h0, an, b[c][nt][1][0], b[c][nt][1][1], false);
-                mma16816(h1, an, b[c][nt][3][0], b[c][nt][3][1], false);
+                mma16816(negc[c][nt], an, b[c][nt][0][0], b[c][nt][0][1], true);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) negc[c][nt][e] = h0[e] + h1[e];
+                for (int jj = 1; jj < 4; ++jj)
+                    mma16816(negc[c][nt], an, b[c][nt][jj][0], b[c][nt][jj][1], false);
             }
     }
     // ---- every m-tile
@@ -218,8 +213,8 @@ __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint16_t s16;
-                if (ssc) {
-                    s16 = sp[c][(16 * i + 8 * h) * srow];
+                if constexpr (SSC) {
+                    s16 = sp[c][(16 * i + 8 * h) * kRbSrow];
                 } else {
                     const int64_t n = grow0 + 16 * i + 8 * h;
                     s16 = (n < N && grp[c] < groups) ? __ldg(gscales + n * groups + grp[c])
@@ -250,25 +245,25 @@ __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
             }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                float p0[4], p1[4];
-                mma16816(p0, A[0], b[c][nt][0][0], b[c][nt][0][1], true);
-                mma16816(p1, A[2], b[c][nt][2][0], b[c][nt][2][1], true);
-                mma16816(p0, A[1], b[c][nt][1][0], b[c][nt][1][1], false);
-                mma16816(p1, A[3], b[c][nt][3][0], b[c][nt][3][1], false);
+                float part[4];
+                mma16816_c(part, A[0], b[c][nt][0][0], b[c][nt][0][1], negc[c][nt]);
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    acc[i][nt][e] = fmaf((p0[e] + p1[e]) + negc[c][nt][e], sv[e >> 1], acc[i][nt][e]);
+                for (int jj = 1; jj < 4; ++jj) mma16816(part, A[jj], b[c][nt][jj][0], b[c][nt][jj][1], false);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[i][nt][e] = fmaf(part[e], sv[e >> 1], acc[i][nt][e]);
             }
         }
     }
 }
 
-template <int BITS, int MT, int NT>
+template <int BITS, int MT, int NT, bool SSC>
 __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_constant__ RbParams p) {
     constexpr int GPS = BITS == 4 ? 4 : 2;      // groups per 128-byte stage
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned start, reached by an offset from the shared array
+    // itself so every access below stays a shared-memory access
+    const uint32_t s0 = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
+    uint8_t* smem = smem_raw + ((1024u - (s0 & 1023u)) & 1023u);
     uint8_t* ring = smem;
     RbBars* bars = reinterpret_cast<RbBars*>(smem + p.bar_off);
     volatile int* abort_flag = &bars->abort;
@@ -278,7 +273,7 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
     const int RB = 16 * MT;                     // rows of a block (== 16 * p.tc)
     const int cbytes = RB * 128 * p.S;          // code bytes of a slot
     const uint32_t x_bytes = static_cast<uint32_t>(p.J * p.M * 128);
-    const uint32_t s_bytes = p.ssc ? static_cast<uint32_t>(RB * p.srow * 2) : 0u;
+    const uint32_t s_bytes = SSC ? static_cast<uint32_t>(RB * kRbSrow * 2) : 0u;
 
     // Loads of the CTA's slot i (block blk, slot sl of the block) into ring slot r.
     auto issue_w = [&](int r, int blk, int sl) {
@@ -294,7 +289,7 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
             for (int s = 0; s < p.S; ++s)
                 tma_load_2d(dst + s * RB * 128, &p.tm_w[m], &bars->full[r], (st0 + s) * 128, row0, pol);
         }
-        if (p.ssc)
+        if constexpr (SSC)
             tma_load_2d(dst + p.s_off, &p.tm_s[m], &bars->full[r], (st0 * GPS) & ~7, row0, pol);
     };
     auto issue_x = [&](int r, int blk, int sl) {
@@ -315,7 +310,7 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
             if (p.y[m] == nullptr) break;
             if (m < p.nx) tma_prefetch_desc(&p.tm_x[m]);
             tma_prefetch_desc(&p.tm_w[m]);
-            if (p.ssc) tma_prefetch_desc(&p.tm_s[m]);
+            if (SSC) tma_prefetch_desc(&p.tm_s[m]);
         }
         // codes and scales of the first block's first slots: they never
         // depend on the previous grid, so they go out before waiting on it
@@ -336,7 +331,29 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
     const int g = lane >> 2;
     const int t = lane & 3;
     const int prow = phys_row<BITS>(g);
+    // This warp's columns of a slot are j = warp + 8c: for int4 stage
+    // warp/4 + 2c, group warp%4 of it; for int8 stage warp/2 + 4c, group
+    // warp%2.  Every per-column offset below is a constant plus c strides.
+    constexpr int CPS = kRbWarps / GPS;                 // stages between a warp's columns
+    const int q0 = warp % GPS;
+    int coff;
+    if constexpr (BITS == 4)
+        coff = prow * 128 + (((2 * q0 + (t >> 1)) ^ (prow & 7)) << 4) + ((t & 1) << 3);
+    else
+        coff = prow * 128 + (((4 * q0 + t) ^ (prow & 7)) << 4);
+    const int code0 = (warp / GPS) * RB * 128 + coff;   // the warp's first column in a slot
+    const int code_step = CPS * RB * 128;
+    int xrow0[NT], xph[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int line = warp * p.M + min(nt * 8 + g, p.M - 1);
+        xrow0[nt] = p.x_off + line * 128;
+        xph[nt] = line & 7;                             // unchanged by the 8*M-line column stride
+    }
+    const int x_step = kRbWarps * p.M * 128;
     int gi = 0;                 // the CTA's slot index (over all its blocks)
+    int r = 0;                  // its ring slot (gi % SG) and that slot's phase
+    uint32_t ph = 0;
     bool dead = false;
     int kb = 0;                 // blocks done by this CTA
     for (int blk = blockIdx.x; blk < p.nblocks; blk += gridDim.x, ++kb) {
@@ -346,11 +363,12 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
             // a later block: the ring was the previous block's reduction
             // buffer, so its first slots go out only now
             const int n_pre = min(SG, p.slots);
+            int rq = r;
             for (int q = 0; q < n_pre; ++q) {
-                const int r = (gi + q) % SG;
-                bars->issued_hi[r] = gi + q;
-                issue_w(r, blk, q);
-                issue_x(r, blk, q);
+                bars->issued_hi[rq] = gi + q;
+                issue_w(rq, blk, q);
+                issue_x(rq, blk, q);
+                if (++rq == SG) rq = 0;
             }
         }
         float acc[MT][NT][4];
@@ -361,54 +379,42 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[i][nt][e] = 0.0f;
         for (int sl = 0; sl < p.slots; ++sl, ++gi) {
-            const int r = gi % SG;
-            if (!dead && !mbar_wait(&bars->full[r], static_cast<uint32_t>(gi / SG) & 1, abort_flag,
-                                    p.timeout_ns, p.status))
+            if (!dead && !mbar_wait(&bars->full[r], ph, abort_flag, p.timeout_ns, p.status))
                 dead = true;
             const int grp0 = sl * p.J;                  // first group of the slot
             int jn = p.groups - grp0;                   // group columns holding data
             if (jn > p.J) jn = p.J;
             if (!dead) {
                 const uint8_t* base = ring + r * p.slot_bytes;
-                // this warp's columns j = warp, warp + 8, ...: two at a time
-                auto col = [&](int j, const uint8_t*& cw0, const uint16_t*& sp, int (&xl)[NT]) {
-                    const int s = j / GPS;
-                    const int q = j - s * GPS;
-                    int coff;
-                    if constexpr (BITS == 4)
-                        coff = prow * 128 + (((2 * q + (t >> 1)) ^ (prow & 7)) << 4) + ((t & 1) << 3);
-                    else
-                        coff = prow * 128 + (((4 * q + t) ^ (prow & 7)) << 4);
-                    cw0 = base + s * RB * 128 + coff;
-                    sp = reinterpret_cast<const uint16_t*>(base + p.s_off) + prow * p.srow +
-                         ((grp0 & 7) + j);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) xl[nt] = j * p.M + min(nt * 8 + g, p.M - 1);
-                };
-                int j = warp;
+                const uint8_t* cbase = base + code0;
+                const uint16_t* sbase = reinterpret_cast<const uint16_t*>(base + p.s_off) +
+                                        prow * kRbSrow + (grp0 & 7) + warp;
+                int c = 0;
                 // (pairs only for one token tile: larger M takes one column
                 // per warp and slot, and the registers go to its tiles)
                 if constexpr (NT == 1)
-                for (; j + kRbWarps < jn; j += 2 * kRbWarps) {
-                    const uint8_t* cw0[2];
-                    const uint16_t* sp[2];
-                    int xl[2][NT];
-                    col(j, cw0[0], sp[0], xl[0]);
-                    col(j + kRbWarps, cw0[1], sp[1], xl[1]);
-                    const uint8_t* xg[2] = {base + p.x_off, base + p.x_off};
-                    const int gr[2] = {grp0 + j, grp0 + j + kRbWarps};
-                    rb_columns<BITS, MT, NT, 2>(cw0, sp, p.srow, xg, xl, t, acc, p.ssc != 0,
-                                                p.scales[m], row0 + prow, p.groups, gr, p.N);
+                for (; warp + kRbWarps * (c + 1) < jn; c += 2) {
+                    const uint8_t* cw0[2] = {cbase + c * code_step, cbase + (c + 1) * code_step};
+                    const uint16_t* sp[2] = {sbase + kRbWarps * c, sbase + kRbWarps * (c + 1)};
+                    int xr[2][NT];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        xr[0][nt] = xrow0[nt] + c * x_step;
+                        xr[1][nt] = xrow0[nt] + (c + 1) * x_step;
+                    }
+                    const int gr[2] = {grp0 + warp + kRbWarps * c, grp0 + warp + kRbWarps * (c + 1)};
+                    rb_columns<BITS, MT, NT, 2, SSC>(cw0, sp, base, xr, xph, t, acc, p.scales[m],
+                                                     row0 + prow, p.groups, gr, p.N);
                 }
-                for (; j < jn; j += kRbWarps) {
-                    const uint8_t* cw0[1];
-                    const uint16_t* sp[1];
-                    int xl[1][NT];
-                    col(j, cw0[0], sp[0], xl[0]);
-                    const uint8_t* xg[1] = {base + p.x_off};
-                    const int gr[1] = {grp0 + j};
-                    rb_columns<BITS, MT, NT, 1>(cw0, sp, p.srow, xg, xl, t, acc, p.ssc != 0,
-                                                p.scales[m], row0 + prow, p.groups, gr, p.N);
+                for (; warp + kRbWarps * c < jn; ++c) {
+                    const uint8_t* cw0[1] = {cbase + c * code_step};
+                    const uint16_t* sp[1] = {sbase + kRbWarps * c};
+                    int xr[1][NT];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) xr[0][nt] = xrow0[nt] + c * x_step;
+                    const int gr[1] = {grp0 + warp + kRbWarps * c};
+                    rb_columns<BITS, MT, NT, 1, SSC>(cw0, sp, base, xr, xph, t, acc, p.scales[m],
+                                                     row0 + prow, p.groups, gr, p.N);
                 }
             }
             // ---- release the slot; the last warp out refills it with the
@@ -430,6 +436,10 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
                         issue_x(r, blk, nsl);
                     }
                 }
+            }
+            if (++r == SG) {
+                r = 0;
+                ph ^= 1u;
             }
         }
         // ---- the block's sums: warps deposit, then add in warp order
@@ -545,7 +555,7 @@ static bool rb_plan(int64_t M, int64_t K, int64_t N, int bits, int nmat, RbPlan*
     P->S = S;
     P->J = S * GPS;
     P->slots = (P->stages + S - 1) / S;
-    P->srow = rb_align(P->J + 8, 8);
+    P->srow = kRbSrow;
     const int cbytes = RB * 128 * S;
     P->s_off = cbytes;
     P->x_off = rb_align(P->s_off + RB * P->srow * 2, 1024);
@@ -575,10 +585,10 @@ bool gemv_rowblock_fits(int64_t M, int64_t K, int64_t N, int bits, int nmat) {
     return rb_plan(M, K, N, bits, nmat, &P);
 }
 
-template <int BITS, int MT, int NT>
+template <int BITS, int MT, int NT, bool SSC>
 static cudaError_t rb_launch(RbParams& prm, const RbPlan& P, const uint16_t* const* xs,
                              const void* const* codes, int nmat, cudaStream_t s) {
-    auto kern = gemv_rb_kernel<BITS, MT, NT>;
+    auto kern = gemv_rb_kernel<BITS, MT, NT, SSC>;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -633,19 +643,26 @@ static cudaError_t rb_launch(RbParams& prm, const RbPlan& P, const uint16_t* con
     return cudaLaunchKernelEx(&cfg, kern, static_cast<const RbParams&>(prm));
 }
 
-template <int BITS, int NT>
+template <int BITS, int NT, bool SSC>
 static cudaError_t rb_dispatch_mt(RbParams& prm, const RbPlan& P, const uint16_t* const* x,
                                   const void* const* codes, int nmat, cudaStream_t s) {
     switch (P.tc) {
-        case 1: return rb_launch<BITS, 1, NT>(prm, P, x, codes, nmat, s);
-        case 2: return rb_launch<BITS, 2, NT>(prm, P, x, codes, nmat, s);
-        case 3: return rb_launch<BITS, 3, NT>(prm, P, x, codes, nmat, s);
-        case 4: return rb_launch<BITS, 4, NT>(prm, P, x, codes, nmat, s);
-        case 5: return rb_launch<BITS, 5, NT>(prm, P, x, codes, nmat, s);
-        case 6: return rb_launch<BITS, 6, NT>(prm, P, x, codes, nmat, s);
-        case 7: return rb_launch<BITS, 7, NT>(prm, P, x, codes, nmat, s);
-        default: return rb_launch<BITS, 8, NT>(prm, P, x, codes, nmat, s);
+        case 1: return rb_launch<BITS, 1, NT, SSC>(prm, P, x, codes, nmat, s);
+        case 2: return rb_launch<BITS, 2, NT, SSC>(prm, P, x, codes, nmat, s);
+        case 3: return rb_launch<BITS, 3, NT, SSC>(prm, P, x, codes, nmat, s);
+        case 4: return rb_launch<BITS, 4, NT, SSC>(prm, P, x, codes, nmat, s);
+        case 5: return rb_launch<BITS, 5, NT, SSC>(prm, P, x, codes, nmat, s);
+        case 6: return rb_launch<BITS, 6, NT, SSC>(prm, P, x, codes, nmat, s);
+        case 7: return rb_launch<BITS, 7, NT, SSC>(prm, P, x, codes, nmat, s);
+        default: return rb_launch<BITS, 8, NT, SSC>(prm, P, x, codes, nmat, s);
     }
+}
+
+template <int BITS, int NT>
+static cudaError_t rb_dispatch_ssc(RbParams& prm, const RbPlan& P, const uint16_t* const* x,
+                                   const void* const* codes, int nmat, cudaStream_t s) {
+    return prm.ssc ? rb_dispatch_mt<BITS, NT, true>(prm, P, x, codes, nmat, s)
+                   : rb_dispatch_mt<BITS, NT, false>(prm, P, x, codes, nmat, s);
 }
 
 cudaError_t launch_gemv_rowblock(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
@@ -694,12 +711,12 @@ cudaError_t launch_gemv_rowblock_ex(const uint16_t* const* xs, int nx, int64_t M
         prm.y[i] = w[i].y;
     }
     if (bits == 4)
-        return M <= 8    ? rb_dispatch_mt<4, 1>(prm, P, x, codes, nmat, s)
-               : M <= 16 ? rb_dispatch_mt<4, 2>(prm, P, x, codes, nmat, s)
-                         : rb_dispatch_mt<4, 4>(prm, P, x, codes, nmat, s);
-    return M <= 8    ? rb_dispatch_mt<8, 1>(prm, P, x, codes, nmat, s)
-           : M <= 16 ? rb_dispatch_mt<8, 2>(prm, P, x, codes, nmat, s)
-                     : rb_dispatch_mt<8, 4>(prm, P, x, codes, nmat, s);
+        return M <= 8    ? rb_dispatch_ssc<4, 1>(prm, P, x, codes, nmat, s)
+               : M <= 16 ? rb_dispatch_ssc<4, 2>(prm, P, x, codes, nmat, s)
+                         : rb_dispatch_ssc<4, 4>(prm, P, x, codes, nmat, s);
+    return M <= 8    ? rb_dispatch_ssc<8, 1>(prm, P, x, codes, nmat, s)
+           : M <= 16 ? rb_dispatch_ssc<8, 2>(prm, P, x, codes, nmat, s)
+                     : rb_dispatch_ssc<8, 4>(prm, P, x, codes, nmat, s);
 }
 
 }  // namespace rq
