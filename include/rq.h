@@ -168,6 +168,31 @@ rq_status rq_quantize_p4a_g32(const float *W, int64_t N, int64_t K, const float 
                               rq_stream_t stream);
 
 /*
+ * Decode products of the two preset formats (the formats above, as their
+ * quantizers write them): y[M, N] = x[M, K] W_hat^T with
+ *
+ * rq_gemv_p8_g16  -- W_hat[n, k] = codes[n, k] * scales[n, k / 16];
+ * rq_gemv_p4a_g32 -- W_hat[n, k] = S q + O, q the unsigned nibble of k,
+ *   S = ds a and O = -(dm b) with (a, b) = sub[n, k / 32] and (ds, dm) =
+ *   sup[n, k / 256], each product one fp32 rounding.
+ *
+ * Each group's sum x * codes is exact in fp32 before its scale (and, for the
+ * asymmetric format, its offset times the group's sum of x) is applied in
+ * fp32; groups are added in an order fixed per shape, so results are
+ * deterministic.  x fp16 [M, K] row-major, 1 <= M <= 32 (else RQ_ERR_SHAPE);
+ * y fp32 [M, N].  K % 128 == 0 (int8 preset) or K % 256 == 0 (int4 preset),
+ * else RQ_ERR_SHAPE; x, codes, scales / sub, sup and y 16-byte aligned (else
+ * RQ_ERR_ALIGN); NULL pointers: RQ_ERR_NULL.  Non-finite scales or x give
+ * non-finite outputs.  Same kernel, data path and wait bound as the row-block
+ * decode kernel of rq_gemv_wq; needs no workspace; asynchronous on `stream`.
+ */
+rq_status rq_gemv_p8_g16(const uint16_t *x, int64_t M, int64_t K, const void *codes,
+                         const uint16_t *scales, int64_t N, float *y, rq_stream_t stream);
+rq_status rq_gemv_p4a_g32(const uint16_t *x, int64_t M, int64_t K, const void *codes,
+                          const uint8_t *sub, const uint16_t *sup, int64_t N, float *y,
+                          rq_stream_t stream);
+
+/*
  * GPTQ on the same group-64 grid -- the "GPTQ-calibrated, symmetric, group
  * 64" int4 of the "Hakureirm/rwkv7-sglang-w4gptq-1.5b" model card (opening
  * summary), run "on the preset's grid without changing the format or the

@@ -104,24 +104,27 @@ def test_control_calls(L):
 
 
 def test_decode_kernel_choice(L):
-    """The automatic choice between the decode kernels (host logic, no GPU):
-    row tiles for M <= 8; the cluster kernel for M > 16; for 9 <= M <= 16
-    the cluster kernel on launches of >= 6144 rows with K <= 4096 (the fused
-    R/K/V and channel-mix key of the 1.5B-shaped layer), row tiles otherwise."""
+    """The automatic choice between the decode kernels (host logic, no GPU,
+    so the SM count is taken as 148): the row-block kernel at every M for
+    launches of at least one 16-row m-tile per SM (the fused R/K/V and the
+    channel-mix key of the 1.5B-shaped layer); below that the row-tile kernel
+    for M <= 16 and the cluster kernel for M > 16."""
     D = 2048
     layer = {"rkv": (D, D, 3), "o": (D, D, 1), "key": (4 * D, D, 1), "value": (D, 4 * D, 1)}
-    for M in (1, 4, 8):
-        for name, (N, K, nmat) in layer.items():
-            assert rq.decode_kernel_for(M, K, N, 4, nmat) == "rowtile", (M, name)
-    for M in (17, 24, 32):
-        for name, (N, K, nmat) in layer.items():
-            assert rq.decode_kernel_for(M, K, N, 4, nmat) == "cluster", (M, name)
-    for M in (9, 16):
-        assert rq.decode_kernel_for(M, D, D, 4, 3) == "cluster"
-        assert rq.decode_kernel_for(M, D, 4 * D, 4, 1) == "cluster"
-        assert rq.decode_kernel_for(M, D, D, 4, 1) == "rowtile"
-        assert rq.decode_kernel_for(M, 4 * D, D, 4, 1) == "rowtile"
-        assert rq.decode_kernel_for(M, 16384, 16384, 4, 1) == "rowtile"   # K > 4096
+    for M in (1, 4, 8, 9, 16, 17, 24, 32):
+        for name in ("rkv", "key"):
+            N, K, nmat = layer[name]
+            assert rq.decode_kernel_for(M, K, N, 4, nmat) == "rowblock", (M, name)
+            assert rq.decode_kernel_for(M, K, N, 8, nmat) == "rowblock", (M, name)
+        for name in ("o", "value"):
+            N, K, nmat = layer[name]
+            want = "rowtile" if M <= 16 else "cluster"
+            assert rq.decode_kernel_for(M, K, N, 4, nmat) == want, (M, name)
+    # the boundary: 148 m-tiles (2368 rows) in the launch
+    assert rq.decode_kernel_for(1, D, 2368, 4, 1) == "rowblock"
+    assert rq.decode_kernel_for(1, D, 2352, 4, 1) == "rowtile"
+    assert rq.decode_kernel_for(1, 16384, 16384, 4, 1) == "rowblock"
+    assert rq.decode_kernel_for(32, 16384, 16384, 4, 1) == "rowblock"
     # a selection overrides the automatic choice
     for kind in ("rowtile", "cluster"):
         with rq.decode_kernel(kind):
@@ -185,6 +188,29 @@ def test_decode_variant_argument_errors(L):
     assert f(p, p, odd, 1, 128, 64, 4, p, p, p, p, p, p, p, p, p, 0, None) == rq.ERR_ALIGN
     assert f(p, p, p, 0, 128, 64, 4, p, p, p, p, p, p, p, p, p, 0, None) == rq.ERR_SHAPE
     assert f(p, p, p, 1, 128, 64, 4, p, p, p, p, p, None, p, p, p, 0, None) == rq.ERR_NULL
+
+
+def test_preset_decode_argument_errors(L):
+    """rq_gemv_p8_g16 / rq_gemv_p4a_g32 reject bad arguments before any launch."""
+    p = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    g8 = L.rq_gemv_p8_g16
+    assert g8(p, 1, 192, p, p, 64, p, None) == rq.ERR_SHAPE        # K % 128
+    assert g8(p, 0, 128, p, p, 64, p, None) == rq.ERR_SHAPE
+    assert g8(p, 33, 128, p, p, 64, p, None) == rq.ERR_SHAPE
+    assert g8(p, 1, 128, p, p, 0, p, None) == rq.ERR_SHAPE
+    assert g8(None, 1, 128, p, p, 64, p, None) == rq.ERR_NULL
+    assert g8(p, 1, 128, p, None, 64, p, None) == rq.ERR_NULL
+    assert g8(p, 1, 128, p, p, 64, None, None) == rq.ERR_NULL
+    assert g8(odd, 1, 128, p, p, 64, p, None) == rq.ERR_ALIGN
+    assert g8(p, 1, 128, odd, p, 64, p, None) == rq.ERR_ALIGN
+    g4 = L.rq_gemv_p4a_g32
+    assert g4(p, 1, 128, p, p, p, 64, p, None) == rq.ERR_SHAPE     # K % 256
+    assert g4(p, 33, 256, p, p, p, 64, p, None) == rq.ERR_SHAPE
+    assert g4(p, 1, 256, p, None, p, 64, p, None) == rq.ERR_NULL
+    assert g4(p, 1, 256, p, p, None, 64, p, None) == rq.ERR_NULL
+    assert g4(p, 1, 256, p, p, odd, 64, p, None) == rq.ERR_ALIGN
+    assert g4(p, 1, 256, p, odd, p, 64, p, None) == rq.ERR_ALIGN
 
 
 def test_gptq_argument_errors(L):

@@ -5,6 +5,7 @@ Usage: python -m weight_only_quantized_g64_b200.build [--force] [--verbose-ptxas
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -15,6 +16,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librq.so")
+OBJ = os.path.join(PKG, "_build")             # per-file objects, removed after the link
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -41,23 +43,47 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in deps())
 
 
+def _flags():
+    return [*ARCH, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC",
+            "-I" + os.path.join(ROOT, "include"), "-I" + CSRC, "--expt-relaxed-constexpr"]
+
+
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    """Compile every source to an object (in parallel, one nvcc per file) and
+    link them into librq.so with the CUDA runtime linked statically."""
     if not force and up_to_date():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, "-lineinfo", "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-I" + os.path.join(ROOT, "include"), "-I" + CSRC,
-           "--expt-relaxed-constexpr", "-cudart", "static",
-           *sources(), "-o", tmp]
-    if ptxas_verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building librq.so")
-    if ptxas_verbose:
-        sys.stdout.write(r.stdout + r.stderr)
-    os.replace(tmp, LIB)
+    os.makedirs(OBJ, exist_ok=True)
+    tag = f".{os.getpid()}"
+    jobs = []
+    for src in sources():
+        obj = os.path.join(OBJ, os.path.basename(src)[:-3] + tag + ".o")
+        cmd = [nvcc(), *_flags(), "-c", src, "-o", obj]
+        if ptxas_verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        jobs.append((cmd, obj))
+    workers = max(1, min(len(jobs), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+        results = list(ex.map(lambda j: subprocess.run(j[0], capture_output=True, text=True), jobs))
+    failed = [r for r in results if r.returncode != 0]
+    for r in results:
+        if r.returncode != 0 or ptxas_verbose:
+            (sys.stderr if r.returncode != 0 else sys.stdout).write(r.stdout + r.stderr)
+    objs = [o for _, o in jobs]
+    try:
+        if failed:
+            raise RuntimeError("nvcc failed building librq.so")
+        tmp = LIB + f".tmp{os.getpid()}"
+        r = subprocess.run([nvcc(), *ARCH, "-shared", "-cudart", "static", *objs, "-o", tmp],
+                           capture_output=True, text=True)
+        if r.returncode != 0:
+            sys.stderr.write(r.stdout + r.stderr)
+            raise RuntimeError("nvcc failed linking librq.so")
+        os.replace(tmp, LIB)
+    finally:
+        for o in objs:
+            if os.path.exists(o):
+                os.remove(o)
     return LIB
 
 

@@ -45,12 +45,14 @@ int decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat) {
     if (g_decode_kernel == RQ_DECODE_ROWTILE) return RQ_DECODE_ROWTILE;
     if (g_decode_kernel == RQ_DECODE_ROWBLOCK)
         return gemv_rowblock_fits(M, K, N, bits, nmat) ? RQ_DECODE_ROWBLOCK : -1;
-    // measured on B200 (graph-replayed chains, int4): the cluster kernel is
-    // ahead for M > 16 on every projection shape, and for M 9..16 on tall
-    // ones (>= 6144 rows per launch, K <= 4096); the row-tile kernel
-    // elsewhere
-    if (!fits || M <= 8) return RQ_DECODE_ROWTILE;
-    if (M > 16 || (static_cast<int64_t>(nmat) * N >= 6144 && K <= 4096)) return RQ_DECODE_CLUSTER;
+    // measured on B200 (graph-replayed chains, int4): the row-block kernel
+    // is ahead at every M once the launch has at least one 16-row m-tile per
+    // SM; below that (its CTAs would leave SMs idle) the row-tile kernel,
+    // which also splits K, for M <= 16 and the cluster kernel for M > 16
+    if (static_cast<int64_t>(nmat) * ((N + 15) / 16) >= num_sms() &&
+        gemv_rowblock_fits(M, K, N, bits, nmat))
+        return RQ_DECODE_ROWBLOCK;
+    if (fits && M > 16) return RQ_DECODE_CLUSTER;
     return RQ_DECODE_ROWTILE;
 }
 
@@ -389,6 +391,38 @@ rq_status rq_rkv_fused3(const uint16_t* x_r, const uint16_t* x_k, const uint16_t
     const uint16_t* xs[3] = {x_r, x_k, x_v};
     const cudaError_t e = launch_gemv_rowblock_ex(xs, 3, M, K, N, bits, w, 3, out_dtype == RQ_OUT_F16,
                                                   RQ_EPI_NONE, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+rq_status rq_gemv_p8_g16(const uint16_t* x, int64_t M, int64_t K, const void* codes,
+                         const uint16_t* scales, int64_t N, float* y, rq_stream_t stream) {
+    rq_status st = check_product(x, M, K, N, 8, RQ_MAX_DECODE_M);
+    if (st != RQ_OK) return st;
+    if (K % 128 != 0) return RQ_ERR_SHAPE;
+    if ((st = check_operand(codes, scales, y)) != RQ_OK) return st;
+    if (!gemv_rowblock_fits(M, K, N, 8, 1, FMT_P8)) return RQ_ERR_SHAPE;
+    WOperand w = {codes, scales, y};
+    const uint16_t* xs[1] = {x};
+    const cudaError_t e = launch_gemv_rowblock_fmt(xs, 1, M, K, N, 8, FMT_P8, &w, nullptr, 1, false,
+                                                   RQ_EPI_NONE, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+rq_status rq_gemv_p4a_g32(const uint16_t* x, int64_t M, int64_t K, const void* codes,
+                          const uint8_t* sub, const uint16_t* sup, int64_t N, float* y,
+                          rq_stream_t stream) {
+    rq_status st = check_product(x, M, K, N, 4, RQ_MAX_DECODE_M);
+    if (st != RQ_OK) return st;
+    if (K % 256 != 0) return RQ_ERR_SHAPE;
+    if ((st = check_operand(codes, reinterpret_cast<const uint16_t*>(sub), y)) != RQ_OK) return st;
+    if (sup == nullptr) return RQ_ERR_NULL;
+    if (!aligned16(sup)) return RQ_ERR_ALIGN;
+    if (!gemv_rowblock_fits(M, K, N, 4, 1, FMT_P4A)) return RQ_ERR_SHAPE;
+    WOperand w = {codes, reinterpret_cast<const uint16_t*>(sub), y};
+    const uint16_t* xs[1] = {x};
+    const uint32_t* sp[1] = {reinterpret_cast<const uint32_t*>(sup)};
+    const cudaError_t e = launch_gemv_rowblock_fmt(xs, 1, M, K, N, 4, FMT_P4A, &w, sp, 1, false,
+                                                   RQ_EPI_NONE, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? RQ_OK : cuda_fail(e);
 }
 

@@ -489,16 +489,6 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_wq_kernel(const __grid_con
 
 // ------------------------------------------------------------- launcher --
 
-static int gv_num_sms() {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
-    return sms;
-}
 
 constexpr int kSmemMaxCTA = 227 * 1024;   // dynamic shared memory per CTA, opt-in limit
 
@@ -582,7 +572,7 @@ static cudaError_t gv_launch(GvParams& prm, const uint16_t* x, const void* const
     // Grid: one CTA per SM at most.  Whole row tiles per CTA (nothing is
     // reduced across CTAs) when they balance over the SMs -- one tile per CTA
     // for small projections; otherwise stream-K over equal runs of units.
-    const int sms = gv_num_sms();
+    const int sms = num_sms();
     int grid = 0;
     if (gv_whole_tiles(prm.tiles, sms)) {
         grid = prm.tiles < sms ? prm.tiles : sms;
@@ -685,7 +675,7 @@ static cudaError_t gv_launch(GvParams& prm, const uint16_t* x, const void* const
 // stream-K.  M > 16: warps split the rows of 128-row tiles (WK = 1), so the
 // x of a stage, large at this M, is loaded once for all 8 warps.
 static int gv_pick_mtw(int N) {
-    const int sms = gv_num_sms();
+    const int sms = num_sms();
     if ((N + 15) / 16 <= sms) return 1;
     // relative speed of a warp's unit by m-tiles per unit, measured on B200:
     // 44 / 47 / 49 weights per cycle and SM for 1 / 2 / 4 m-tiles
@@ -710,7 +700,7 @@ static cudaError_t gv_dispatch_mt(GvParams& prm, const uint16_t* x, const void* 
         // rows split over the warps (x of a stage loaded once for 8 warps) when
         // whole 128-row tiles balance; else k split with fewer stages per
         // group (the x of 8 stages of 32 tokens does not fit twice)
-        if (gv_whole_tiles((prm.N + 127) / 128, gv_num_sms()))
+        if (gv_whole_tiles((prm.N + 127) / 128, num_sms()))
             return gv_launch<BITS, NMAT, 1, 4, 1>(prm, x, codes, s, sc);
         return gv_launch<BITS, NMAT, 1, 4, 8>(prm, x, codes, s, sc);
     } else if constexpr (NMAT == 3) {

@@ -376,16 +376,6 @@ __global__ void __launch_bounds__(NW * 32, 1)
 
 // ------------------------------------------------------------- launcher --
 
-static int ck_num_sms() {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
-    return sms;
-}
 
 constexpr int kCkSmemMax = 227 * 1024;
 constexpr int kCkSmemOneCta = 120 * 1024;   // more than half an SM's shared memory
@@ -449,7 +439,7 @@ static int ck_max_clusters(int C, int smem) {
     if (cudaOccupancyMaxActiveClusters(&n, gemv_ck_kernel<BITS, MTW, NT, WK, NW>, &cfg) != cudaSuccess ||
         n <= 0) {
         cudaGetLastError();
-        n = ck_num_sms() / C;
+        n = num_sms() / C;
     }
     if (sb < 64) cache[C][sb] = n;
     return n;

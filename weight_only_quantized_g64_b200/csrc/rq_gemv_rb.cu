@@ -1,512 +1,18 @@
-// rq_gemv_rb.cu -- decode product (1 <= M <= 32) on group-64 quantized
-// weights, row blocks over full K: the row-block decode kernel.
-//
-//   y[m, n] = sum_g s16[n, g] * sum_{k in g} x[m, k] * code[n, k]
-//
-// The "Hakureirm/rwkv7-sglang-w4gptq-1.5b" model card (opening summary)
-// credits its decode speed-up to a hand-written int4 GEMV / small-M kernel
-// family streaming the g64 codes; the "RWKV-7 Quantization Toolkit"
-// (rwkv-quant-nv 1.2.1), "Key Design", keeps weights quantized on the path and
-// runs R/K/V in one launch.  This is the B200 form of that decode step.
-//
-// Work decomposition.  The rows of each matrix are cut into 16-row m-tiles
-// and the m-tiles into blocks of TC consecutive m-tiles (TC = the m-tiles
-// per SM, rounded up); a CTA owns whole blocks over the FULL K range, so
-// every output is finished inside one CTA: no partial sums leave the SM, no
-// workspace, no counters.  (An SM that owns fewer m-tiles than another simply
-// finishes early; one CTA can pull well above its share of HBM bandwidth, so
-// the busiest SMs set the pace only when their share exceeds what one SM can
-// stream.)  Fused R/K/V: the three matrices' blocks are concatenated; a block
-// never straddles two matrices.
-//
-// Data path.  A ring of slots in shared memory; a slot holds, for the
-// block's rows, S consecutive 128-byte code stages (one 3-D TMA box
-// {128 B, 16*TC rows, S stages}, 128-byte swizzled), their fp16 scales (one
-// 2-D box) and the x of their groups (one 3-D box {64 k, M tokens, groups}).
-// Codes and scales of the first slots are requested by thread 0 before the
-// kernel waits on the previous grid (they never depend on it); x after.  The
-// last warp to finish with a slot refills it (an arrival counter in shared
-// memory), so no warp waits to refill.  The 8 warps, all computing, split a
-// slot's group columns (warp w takes columns w, w+8, ...) and
-// each takes every m-tile of the block for its columns, so an x fragment is
-// loaded once per warp and column and used TC times.  At the end of a block
-// the warps' partial sums meet in shared memory (the ring, reused) and are
-// added in warp order, so the result is deterministic.
-//
-// Math.  Thread (g = lane/4, t = lane%4) owns, per group of 64 k, the 16 k
-// [16t, 16t+16) of rows g and g+8 of each m-tile (a k-permutation inside the
-// group, the same on the A and B side, so the sum over k is unchanged).  Codes
-// are turned into BIASED fp16 values with one lop3 per pair (the bit placement
-// of Kim et al., arXiv:2211.10017, without the exact bias subtraction): int4
-// low nibbles become 1032 + c (exponent of [1024, 2048)), high nibbles
-// 72 + c (exponent of [64, 128), the nibble at mantissa bits 4..7); int8
-// bytes 1152 + c.  mma.sync.m16n8k16 sums x * (code + bias) in fp32, starting
-// from -sum_k bias_k x_k of the group, which one chain of MMAs with a
-// constant A operand (-bias) computes once per group and 8-token tile and
-// every m-tile reuses.  The group's scale is applied in fp32
-// (acc = fma(part, s16, acc)).  Products x * (code + bias) are exact in fp32
-// (11 x 11 significant bits), so the bias costs only the fp32 rounding of
-// sums of magnitude ~1000 |x|: about 1e-4 of the error budget
-// 2e-3 * sum |x||w_hat| per output.
-#include <cuda_fp16.h>
-
+// rq_gemv_rb.cu -- host side of the row-block decode kernel (rq_gemv_rb.cuh):
+// how a product is cut into blocks and slots, and the launch entry points.
 #include <cstring>
 
-#include "rq_internal.h"
-#include "rq_ptx.cuh"
-#include "rq_gemv_unit.cuh"
+#include "rq_gemv_rb.cuh"
 
 namespace rq {
 
-struct RbParams {
-    CUtensorMap tm_w[3];  // codes: 3-D {128 B, N rows, stages} box {128, RB, S}, or (rows not whole
-                          // stages) 2-D {row bytes, N} box {128, RB}; SWIZZLE_128B
-    CUtensorMap tm_s[3];  // scales [N, groups] fp16: box {SROW, RB} (when ssc)
-    CUtensorMap tm_x[3];  // x of each matrix as 3-D {64, M, groups}: box {64, M, J}, SWIZZLE_128B
-    const uint16_t* scales[3];
-    void* y[3];           // fp32 or (yh) fp16 [M, N]
-    int M, N, K;
-    int groups;           // K / 64
-    int stages;           // 128-byte code stages per row
-    int tc;               // m-tiles per block (TC)
-    int bpm;              // blocks per matrix
-    int nblocks;          // blocks in all matrices
-    int S;                // stages per slot
-    int J;                // group columns per slot (S * groups per stage)
-    int slots;            // slots per block: ceil(stages / S)
-    int sg;               // ring depth (slots)
-    int three_d;          // codes through the 3-D map
-    int ssc;              // scales staged by TMA
-    int srow;             // scale row length in a slot (fp16, 16-byte multiple)
-    int slot_bytes, s_off, x_off, bar_off, red_stride;
-    int nx;               // distinct inputs: 1 (shared x) or 3 (one per matrix)
-    int yh;               // y stored as fp16 (round to nearest even)
-    int epi;              // epilogue: 0 none, 1 relu(y)^2
-    int* status;
-    uint64_t timeout_ns;
-};
-
-constexpr int kRbSrow = 40;                     // fp16 scales per staged row (J <= 32, + slack)
-constexpr int kRbWarps = 8;                     // warps, all computing
-constexpr int kRbThreads = kRbWarps * 32;
-constexpr int kRbMaxSG = 8;
-
-struct RbBars {
-    uint64_t full[kRbMaxSG];   // the slot holds its codes, scales and x
-    int done[kRbMaxSG];        // warps finished with the slot's current round
-    int issued_hi[kRbMaxSG];   // last slot index issued into each ring slot
-    int abort;
-};
-
-// D = A * B + C (fp16 inputs, fp32 accumulate), C and D distinct.
-__device__ __forceinline__ void mma16816_c(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                           uint32_t b1, const float (&c)[4]) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%10,%11,%12,%13};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]),
-          "f"(c[2]), "f"(c[3]));
-}
-
-// int4, permuted pair order, biased: one code word (positions 0..7 of a row,
-// position 2i in the low nibble of byte i) -> pairs (p0,p4) and (p2,p6) as
-// 1032 + c, pairs (p1,p5) and (p3,p7) as 72 + c.  5 instructions per 8 codes.
-__device__ __forceinline__ void i4_word_biased(uint32_t w, uint32_t (&P)[4]) {
-    const uint32_t w8 = w >> 8;
-    P[0] = lop3_bmux(w, 0x000F000Fu, 0x64086408u);    // 0x6400 | (nibble ^ 8)       = 1032 + c
-    P[1] = lop3_bmux(w, 0x00F000F0u, 0x54805480u);    // 0x5400 | (nibble ^ 8) << 4  = 72 + c
-    P[2] = lop3_bmux(w8, 0x000F000Fu, 0x64086408u);
-    P[3] = lop3_bmux(w8, 0x00F000F0u, 0x54805480u);
-}
-
-// int8, biased: one 32-bit word (positions 0..3) -> pairs (p0,p1), (p2,p3) as
-// 1152 + c.  3 instructions per 4 codes.
-__device__ __forceinline__ void i8_word_biased(uint32_t w, uint32_t (&Q)[2]) {
-    w ^= 0x80808080u;
-    Q[0] = __byte_perm(w, 0x64646464u, 0x5140u);
-    Q[1] = __byte_perm(w, 0x64646464u, 0x5342u);
-}
-
-// Group columns of one warp (NC of them, processed together for independent
-// dependency chains): every m-tile of the block (MT of them) times the x of
-// the column's group, for NT 8-token tiles.  Per column c:
-//   cw0[c]  codes of the column's stage, m-tile 0, this thread's physical row
-//           and chunk (rows 16i + prow and +8 of m-tile i are 16*128*i and
-//           8*128 further)
-//   sp[c]   scales: (row 16i + 8h + prow, this group) at sp[c][(16i + 8h) * kRbSrow]
-//   xrow    byte offsets (from xbase) of the 128-byte x rows of the column's
-//           group for the tokens nt*8+g; xph[nt] their swizzle phase
-//   grp[c]  the group (for scales read from global memory when !SSC)
-// The group's four MMA steps run as one chain that starts from the bias term
-// (so no additions are needed), and the scale is applied with one fma.
-template <int BITS, int MT, int NT, int NC, bool SSC>
-__device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
-                                           const uint16_t* const (&sp)[NC], const uint8_t* xbase,
-                                           const int (&xrow)[NC][NT], const int (&xph)[NT], int t,
-                                           float (&acc)[MT][NT][4], const uint16_t* gscales,
-                                           int64_t grow0, int groups, const int (&grp)[NC], int N) {
-    constexpr int CW = BITS == 4 ? 2 : 4;   // code words per row and group
-    // ---- x fragments: token nt*8+g, positions 16t .. 16t+15 of the group
-    uint32_t b[NC][NT][4][2];
-#pragma unroll
-    for (int c = 0; c < NC; ++c)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const uint8_t* xr = xbase + xrow[c][nt];
-            const int c0 = ((2 * t) ^ xph[nt]) << 4;
-            const uint4 v0 = lds128(xr + c0);
-            const uint4 v1 = lds128(xr + (c0 ^ 16));
-            const uint32_t X[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                if constexpr (BITS == 4) {
-                    // step jj pairs (p0,p4),(p1,p5) or (p2,p6),(p3,p7) of word jj/2
-                    const int wb = (jj >> 1) * 4 + (jj & 1);
-                    b[c][nt][jj][0] = __byte_perm(X[wb], X[wb + 2], 0x5410);
-                    b[c][nt][jj][1] = __byte_perm(X[wb], X[wb + 2], 0x7632);
-                } else {
-                    b[c][nt][jj][0] = X[2 * jj];
-                    b[c][nt][jj][1] = X[2 * jj + 1];
-                }
-            }
-        }
-    // ---- -sum_k bias_k x_k of each column's group, per token tile (the same
-    // for every row)
-    float negc[NC][NT][4];
-    {
-        uint32_t an[4];
-        if constexpr (BITS == 4) {
-            an[0] = an[1] = 0xE408E408u;   // -1032 (slots 2t, 2t+1: low-nibble pairs)
-            an[2] = an[3] = 0xD480D480u;   // -72   (slots 2t+8, 2t+9: high-nibble pairs)
-        } else {
-            an[0] = an[1] = an[2] = an[3] = 0xE480E480u;   // -1152
-        }
-#pragma unroll
-        for (int c = 0; c < NC; ++c)
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                mma16816(negc[c][nt], an, b[c][nt][0][0], b[c][nt][0][1], true);
-#pragma unroll
-                for (int jj = 1; jj < 4; ++jj)
-                    mma16816(negc[c][nt], an, b[c][nt][jj][0], b[c][nt][jj][1], false);
-            }
-    }
-    // ---- every m-tile
-#pragma unroll
-    for (int i = 0; i < MT; ++i) {
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            uint32_t cw[2][CW];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint8_t* cp = cw0[c] + (16 * i + 8 * h) * 128;
-                if constexpr (BITS == 4) {
-                    const uint2 v = lds64(cp);
-                    cw[h][0] = v.x;
-                    cw[h][1] = v.y;
-                } else {
-                    const uint4 v = lds128(cp);
-                    cw[h][0] = v.x; cw[h][1] = v.y; cw[h][2] = v.z; cw[h][3] = v.w;
-                }
-            }
-            float sv[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint16_t s16;
-                if constexpr (SSC) {
-                    s16 = sp[c][(16 * i + 8 * h) * kRbSrow];
-                } else {
-                    const int64_t n = grow0 + 16 * i + 8 * h;
-                    s16 = (n < N && grp[c] < groups) ? __ldg(gscales + n * groups + grp[c])
-                                                     : static_cast<uint16_t>(0);
-                }
-                sv[h] = __half2float(__ushort_as_half(s16));
-            }
-            uint32_t A[4][4];   // [step][a-reg]
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                if constexpr (BITS == 4) {
-                    uint32_t P0[4], P1[4];
-                    i4_word_biased(cw[h][0], P0);
-                    i4_word_biased(cw[h][1], P1);
-                    A[0][h] = P0[0]; A[0][h + 2] = P0[1];
-                    A[1][h] = P0[2]; A[1][h + 2] = P0[3];
-                    A[2][h] = P1[0]; A[2][h + 2] = P1[1];
-                    A[3][h] = P1[2]; A[3][h + 2] = P1[3];
-                } else {
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        uint32_t Q[2];
-                        i8_word_biased(cw[h][jj], Q);
-                        A[jj][h] = Q[0];
-                        A[jj][h + 2] = Q[1];
-                    }
-                }
-            }
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                float part[4];
-                mma16816_c(part, A[0], b[c][nt][0][0], b[c][nt][0][1], negc[c][nt]);
-#pragma unroll
-                for (int jj = 1; jj < 4; ++jj) mma16816(part, A[jj], b[c][nt][jj][0], b[c][nt][jj][1], false);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[i][nt][e] = fmaf(part[e], sv[e >> 1], acc[i][nt][e]);
-            }
-        }
-    }
-}
-
-template <int BITS, int MT, int NT, bool SSC>
-__global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_constant__ RbParams p) {
-    constexpr int GPS = BITS == 4 ? 4 : 2;      // groups per 128-byte stage
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // 1024-byte aligned start, reached by an offset from the shared array
-    // itself so every access below stays a shared-memory access
-    const uint32_t s0 = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
-    uint8_t* smem = smem_raw + ((1024u - (s0 & 1023u)) & 1023u);
-    uint8_t* ring = smem;
-    RbBars* bars = reinterpret_cast<RbBars*>(smem + p.bar_off);
-    volatile int* abort_flag = &bars->abort;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int SG = p.sg;
-    const int RB = 16 * MT;                     // rows of a block (== 16 * p.tc)
-    const int cbytes = RB * 128 * p.S;          // code bytes of a slot
-    const uint32_t x_bytes = static_cast<uint32_t>(p.J * p.M * 128);
-    const uint32_t s_bytes = SSC ? static_cast<uint32_t>(RB * kRbSrow * 2) : 0u;
-
-    // Loads of the CTA's slot i (block blk, slot sl of the block) into ring slot r.
-    auto issue_w = [&](int r, int blk, int sl) {
-        uint8_t* dst = ring + r * p.slot_bytes;
-        const int m = blk / p.bpm;
-        const int row0 = (blk - m * p.bpm) * RB;
-        const int st0 = sl * p.S;
-        const uint64_t pol = l2_policy_evict_first();
-        mbar_arrive_expect_tx(&bars->full[r], static_cast<uint32_t>(cbytes) + s_bytes + x_bytes);
-        if (p.three_d) {
-            tma_load_3d(dst, &p.tm_w[m], &bars->full[r], 0, row0, st0, pol);
-        } else {
-            for (int s = 0; s < p.S; ++s)
-                tma_load_2d(dst + s * RB * 128, &p.tm_w[m], &bars->full[r], (st0 + s) * 128, row0, pol);
-        }
-        if constexpr (SSC)
-            tma_load_2d(dst + p.s_off, &p.tm_s[m], &bars->full[r], (st0 * GPS) & ~7, row0, pol);
-    };
-    auto issue_x = [&](int r, int blk, int sl) {
-        const int m = p.nx > 1 ? blk / p.bpm : 0;
-        tma_load_3d(ring + r * p.slot_bytes + p.x_off, &p.tm_x[m], &bars->full[r], 0, 0, sl * p.J,
-                    l2_policy_evict_last());
-    };
-
-    if (threadIdx.x == 0) {
-        for (int r = 0; r < SG; ++r) {
-            mbar_init(&bars->full[r], 1);
-            bars->done[r] = 0;
-            bars->issued_hi[r] = -1;
-        }
-        bars->abort = 0;
-        fence_mbar_init();
-        for (int m = 0; m < 3; ++m) {
-            if (p.y[m] == nullptr) break;
-            if (m < p.nx) tma_prefetch_desc(&p.tm_x[m]);
-            tma_prefetch_desc(&p.tm_w[m]);
-            if (SSC) tma_prefetch_desc(&p.tm_s[m]);
-        }
-        // codes and scales of the first block's first slots: they never
-        // depend on the previous grid, so they go out before waiting on it
-        const int n_pre = min(SG, p.slots);
-        for (int r = 0; r < n_pre; ++r) {
-            bars->issued_hi[r] = r;
-            issue_w(r, blockIdx.x, r);
-        }
-    }
-    __syncthreads();
-    pdl_launch_dependents();
-    pdl_wait();   // x (and y) may be used by the previous kernel
-    if (threadIdx.x == 0) {
-        const int n_pre = min(SG, p.slots);
-        for (int r = 0; r < n_pre; ++r) issue_x(r, blockIdx.x, r);
-    }
-
-    const int g = lane >> 2;
-    const int t = lane & 3;
-    const int prow = phys_row<BITS>(g);
-    // This warp's columns of a slot are j = warp + 8c: for int4 stage
-    // warp/4 + 2c, group warp%4 of it; for int8 stage warp/2 + 4c, group
-    // warp%2.  Every per-column offset below is a constant plus c strides.
-    constexpr int CPS = kRbWarps / GPS;                 // stages between a warp's columns
-    const int q0 = warp % GPS;
-    int coff;
-    if constexpr (BITS == 4)
-        coff = prow * 128 + (((2 * q0 + (t >> 1)) ^ (prow & 7)) << 4) + ((t & 1) << 3);
-    else
-        coff = prow * 128 + (((4 * q0 + t) ^ (prow & 7)) << 4);
-    const int code0 = (warp / GPS) * RB * 128 + coff;   // the warp's first column in a slot
-    const int code_step = CPS * RB * 128;
-    int xrow0[NT], xph[NT];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int line = warp * p.M + min(nt * 8 + g, p.M - 1);
-        xrow0[nt] = p.x_off + line * 128;
-        xph[nt] = line & 7;                             // unchanged by the 8*M-line column stride
-    }
-    const int x_step = kRbWarps * p.M * 128;
-    int gi = 0;                 // the CTA's slot index (over all its blocks)
-    int r = 0;                  // its ring slot (gi % SG) and that slot's phase
-    uint32_t ph = 0;
-    bool dead = false;
-    int kb = 0;                 // blocks done by this CTA
-    for (int blk = blockIdx.x; blk < p.nblocks; blk += gridDim.x, ++kb) {
-        const int m = blk / p.bpm;
-        const int row0 = (blk - m * p.bpm) * RB;
-        if (kb > 0 && threadIdx.x == 0) {
-            // a later block: the ring was the previous block's reduction
-            // buffer, so its first slots go out only now
-            const int n_pre = min(SG, p.slots);
-            int rq = r;
-            for (int q = 0; q < n_pre; ++q) {
-                bars->issued_hi[rq] = gi + q;
-                issue_w(rq, blk, q);
-                issue_x(rq, blk, q);
-                if (++rq == SG) rq = 0;
-            }
-        }
-        float acc[MT][NT][4];
-#pragma unroll
-        for (int i = 0; i < MT; ++i)
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[i][nt][e] = 0.0f;
-        for (int sl = 0; sl < p.slots; ++sl, ++gi) {
-            if (!dead && !mbar_wait(&bars->full[r], ph, abort_flag, p.timeout_ns, p.status))
-                dead = true;
-            const int grp0 = sl * p.J;                  // first group of the slot
-            int jn = p.groups - grp0;                   // group columns holding data
-            if (jn > p.J) jn = p.J;
-            if (!dead) {
-                const uint8_t* base = ring + r * p.slot_bytes;
-                const uint8_t* cbase = base + code0;
-                const uint16_t* sbase = reinterpret_cast<const uint16_t*>(base + p.s_off) +
-                                        prow * kRbSrow + (grp0 & 7) + warp;
-                int c = 0;
-                // (pairs only for one token tile: larger M takes one column
-                // per warp and slot, and the registers go to its tiles)
-                if constexpr (NT == 1)
-                for (; warp + kRbWarps * (c + 1) < jn; c += 2) {
-                    const uint8_t* cw0[2] = {cbase + c * code_step, cbase + (c + 1) * code_step};
-                    const uint16_t* sp[2] = {sbase + kRbWarps * c, sbase + kRbWarps * (c + 1)};
-                    int xr[2][NT];
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        xr[0][nt] = xrow0[nt] + c * x_step;
-                        xr[1][nt] = xrow0[nt] + (c + 1) * x_step;
-                    }
-                    const int gr[2] = {grp0 + warp + kRbWarps * c, grp0 + warp + kRbWarps * (c + 1)};
-                    rb_columns<BITS, MT, NT, 2, SSC>(cw0, sp, base, xr, xph, t, acc, p.scales[m],
-                                                     row0 + prow, p.groups, gr, p.N);
-                }
-                for (; warp + kRbWarps * c < jn; ++c) {
-                    const uint8_t* cw0[1] = {cbase + c * code_step};
-                    const uint16_t* sp[1] = {sbase + kRbWarps * c};
-                    int xr[1][NT];
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) xr[0][nt] = xrow0[nt] + c * x_step;
-                    const int gr[1] = {grp0 + warp + kRbWarps * c};
-                    rb_columns<BITS, MT, NT, 1, SSC>(cw0, sp, base, xr, xph, t, acc, p.scales[m],
-                                                     row0 + prow, p.groups, gr, p.N);
-                }
-            }
-            // ---- release the slot; the last warp out refills it with the
-            // block's slot sl + SG (later blocks refill after their reduction)
-            __syncwarp();
-            if (lane == 0) {
-                __threadfence_block();
-                const int prev = atomicAdd(&bars->done[r], 1);
-                if (prev == kRbWarps - 1) {
-                    __threadfence_block();
-                    bars->done[r] = 0;
-                    const int nsl = sl + SG;
-                    if (nsl < p.slots && !dead && *abort_flag == 0) {
-                        bars->issued_hi[r] = gi + SG;
-                        // order every warp's generic reads of the slot before
-                        // the asynchronous writes into it
-                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                        issue_w(r, blk, nsl);
-                        issue_x(r, blk, nsl);
-                    }
-                }
-            }
-            if (++r == SG) {
-                r = 0;
-                ph ^= 1u;
-            }
-        }
-        // ---- the block's sums: warps deposit, then add in warp order
-        __syncthreads();   // every warp is done reading the ring
-        float* red = reinterpret_cast<float*>(ring);
-        const int RS = p.red_stride;                   // floats per (warp, token)
-        for (int nt0 = 0; nt0 < NT; ++nt0) {
-            // round nt0: tokens [8 nt0, 8 nt0 + 8)
-#pragma unroll
-            for (int i = 0; i < MT; ++i)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int tl = 2 * t + (e & 1);
-                    const int rr = 16 * i + 8 * (e >> 1) + prow;
-                    float v = 0.0f;
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-                        if (nt == nt0) v = acc[i][nt][e];
-                    red[(warp * 8 + tl) * RS + rr] = v;
-                }
-            __syncthreads();
-            const int ntok = min(8, p.M - 8 * nt0);
-            for (int o = threadIdx.x; o < ntok * RB; o += kRbThreads) {
-                const int tl = o / RB;
-                const int rr = o - tl * RB;
-                float v = 0.0f;
-#pragma unroll
-                for (int w = 0; w < kRbWarps; ++w) v += red[(w * 8 + tl) * RS + rr];
-                if (p.epi == 1) {
-                    v = fmaxf(v, 0.0f);
-                    v = v * v;
-                }
-                const int n = row0 + rr;
-                if (n < p.N && !dead && *abort_flag == 0) {
-                    const int64_t at = static_cast<int64_t>(8 * nt0 + tl) * p.N + n;
-                    if (p.yh)
-                        static_cast<__half*>(p.y[m])[at] = __float2half_rn(v);
-                    else
-                        static_cast<float*>(p.y[m])[at] = v;
-                }
-            }
-            __syncthreads();
-        }
-    }
-    // After a timeout some issued copies may never have been waited for:
-    // wait (bounded) for the last one of every slot before the CTA exits.
-    __syncthreads();
-    if (threadIdx.x == 0 && *abort_flag) {
-        int dummy_abort = 0;
-        for (int r = 0; r < SG; ++r) {
-            const int il = bars->issued_hi[r];
-            if (il >= 0)
-                mbar_wait(&bars->full[r], static_cast<uint32_t>(il / SG) & 1, &dummy_abort,
-                          p.timeout_ns, p.status);
-        }
-    }
-}
-
-// ------------------------------------------------------------- launcher --
-
-static int rb_num_sms() {
+int num_sms() {
     static int sms[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
     if (sms[dev] == 0) {
         int v = 0;
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) v = 0;
         sms[dev] = v > 0 ? v : 148;
     }
     return sms[dev];
@@ -519,20 +25,15 @@ constexpr int kRbMaxTC = 8;                       // m-tiles per block at most
 
 static int rb_align(int v, int a) { return (v + a - 1) / a * a; }
 
-// How a decode product of this shape is cut for the row-block kernel.
-struct RbPlan {
-    int tc, bpm, nblocks, grid, stages, S, J, slots, sg, srow;
-    int slot_bytes, s_off, x_off, bar_off, red_stride, smem;
-    bool three_d;
-};
-
-static bool rb_plan(int64_t M, int64_t K, int64_t N, int bits, int nmat, RbPlan* P) {
+// fmt: FMT_G64 (bits 4 or 8), FMT_P8 (bits 8), FMT_P4A (bits 4).
+static bool rb_plan(int64_t M, int64_t K, int64_t N, int bits, int nmat, int fmt, RbPlan* P) {
     const int GPS = bits == 4 ? 4 : 2;
-    const int sms = rb_num_sms();
+    const int sms = num_sms();
     const int64_t tm = (N + 15) / 16;                 // m-tiles per matrix
     const int64_t T = tm * nmat;
     int64_t tc = (T + sms - 1) / sms;
     if (tc > kRbMaxTC) tc = kRbMaxTC;
+    if (fmt != FMT_G64 && M > 16 && tc > 4) tc = 4;   // (taller preset blocks spill at M > 16)
     if (tc < 1) tc = 1;
     P->tc = static_cast<int>(tc);
     P->bpm = static_cast<int>((tm + tc - 1) / tc);
@@ -544,21 +45,39 @@ static bool rb_plan(int64_t M, int64_t K, int64_t N, int bits, int nmat, RbPlan*
     P->three_d = row_bytes % 128 == 0;
     // stages per slot: about 16 KB of codes, at least 16 group columns (two
     // per warp, processed together) for M <= 8 and 8 otherwise, when the row
-    // has them, and at most 16 KB of x (32 KB for M > 16)
-    const int smin = (M <= 8 ? 16 : 8) / GPS;
-    const int64_t x_cap = M > 16 ? 32768 : 16384;
+    // has them, and at most 16 KB of x (32 KB for M > 16).  Short blocks (one
+    // or two m-tiles) take at least 32 columns and up to 32 KB of x: their
+    // slots are small, and fewer, larger slots measured faster on B200.
+    const bool short_blk = P->tc <= 2;
+    const int smin = (M <= 8 ? (short_blk ? 32 : 16) : 8) / GPS;
+    const int64_t x_cap = M > 16 || short_blk ? 32768 : 16384;
     int S = 1;
     while (S * 2 * RB * 128 <= 16384 && S < 16) S *= 2;
     if (S < smin) S = smin;
     while (S > smin && static_cast<int64_t>(S) * GPS * M * 128 > x_cap) S /= 2;
+    // the int8 preset stages 4 scales per column in a row of kRbSrowP8
+    if (fmt == FMT_P8)
+        while (S * GPS > 16) S /= 2;
     if (S > P->stages) S = P->stages;
     P->S = S;
     P->J = S * GPS;
     P->slots = (P->stages + S - 1) / S;
-    P->srow = kRbSrow;
+    // staged metadata row: elements of the scale map's box and its bytes
+    int srow_bytes;
+    if (fmt == FMT_P8) {
+        if (P->J > 16) return false;
+        P->srow = kRbSrowP8;
+        srow_bytes = 2 * kRbSrowP8;
+    } else if (fmt == FMT_P4A) {
+        P->srow = 4 * P->J;          // (a, b) of the slot's 2 J groups
+        srow_bytes = P->srow;
+    } else {
+        P->srow = kRbSrow;
+        srow_bytes = 2 * kRbSrow;
+    }
     const int cbytes = RB * 128 * S;
     P->s_off = cbytes;
-    P->x_off = rb_align(P->s_off + RB * P->srow * 2, 1024);
+    P->x_off = rb_align(P->s_off + RB * srow_bytes, 1024);
     P->slot_bytes = rb_align(P->x_off + P->J * static_cast<int>(M) * 128, 1024);
     P->red_stride = RB + 4;
     const int red_bytes = kRbWarps * 8 * P->red_stride * 4;
@@ -579,90 +98,12 @@ static bool rb_plan(int64_t M, int64_t K, int64_t N, int bits, int nmat, RbPlan*
     return false;
 }
 
-bool gemv_rowblock_fits(int64_t M, int64_t K, int64_t N, int bits, int nmat) {
+bool gemv_rowblock_fits(int64_t M, int64_t K, int64_t N, int bits, int nmat, int fmt) {
     if (M < 1 || M > 32) return false;
+    if (fmt == FMT_P8 && (bits != 8 || K % 128 != 0)) return false;
+    if (fmt == FMT_P4A && (bits != 4 || K % 256 != 0)) return false;
     RbPlan P;
-    return rb_plan(M, K, N, bits, nmat, &P);
-}
-
-template <int BITS, int MT, int NT, bool SSC>
-static cudaError_t rb_launch(RbParams& prm, const RbPlan& P, const uint16_t* const* xs,
-                             const void* const* codes, int nmat, cudaStream_t s) {
-    auto kern = gemv_rb_kernel<BITS, MT, NT, SSC>;
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
-    const int RB = 16 * MT;
-    const uint64_t row_bytes = static_cast<uint64_t>(prm.K) * BITS / 8;
-    for (int i = 0; i < nmat; ++i) {
-        const bool okw =
-            P.three_d
-                ? make_tmap_3d(&prm.tm_w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, codes[i], 128,
-                               static_cast<uint64_t>(prm.N), static_cast<uint64_t>(P.stages),
-                               row_bytes, 128, 128, static_cast<uint32_t>(RB),
-                               static_cast<uint32_t>(P.S), CU_TENSOR_MAP_SWIZZLE_128B)
-                : make_tmap_2d(&prm.tm_w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, codes[i], row_bytes,
-                               static_cast<uint64_t>(prm.N), row_bytes, 128,
-                               static_cast<uint32_t>(RB), CU_TENSOR_MAP_SWIZZLE_128B);
-        if (!okw) return cudaErrorInvalidValue;
-        if (prm.ssc &&
-            !make_tmap_2d(&prm.tm_s[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, prm.scales[i],
-                          static_cast<uint64_t>(prm.groups), static_cast<uint64_t>(prm.N),
-                          static_cast<uint64_t>(prm.groups) * 2, static_cast<uint32_t>(P.srow),
-                          static_cast<uint32_t>(RB), CU_TENSOR_MAP_SWIZZLE_NONE))
-            return cudaErrorInvalidValue;
-    }
-    for (int i = 0; i < prm.nx; ++i)
-        if (!make_tmap_3d(&prm.tm_x[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs[i], 64,
-                          static_cast<uint64_t>(prm.M), static_cast<uint64_t>(prm.groups),
-                          static_cast<uint64_t>(prm.K) * 2, 128, 64, static_cast<uint32_t>(prm.M),
-                          static_cast<uint32_t>(P.J), CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(P.grid), 1, 1);
-    cfg.blockDim = dim3(kRbThreads, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(P.smem);
-    cfg.stream = s;
-    cudaLaunchAttribute attrs[1];
-    int na = 0;
-    if (pdl_enabled()) {
-        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attrs[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-    }
-    cfg.attrs = attrs;
-    cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, kern, static_cast<const RbParams&>(prm));
-}
-
-template <int BITS, int NT, bool SSC>
-static cudaError_t rb_dispatch_mt(RbParams& prm, const RbPlan& P, const uint16_t* const* x,
-                                  const void* const* codes, int nmat, cudaStream_t s) {
-    switch (P.tc) {
-        case 1: return rb_launch<BITS, 1, NT, SSC>(prm, P, x, codes, nmat, s);
-        case 2: return rb_launch<BITS, 2, NT, SSC>(prm, P, x, codes, nmat, s);
-        case 3: return rb_launch<BITS, 3, NT, SSC>(prm, P, x, codes, nmat, s);
-        case 4: return rb_launch<BITS, 4, NT, SSC>(prm, P, x, codes, nmat, s);
-        case 5: return rb_launch<BITS, 5, NT, SSC>(prm, P, x, codes, nmat, s);
-        case 6: return rb_launch<BITS, 6, NT, SSC>(prm, P, x, codes, nmat, s);
-        case 7: return rb_launch<BITS, 7, NT, SSC>(prm, P, x, codes, nmat, s);
-        default: return rb_launch<BITS, 8, NT, SSC>(prm, P, x, codes, nmat, s);
-    }
-}
-
-template <int BITS, int NT>
-static cudaError_t rb_dispatch_ssc(RbParams& prm, const RbPlan& P, const uint16_t* const* x,
-                                   const void* const* codes, int nmat, cudaStream_t s) {
-    return prm.ssc ? rb_dispatch_mt<BITS, NT, true>(prm, P, x, codes, nmat, s)
-                   : rb_dispatch_mt<BITS, NT, false>(prm, P, x, codes, nmat, s);
+    return rb_plan(M, K, N, bits, nmat, fmt, &P);
 }
 
 cudaError_t launch_gemv_rowblock(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
@@ -674,9 +115,19 @@ cudaError_t launch_gemv_rowblock(const uint16_t* x, int64_t M, int64_t K, int64_
 cudaError_t launch_gemv_rowblock_ex(const uint16_t* const* xs, int nx, int64_t M, int64_t K,
                                     int64_t N, int bits, const WOperand* w, int nmat, bool y_half,
                                     int epilogue, cudaStream_t s) {
+    return launch_gemv_rowblock_fmt(xs, nx, M, K, N, bits, FMT_G64, w, nullptr, nmat, y_half,
+                                    epilogue, s);
+}
+
+cudaError_t launch_gemv_rowblock_fmt(const uint16_t* const* xs, int nx, int64_t M, int64_t K,
+                                     int64_t N, int bits, int fmt, const WOperand* w,
+                                     const uint32_t* const* sup, int nmat, bool y_half,
+                                     int epilogue, cudaStream_t s) {
     RbPlan P;
     const uint16_t* const* x = xs;
-    if (M < 1 || M > 32 || !rb_plan(M, K, N, bits, nmat, &P)) return cudaErrorInvalidValue;
+    if (!gemv_rowblock_fits(M, K, N, bits, nmat, fmt) || !rb_plan(M, K, N, bits, nmat, fmt, &P))
+        return cudaErrorInvalidValue;
+    if (fmt == FMT_P4A && sup == nullptr) return cudaErrorInvalidValue;
     RbParams prm;
     memset(&prm, 0, sizeof(prm));
     prm.M = static_cast<int>(M);
@@ -692,7 +143,8 @@ cudaError_t launch_gemv_rowblock_ex(const uint16_t* const* xs, int nx, int64_t M
     prm.slots = P.slots;
     prm.sg = P.sg;
     prm.three_d = P.three_d ? 1 : 0;
-    prm.ssc = (prm.groups * 2) % 16 == 0 ? 1 : 0;
+    // presets always stage their metadata (their K keeps every row 16-byte aligned)
+    prm.ssc = fmt != FMT_G64 || (prm.groups * 2) % 16 == 0 ? 1 : 0;
     prm.srow = P.srow;
     prm.slot_bytes = P.slot_bytes;
     prm.s_off = P.s_off;
@@ -700,6 +152,7 @@ cudaError_t launch_gemv_rowblock_ex(const uint16_t* const* xs, int nx, int64_t M
     prm.bar_off = P.bar_off;
     prm.red_stride = P.red_stride;
     prm.nx = nx;
+    prm.nsb = static_cast<int>(K / 256);
     prm.yh = y_half ? 1 : 0;
     prm.epi = epilogue;
     prm.status = device_status_ptr();
@@ -709,14 +162,11 @@ cudaError_t launch_gemv_rowblock_ex(const uint16_t* const* xs, int nx, int64_t M
         codes[i] = w[i].codes;
         prm.scales[i] = w[i].scales;
         prm.y[i] = w[i].y;
+        prm.sup[i] = fmt == FMT_P4A ? sup[i] : nullptr;
     }
-    if (bits == 4)
-        return M <= 8    ? rb_dispatch_ssc<4, 1>(prm, P, x, codes, nmat, s)
-               : M <= 16 ? rb_dispatch_ssc<4, 2>(prm, P, x, codes, nmat, s)
-                         : rb_dispatch_ssc<4, 4>(prm, P, x, codes, nmat, s);
-    return M <= 8    ? rb_dispatch_ssc<8, 1>(prm, P, x, codes, nmat, s)
-           : M <= 16 ? rb_dispatch_ssc<8, 2>(prm, P, x, codes, nmat, s)
-                     : rb_dispatch_ssc<8, 4>(prm, P, x, codes, nmat, s);
+    if (fmt == FMT_P8) return rb_run_p8(prm, P, x, codes, nmat, s);
+    if (fmt == FMT_P4A) return rb_run_p4a(prm, P, x, codes, nmat, s);
+    return bits == 4 ? rb_run_g64_4(prm, P, x, codes, nmat, s) : rb_run_g64_8(prm, P, x, codes, nmat, s);
 }
 
 }  // namespace rq

@@ -48,7 +48,7 @@ cudaError_t launch_gemv_cluster(const uint16_t* x, int64_t M, int64_t K, int64_t
 // K (each CTA keeps the x of its K range on chip).
 bool gemv_cluster_fits(int64_t M, int64_t K, int bits);
 
-// Decode product (M <= 16), row blocks over the full K range: every output is
+// Decode product (M <= 32), row blocks over the full K range: every output is
 // finished inside one CTA.  Needs no workspace.
 cudaError_t launch_gemv_rowblock(const uint16_t* x, int64_t M, int64_t K, int64_t N, int bits,
                                  const WOperand* w, int nmat, cudaStream_t s);
@@ -60,8 +60,22 @@ cudaError_t launch_gemv_rowblock_ex(const uint16_t* const* xs, int nx, int64_t M
                                     int64_t N, int bits, const WOperand* w, int nmat, bool y_half,
                                     int epilogue, cudaStream_t s);
 
-// Whether the row-block kernel takes a product of this shape.
-bool gemv_rowblock_fits(int64_t M, int64_t K, int64_t N, int bits, int nmat);
+// Weight formats of the row-block kernel: the symmetric group-64 format, and
+// the two rwkv-quant presets (int8 symmetric in groups of 16: codes int8
+// [N, K], scales fp16 [N, K/16], K % 128 == 0; int4 asymmetric in groups of
+// 32 under super-blocks of 256: codes u8 [N, K/2], sub-codes u8 [N, K/32, 2]
+// in place of the scales, (ds, dm) fp16 [N, K/256, 2], K % 256 == 0).
+constexpr int FMT_G64 = 0, FMT_P8 = 1, FMT_P4A = 2;
+
+// The row-block kernel for weights of format fmt (bits 8 for FMT_P8, 4 for
+// FMT_P4A); sup[i]: the (ds, dm) pairs of matrix i for FMT_P4A, else unused.
+cudaError_t launch_gemv_rowblock_fmt(const uint16_t* const* xs, int nx, int64_t M, int64_t K,
+                                     int64_t N, int bits, int fmt, const WOperand* w,
+                                     const uint32_t* const* sup, int nmat, bool y_half,
+                                     int epilogue, cudaStream_t s);
+
+// Whether the row-block kernel takes a product of this shape and format.
+bool gemv_rowblock_fits(int64_t M, int64_t K, int64_t N, int bits, int nmat, int fmt = FMT_G64);
 
 // The decode kernel a product of this shape runs on: RQ_DECODE_ROWTILE,
 // RQ_DECODE_CLUSTER or RQ_DECODE_ROWBLOCK (the selection of
@@ -123,6 +137,9 @@ bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
 bool pdl_enabled();
 
 // Device address of the library status word on the current device.
+// SMs of the current device (148 when it cannot be queried), cached per device.
+int num_sms();
+
 int* device_status_ptr();
 
 // Time limit of every bounded on-chip wait, in nanoseconds.

@@ -407,17 +407,6 @@ struct TcChoice {
     int ksplit;   // cluster size along K
 };
 
-static int num_sms() {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
-    return sms;
-}
-
 static TcChoice choose(int64_t M, int64_t N, int64_t K, int nmat) {
     TcChoice c;
     if (M <= 16) c.bnt = 16;

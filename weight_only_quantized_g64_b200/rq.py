@@ -76,6 +76,10 @@ def lib():
     L.rq_quantize_p8_g16.restype = i32
     L.rq_quantize_p4a_g32.argtypes = [vp, i64, i64, vp, vp, i32, vp, vp, vp, vp, vp, vp]
     L.rq_quantize_p4a_g32.restype = i32
+    L.rq_gemv_p8_g16.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp]
+    L.rq_gemv_p8_g16.restype = i32
+    L.rq_gemv_p4a_g32.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp]
+    L.rq_gemv_p4a_g32.restype = i32
     L.rq_set_pdl.argtypes = [i32]
     L.rq_set_pdl.restype = i32
     L.rq_set_decode_kernel.argtypes = [i32]
@@ -228,6 +232,27 @@ def gemv_wq(x: torch.Tensor, codes, scales, N: int, bits: int, y=None, stream=No
         y = torch.empty((M, N), dtype=torch.float32, device=x.device)
     _check(lib().rq_gemv_wq(_p(x), M, K, _p(codes), _p(scales), N, bits, _p(y), _stream(stream)),
            "rq_gemv_wq")
+    return y
+
+
+def gemv_p8_g16(x: torch.Tensor, codes, scales, N: int, y=None, stream=None):
+    """Decode product of the int8 preset (codes [N, K], scales fp16 [N, K/16])."""
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _check(lib().rq_gemv_p8_g16(_p(x), M, K, _p(codes), _p(scales), N, _p(y), _stream(stream)),
+           "rq_gemv_p8_g16")
+    return y
+
+
+def gemv_p4a_g32(x: torch.Tensor, codes, sub, sup, N: int, y=None, stream=None):
+    """Decode product of the int4 asymmetric preset (codes [N, K/2], sub
+    [N, K/32, 2], sup fp16 [N, K/256, 2])."""
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _check(lib().rq_gemv_p4a_g32(_p(x), M, K, _p(codes), _p(sub), _p(sup), N, _p(y),
+                                 _stream(stream)), "rq_gemv_p4a_g32")
     return y
 
 
