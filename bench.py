@@ -53,7 +53,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # (comments and whitespace ignored) differs, the bench reports traffic as null
 # until a new capture is taken.
 DECODE_SOURCES = ("rq_api.cu", "rq_gemv.cu", "rq_gemv_ck.cu", "rq_gemv_unit.cuh", "rq_ptx.cuh",
-                  "rq_internal.h")
+                  "rq_internal.h", "rq_gemv_rb.cuh", "rq_gemv_rb.cu", "rq_gemv_rb_g64_4.cu",
+                  "rq_gemv_rb_g64_8.cu")
+KERNEL_NAMES = {"rowtile": "gemv_wq_kernel (row tiles)", "cluster": "gemv_ck_kernel (cluster split-K)",
+                "rowblock": "gemv_rb_kernel (row blocks)"}
 DECODE_TRAFFIC = {"code_sha256_16": "076aa3b7224c42d8", "bytes_per_launch": 6823383}
 
 
@@ -203,6 +206,17 @@ class DecodeStack:
         self.bytes_per_pass = wl.layers * sum(
             synth.algorithmic_weight_bytes(p.N, p.K, wl.bits) for p in wl.projs)
         self.launches_per_pass = wl.layers * 4
+
+    def kernels(self):
+        """{decode kernel: [launch names]} that one pass at each M runs on."""
+        wl, out = self.wl, {}
+        shapes = [("rkv", wl.projs[0], 3), ("o", wl.projs[3], 1), ("key", wl.projs[4], 1),
+                  ("value", wl.projs[5], 1)]
+        for M in wl.Ms:
+            for name, p, nmat in shapes:
+                k = rq.decode_kernel_for(M, p.K, p.N, wl.bits, nmat)
+                out.setdefault(k, []).append(f"{name}@M{M}")
+        return out
 
     def buffers(self, M):
         wl = self.wl
@@ -616,8 +630,9 @@ def main():
             "per_M": per_m,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": decode_traffic(),
-                         "kernel": "decode products (fused RKV + O + key + value, all M): "
-                                   "gemv_wq_kernel (row tiles) and gemv_ck_kernel (cluster split-K)",
+                         "kernel": "decode products (fused RKV + O + key + value, all M): " +
+                                   ", ".join(f"{KERNEL_NAMES[k]} x{len(v)}" for k, v in
+                                             sorted(stack.kernels().items())),
                          "bytes_per_launch": bytes_per_step / launches_per_step,
                          "us_per_launch": ms_per_step * 1e3 / launches_per_step,
                          "peak_kind": peak_kind + " copy bandwidth"},

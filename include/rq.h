@@ -385,18 +385,25 @@ rq_status rq_set_pdl(int enable);
  *                          each CTA's x held in shared memory, partial sums
  *                          added through distributed shared memory;
  *   RQ_DECODE_ROWBLOCK (3) blocks of rows over the full K range, each output
- *                          finished inside one CTA; needs no workspace.
+ *                          finished inside one CTA; needs no workspace;
+ *   RQ_DECODE_TENSOR   (4) the fifth-generation tensor cores (tcgen05):
+ *                          weights dequantised to fp16(code * s16) in tensor
+ *                          memory, 256-row blocks with K split over a
+ *                          thread-block cluster, partial sums added through
+ *                          distributed shared memory; needs no workspace.
  * Any other value is rejected with RQ_ERR_RANGE.  Not thread-safe.
  */
 #define RQ_DECODE_AUTO 0
 #define RQ_DECODE_ROWTILE 1
 #define RQ_DECODE_CLUSTER 2
 #define RQ_DECODE_ROWBLOCK 3
+#define RQ_DECODE_TENSOR 4
 rq_status rq_set_decode_kernel(int kernel);
 
 /*
  * rq_decode_kernel_for -- which decode kernel (RQ_DECODE_ROWTILE,
- * RQ_DECODE_CLUSTER or RQ_DECODE_ROWBLOCK) a decode product of this shape would run on under the
+ * RQ_DECODE_CLUSTER, RQ_DECODE_ROWBLOCK or RQ_DECODE_TENSOR) a decode
+ * product of this shape would run on under the
  * current rq_set_decode_kernel selection; nmat is 1 (rq_gemv_wq) or 3
  * (rq_rkv_fused).  Host-only: launches nothing and needs no GPU.  The same
  * argument checks as the products (RQ_ERR_BITS, RQ_ERR_SHAPE); kernel NULL

@@ -88,8 +88,9 @@ def test_control_calls(L):
     assert L.rq_set_wait_limit_ns(0) == rq.ERR_RANGE
     assert L.rq_set_wait_limit_ns(10**9) == rq.OK
     assert L.rq_set_pdl(0) == rq.OK
-    # decode kernel selection: 0 automatic, 1 row tiles, 2 cluster split-K, 3 row blocks
-    for bad in (-1, 4, 1 << 20):
+    # decode kernel selection: 0 automatic, 1 row tiles, 2 cluster split-K, 3 row
+    # blocks, 4 tensor cores
+    for bad in (-1, 5, 1 << 20):
         assert L.rq_set_decode_kernel(bad) == rq.ERR_RANGE
     for kind, code in rq.DECODE_KERNELS.items():
         assert L.rq_set_decode_kernel(code) == rq.OK
@@ -131,10 +132,11 @@ def test_decode_kernel_choice(L):
             for M in (1, 16, 32):
                 assert rq.decode_kernel_for(M, D, D, 8, 1) == kind
     assert rq.decode_kernel_for(1, D, D, 4, 1) == "rowtile"
-    # a forced row-block selection takes every decode batch size
-    with rq.decode_kernel("rowblock"):
-        for M in (1, 9, 16, 17, 32):
-            assert rq.decode_kernel_for(M, D, D, 4, 3) == "rowblock"
+    # forced row-block and tensor-core selections take every decode batch size
+    for kind in ("rowblock", "tensor"):
+        with rq.decode_kernel(kind):
+            for M in (1, 9, 16, 17, 32):
+                assert rq.decode_kernel_for(M, D, D, 4, 3) == kind
     # argument checks
     out = ctypes.c_int()
     assert L.rq_decode_kernel_for(0, D, D, 4, 1, ctypes.byref(out)) == rq.ERR_SHAPE

@@ -47,14 +47,16 @@ def check(y, ref, budget, half, what):
     assert np.all(d <= lim), f"{what}: worst {d.max():.3e} (limit {lim.flat[d.argmax()]:.3e})"
 
 
+@pytest.mark.parametrize("kernel", ["rowblock", "tensor"])
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("M", [1, 3, 8, 13, 17, 32])
 @pytest.mark.parametrize("N,K", [(300, 640), (256, 2048), (129, 128)])
 @pytest.mark.parametrize("out,epi", [(torch.float32, 1), (torch.float16, 0), (torch.float16, 1)])
-def test_gemv_ex(bits, M, N, K, out, epi):
+def test_gemv_ex(kernel, bits, M, N, K, out, epi):
     x, codes, scales = case(N, K, bits, M, seed=4000 + M + N + K)
     cd, sd = up(codes, scales)
-    y = rq.gemv_wq_ex(x, cd, sd, N, bits, out_dtype=out, epilogue=epi)
+    with rq.decode_kernel(kernel):
+        y = rq.gemv_wq_ex(x, cd, sd, N, bits, out_dtype=out, epilogue=epi)
     torch.cuda.synchronize()
     y_ref, bound = oracle.matmul(x.cpu().numpy(), codes, scales, bits)
     delta = TOL * bound
@@ -70,22 +72,24 @@ def test_gemv_ex_plain_matches_gemv():
     """No epilogue, fp32 out: the same values as rq_gemv_wq on the row-block kernel."""
     x, codes, scales = case(512, 1024, 4, 8, seed=41)
     cd, sd = up(codes, scales)
-    y1 = rq.gemv_wq_ex(x, cd, sd, 512, 4)
     with rq.decode_kernel("rowblock"):
+        y1 = rq.gemv_wq_ex(x, cd, sd, 512, 4)
         y2 = rq.gemv_wq(x, cd, sd, 512, 4)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
 
 
+@pytest.mark.parametrize("kernel", ["rowblock", "tensor"])
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("M", [1, 8, 16, 32])
 @pytest.mark.parametrize("out", [torch.float32, torch.float16])
-def test_rkv_fused3(bits, M, out):
+def test_rkv_fused3(kernel, bits, M, out):
     N, K = 200, 512
     cases = [case(N, K, bits, M, seed=5000 + 10 * i + M) for i in range(3)]
     ws = [up(c[1], c[2]) for c in cases]
-    ys = rq.rkv_fused3(cases[0][0], cases[1][0], cases[2][0], ws[0], ws[1], ws[2], N, bits,
-                       out_dtype=out)
+    with rq.decode_kernel(kernel):
+        ys = rq.rkv_fused3(cases[0][0], cases[1][0], cases[2][0], ws[0], ws[1], ws[2], N, bits,
+                           out_dtype=out)
     torch.cuda.synchronize()
     for i in range(3):
         y_ref, bound = oracle.matmul(cases[i][0].cpu().numpy(), cases[i][1], cases[i][2], bits)

@@ -105,7 +105,7 @@ def product_case(N, K, bits, M, seed, massive=None):
     return x, codes, scales
 
 
-DECODE_KERNELS = ["rowtile", "cluster", "rowblock"]
+DECODE_KERNELS = ["rowtile", "cluster", "rowblock", "tensor"]
 
 
 def takes(kernel, M):
@@ -320,7 +320,8 @@ def test_bounded_wait_times_out_cleanly():
 
 
 @pytest.mark.parametrize("kernel,M", [("rowtile", 4), ("cluster", 4), ("cluster", 24),
-                                      ("rowblock", 4), ("rowblock", 13)])
+                                      ("rowblock", 4), ("rowblock", 13), ("tensor", 4),
+                                      ("tensor", 24)])
 def test_pdl_chain_matches(kernel, M):
     """With programmatic dependent launch on, a chain of dependent products
     (each reading the previous output as its input) still matches."""
@@ -353,19 +354,37 @@ def test_pdl_chain_matches(kernel, M):
 # ------------------------------------------------------------ repeatability ---
 
 @pytest.mark.parametrize("path", ["gemv", "gemv-cluster", "gemv-cluster-m32", "gemv-rowblock",
-                                  "gemv-rowblock-m16", "gemm"])
+                                  "gemv-rowblock-m16", "gemv-tensor", "gemv-tensor-m32",
+                                  "gemv-tensor-fused", "gemm"])
 def test_repeat_runs_bit_identical(path):
     """Every kernel sums in a fixed order, so repeated runs must agree bit for
     bit; a pipeline race (a stage read before or after its data) shows up here
     even when it stays within tolerance."""
     kernel = ("cluster" if path.startswith("gemv-cluster") else
-              "rowblock" if path.startswith("gemv-rowblock") else "rowtile")
+              "rowblock" if path.startswith("gemv-rowblock") else
+              "tensor" if path.startswith("gemv-tensor") else "rowtile")
+    if path == "gemv-tensor-fused":
+        # three matrices, partial row blocks across CTAs and matrices
+        N, K, M, bits = 2048, 2048, 24, 4
+        qs = [rq.quantize_g64(synth.weights(N, K, seed=33 + i, device="cuda"), bits) for i in range(3)]
+        x = synth.activations(M, K, seed=33, device="cuda")
+        with rq.decode_kernel(kernel):
+            ref = rq.rkv_fused(x, *qs, N, bits)
+            torch.cuda.synchronize()
+            for _ in range(20):
+                ys = rq.rkv_fused(x, *qs, N, bits)
+                torch.cuda.synchronize()
+                for a, b in zip(ys, ref):
+                    assert torch.equal(a.view(torch.int32), b.view(torch.int32)), path
+        return
     if path == "gemm":
         N, K, M, bits = 1024, 8192, 512, 4
     elif path == "gemv-cluster-m32":
         N, K, M, bits = 2048, 8192, 32, 4
     elif path == "gemv-rowblock-m16":
         N, K, M, bits = 16384, 4096, 16, 4
+    elif path == "gemv-tensor-m32":
+        N, K, M, bits = 16384, 4096, 32, 4
     else:
         N, K, M, bits = 4096, 4096, 5, 4
     W = synth.weights(N, K, seed=31, device="cuda")

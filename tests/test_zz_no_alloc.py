@@ -33,7 +33,7 @@ def _oracle(x, codes, scales, bits):
                          scales.cpu().numpy().view(np.uint16), bits)
 
 
-@pytest.mark.parametrize("kernel", ["auto", "rowtile", "cluster", "rowblock"])
+@pytest.mark.parametrize("kernel", ["auto", "rowtile", "cluster", "rowblock", "tensor"])
 @pytest.mark.parametrize("N,K,M,bits", [(4096, 4096, 1, 4), (2048, 8192, 8, 4),
                                         (300, 640, 17, 4), (2560, 2560, 32, 8),
                                         (129, 128, 3, 8), (4096, 2048, 32, 4)])

@@ -45,6 +45,7 @@ int decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat) {
     if (g_decode_kernel == RQ_DECODE_ROWTILE) return RQ_DECODE_ROWTILE;
     if (g_decode_kernel == RQ_DECODE_ROWBLOCK)
         return gemv_rowblock_fits(M, K, N, bits, nmat) ? RQ_DECODE_ROWBLOCK : -1;
+    if (g_decode_kernel == RQ_DECODE_TENSOR) return tcs_fits(M, K, N, bits) ? RQ_DECODE_TENSOR : -1;
     // measured on B200 (graph-replayed chains, int4): the row-block kernel
     // is ahead at every M once the launch has at least one 16-row m-tile per
     // SM; below that (its CTAs would leave SMs idle) the row-tile kernel,
@@ -212,10 +213,28 @@ static rq_status launch_decode(const uint16_t* x, int64_t M, int64_t K, int64_t 
                                const WOperand* w, int nmat, cudaStream_t s) {
     const int which = decode_kernel_for(M, K, N, bits, nmat);
     if (which < 0) return RQ_ERR_SHAPE;
+    const uint16_t* xs[1] = {x};
     const cudaError_t e =
         which == RQ_DECODE_CLUSTER    ? launch_gemv_cluster(x, M, K, N, bits, w, nmat, s)
         : which == RQ_DECODE_ROWBLOCK ? launch_gemv_rowblock(x, M, K, N, bits, w, nmat, s)
+        : which == RQ_DECODE_TENSOR   ? launch_tcs(xs, 1, M, K, N, bits, w, nmat, false, 0, s)
                                       : launch_gemv_product(x, M, K, N, bits, w, nmat, s);
+    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+}
+
+// The decode variants (per-matrix inputs, fp16 output, fused epilogue) run on
+// the tensor-core kernel when the selection (or the automatic choice) names
+// it, else on the row-block kernel.
+static rq_status launch_decode_ex(const uint16_t* const* xs, int nx, int64_t M, int64_t K,
+                                  int64_t N, int bits, const WOperand* w, int nmat, bool y_half,
+                                  int epilogue, cudaStream_t s) {
+    cudaError_t e;
+    if (decode_kernel_for(M, K, N, bits, nmat) == RQ_DECODE_TENSOR)
+        e = launch_tcs(xs, nx, M, K, N, bits, w, nmat, y_half, epilogue, s);
+    else if (gemv_rowblock_fits(M, K, N, bits, nmat))
+        e = launch_gemv_rowblock_ex(xs, nx, M, K, N, bits, w, nmat, y_half, epilogue, s);
+    else
+        return RQ_ERR_SHAPE;
     return e == cudaSuccess ? RQ_OK : cuda_fail(e);
 }
 
@@ -363,12 +382,10 @@ rq_status rq_gemv_wq_ex(const uint16_t* x, int64_t M, int64_t K, const void* cod
     if (out_dtype != RQ_OUT_F32 && out_dtype != RQ_OUT_F16) return RQ_ERR_RANGE;
     if (epilogue != RQ_EPI_NONE && epilogue != RQ_EPI_RELU_SQ) return RQ_ERR_RANGE;
     if ((st = check_operand(codes, scales, static_cast<const float*>(y))) != RQ_OK) return st;
-    if (!gemv_rowblock_fits(M, K, N, bits, 1)) return RQ_ERR_SHAPE;
     WOperand w = {codes, scales, static_cast<float*>(y)};
     const uint16_t* xs[1] = {x};
-    const cudaError_t e = launch_gemv_rowblock_ex(xs, 1, M, K, N, bits, &w, 1, out_dtype == RQ_OUT_F16,
-                                                  epilogue, reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+    return launch_decode_ex(xs, 1, M, K, N, bits, &w, 1, out_dtype == RQ_OUT_F16, epilogue,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 rq_status rq_rkv_fused3(const uint16_t* x_r, const uint16_t* x_k, const uint16_t* x_v, int64_t M,
@@ -384,14 +401,12 @@ rq_status rq_rkv_fused3(const uint16_t* x_r, const uint16_t* x_k, const uint16_t
     if ((st = check_operand(codes_r, scales_r, static_cast<const float*>(y_r))) != RQ_OK) return st;
     if ((st = check_operand(codes_k, scales_k, static_cast<const float*>(y_k))) != RQ_OK) return st;
     if ((st = check_operand(codes_v, scales_v, static_cast<const float*>(y_v))) != RQ_OK) return st;
-    if (!gemv_rowblock_fits(M, K, N, bits, 3)) return RQ_ERR_SHAPE;
     WOperand w[3] = {{codes_r, scales_r, static_cast<float*>(y_r)},
                      {codes_k, scales_k, static_cast<float*>(y_k)},
                      {codes_v, scales_v, static_cast<float*>(y_v)}};
     const uint16_t* xs[3] = {x_r, x_k, x_v};
-    const cudaError_t e = launch_gemv_rowblock_ex(xs, 3, M, K, N, bits, w, 3, out_dtype == RQ_OUT_F16,
-                                                  RQ_EPI_NONE, reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? RQ_OK : cuda_fail(e);
+    return launch_decode_ex(xs, 3, M, K, N, bits, w, 3, out_dtype == RQ_OUT_F16, RQ_EPI_NONE,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 rq_status rq_gemv_p8_g16(const uint16_t* x, int64_t M, int64_t K, const void* codes,
@@ -444,7 +459,7 @@ rq_status rq_set_pdl(int enable) {
 
 rq_status rq_set_decode_kernel(int kernel) {
     if (kernel != RQ_DECODE_AUTO && kernel != RQ_DECODE_ROWTILE && kernel != RQ_DECODE_CLUSTER &&
-        kernel != RQ_DECODE_ROWBLOCK)
+        kernel != RQ_DECODE_ROWBLOCK && kernel != RQ_DECODE_TENSOR)
         return RQ_ERR_RANGE;
     g_decode_kernel = kernel;
     return RQ_OK;

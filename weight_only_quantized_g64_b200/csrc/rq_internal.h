@@ -74,11 +74,22 @@ cudaError_t launch_gemv_rowblock_fmt(const uint16_t* const* xs, int nx, int64_t 
                                      const uint32_t* const* sup, int nmat, bool y_half,
                                      int epilogue, cudaStream_t s);
 
+// Streaming tensor-core product for 1 <= M <= 64 (tcgen05, dequantised
+// weights in TMEM, 256-row blocks with K split over a thread-block cluster,
+// partial sums added through distributed shared memory; needs no workspace).
+// Inputs and outputs as launch_gemv_rowblock_ex.
+cudaError_t launch_tcs(const uint16_t* const* xs, int nx, int64_t M, int64_t K, int64_t N,
+                       int bits, const WOperand* w, int nmat, bool y_half, int epilogue,
+                       cudaStream_t s);
+bool tcs_fits(int64_t M, int64_t K, int64_t N, int bits);
+// Its K split (cluster size) for a shape.
+int tcs_ksplit(int64_t K, int64_t N, int nmat);
+
 // Whether the row-block kernel takes a product of this shape and format.
 bool gemv_rowblock_fits(int64_t M, int64_t K, int64_t N, int bits, int nmat, int fmt = FMT_G64);
 
 // The decode kernel a product of this shape runs on: RQ_DECODE_ROWTILE,
-// RQ_DECODE_CLUSTER or RQ_DECODE_ROWBLOCK (the selection of
+// RQ_DECODE_CLUSTER, RQ_DECODE_ROWBLOCK or RQ_DECODE_TENSOR (the selection of
 // rq_set_decode_kernel, or the automatic choice), or -1 when the selected
 // kernel cannot take the shape.
 int decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat);

@@ -78,10 +78,12 @@ extern "C" rq_status rq_gemv_wq_noalloc(const uint16_t* x, int64_t M, int64_t K,
     WOperand w = {codes, scales, y};
     const int which = decode_kernel_for(M, K, N, bits, 1);
     if (which < 0) return RQ_ERR_SHAPE;
-    if (which == RQ_DECODE_CLUSTER || which == RQ_DECODE_ROWBLOCK) {
+    if (which == RQ_DECODE_CLUSTER || which == RQ_DECODE_ROWBLOCK || which == RQ_DECODE_TENSOR) {
         // these kernels keep their partial sums on chip: no scratch at all
-        cudaError_t ec = which == RQ_DECODE_CLUSTER ? launch_gemv_cluster(x, M, K, N, bits, &w, 1, s)
-                                                    : launch_gemv_rowblock(x, M, K, N, bits, &w, 1, s);
+        const uint16_t* xs[1] = {x};
+        cudaError_t ec = which == RQ_DECODE_CLUSTER  ? launch_gemv_cluster(x, M, K, N, bits, &w, 1, s)
+                         : which == RQ_DECODE_TENSOR ? launch_tcs(xs, 1, M, K, N, bits, &w, 1, false, 0, s)
+                                                     : launch_gemv_rowblock(x, M, K, N, bits, &w, 1, s);
         if (ec != cudaSuccess) {
             record_cuda_error(ec);
             return RQ_ERR_CUDA;

@@ -22,7 +22,7 @@ MAX_DECODE_M = 32
 STATUS = {0: "RQ_OK", 1: "RQ_ERR_NULL", 2: "RQ_ERR_BITS", 3: "RQ_ERR_SHAPE", 4: "RQ_ERR_ALIGN",
           5: "RQ_ERR_NONFINITE", 6: "RQ_ERR_RANGE", 7: "RQ_ERR_TIMEOUT", 8: "RQ_ERR_CUDA"}
 OK, ERR_NULL, ERR_BITS, ERR_SHAPE, ERR_ALIGN, ERR_NONFINITE, ERR_RANGE, ERR_TIMEOUT, ERR_CUDA = range(9)
-DECODE_KERNELS = {"auto": 0, "rowtile": 1, "cluster": 2, "rowblock": 3}
+DECODE_KERNELS = {"auto": 0, "rowtile": 1, "cluster": 2, "rowblock": 3, "tensor": 4}
 
 _lib = None
 
@@ -328,7 +328,7 @@ def set_decode_kernel(kind: str):
 
 
 def decode_kernel_for(M: int, K: int, N: int, bits: int, nmat: int = 1) -> str:
-    """The decode kernel ("rowtile", "cluster" or "rowblock") a product of this shape runs on."""
+    """The decode kernel ("rowtile", "cluster", "rowblock" or "tensor") a product of this shape runs on."""
     out = ctypes.c_int(-1)
     _check(lib().rq_decode_kernel_for(M, K, N, bits, nmat, ctypes.byref(out)), "rq_decode_kernel_for")
     return {v: k for k, v in DECODE_KERNELS.items()}[out.value]
