@@ -11,10 +11,12 @@
 // built with fast-math.
 //
 // Layout of the work: groups of W are contiguous (row-major W, K % 64 == 0),
-// so the kernel runs flat over all N*K/64 groups.  16 threads own one group
-// (four fp32 each, one 16-byte load), a warp two groups; the group max is a
-// 4-step xor-shuffle inside the 16-lane half.  Bandwidth-bound: 256 B read,
-// 34 B (int4) or 66 B (int8) written per group.
+// so the kernel runs flat over all N*K/64 groups.  8 threads own one group
+// (eight fp32 each, two 16-byte loads, each load instruction covering whole
+// 128-byte lines), a warp four groups; the group max is a 3-step
+// xor-shuffle inside the 8-lane team, so the per-group work (the max, the
+// division, the fp16 rounding, the reciprocal) is shared by 8 weights per
+// lane.  256 B read, 34 B (int4) or 66 B (int8) written per group.
 #include "rq_internal.h"
 #include "rq_ptx.cuh"
 
@@ -37,51 +39,85 @@ __device__ __forceinline__ int rint_quotient(float w, float sf, float r) {
     return __float2int_rn(__fdiv_rn(w, sf));
 }
 
-// One group held by a half-warp, four weights per lane: scale bits, codes,
-// status (0, 5 = NONFINITE, 6 = RANGE).
+// max that propagates NaN (the PTX max.NaN), so one reduction also tells
+// whether the group holds a non-finite weight.
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float d;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+
+// clamp(rint(fl(w / sf)), +-QMAX) without a division where that is provably
+// the same value: t = w * r (r = 1/sf rounded to nearest) lies within
+// |q| * 2^-23 (1 + 2^-25) of the exact quotient q and fl(q) within |q| * 2^-24
+// of it, so when t (clamped to +-QMAX, which both sides would clamp to) is
+// more than (QMAX + 1) * 2^-21 away from every half-integer, no half-integer
+// separates it from fl(q).  Near ties (weights on the grid) take the IEEE
+// division.  Rounding: t + 1.5 * 2^23 rounds to an integer, ties to even, for
+// |t| <= 2^22; its bit pattern minus that of 1.5 * 2^23 is the integer.
+template <int QMAX>
+__device__ __forceinline__ int rint_quotient_q(float w, float sf, float r) {
+    constexpr float kNear = static_cast<float>(QMAX + 1) * 4.76837158203125e-7f;   // 2^-21
+    constexpr float kMagic = 12582912.0f;                                          // 1.5 * 2^23
+    const float t = fminf(fmaxf(__fmul_rn(w, r), static_cast<float>(-QMAX)), static_cast<float>(QMAX));
+    const float m = __fadd_rn(t, kMagic);
+    const float d = __fsub_rn(t, __fsub_rn(m, kMagic));
+    if (fabsf(__fsub_rn(fabsf(d), 0.5f)) > kNear) return __float_as_int(m) - __float_as_int(kMagic);
+    return max(-QMAX, min(QMAX, __float2int_rn(__fdiv_rn(w, sf))));
+}
+
+// One group held by 8 lanes, 8 weights per lane (positions 4l..4l+3 and
+// 32+4l..32+4l+3 of the group): scale bits, codes, status (0, 5 = NONFINITE,
+// 6 = RANGE).
 template <int BITS>
-__device__ __forceinline__ void quantize_group16(const float4 v, unsigned half_mask,
-                                                 uint16_t& s_bits, int (&c)[4], int& status) {
+__device__ __forceinline__ void quantize_group8(const float4 (&v)[2], unsigned mask8,
+                                                uint16_t& s_bits, int (&c)[8], int& status) {
     constexpr int kQmax = BITS == 4 ? 7 : 127;
-    const bool finite = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
-    float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    const float w[8] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w};
+    float a = 0.0f;
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(half_mask, a, off));
-    const bool all_finite = __all_sync(half_mask, finite);
+    for (int i = 0; i < 8; ++i) a = max_nan(a, fabsf(w[i]));
+#pragma unroll
+    for (int off = 4; off > 0; off >>= 1) a = max_nan(a, __shfl_xor_sync(mask8, a, off));
+    // a is NaN or +inf exactly when the group holds a non-finite weight
 
     const float s32 = __fdiv_rn(a, static_cast<float>(kQmax));
     const __half s16 = __float2half_rn(s32);
     s_bits = __half_as_ushort(s16);
     const float sf = __half2float(s16);
     status = 0;
-    c[0] = c[1] = c[2] = c[3] = 0;
-    if (!all_finite) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = 0;
+    if (!isfinite(a)) {
         s_bits = 0x7E00u;
         status = 5;  // RQ_ERR_NONFINITE
     } else if (s_bits == 0x7C00u) {
         status = 6;  // RQ_ERR_RANGE
     } else if (sf != 0.0f) {
         const float r = __frcp_rn(sf);
-        const float w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) c[i] = max(-kQmax, min(kQmax, rint_quotient(w[i], sf, r)));
+        for (int i = 0; i < 8; ++i) c[i] = rint_quotient_q<kQmax>(w[i], sf, r);
     }
 }
 
 template <int BITS>
-__device__ __forceinline__ void store_group16(int64_t gid, int lane16, uint16_t s_bits,
-                                              const int (&c)[4], uint8_t* __restrict__ codes,
-                                              uint16_t* __restrict__ scales) {
-    if (BITS == 4) {
-        const uint16_t packed = static_cast<uint16_t>((c[0] & 0xF) | ((c[1] & 0xF) << 4) |
-                                                      ((c[2] & 0xF) << 8) | ((c[3] & 0xF) << 12));
-        __stcs(reinterpret_cast<unsigned short*>(codes + gid * 32 + lane16 * 2), packed);
-    } else {
-        const uint32_t packed = (c[0] & 0xFF) | ((c[1] & 0xFF) << 8) | ((c[2] & 0xFF) << 16) |
-                                (static_cast<uint32_t>(c[3] & 0xFF) << 24);
-        __stcs(reinterpret_cast<unsigned int*>(codes + gid * 64 + lane16 * 4), packed);
+__device__ __forceinline__ void store_group8(int64_t gid, int l8, uint16_t s_bits, const int (&c)[8],
+                                             uint8_t* __restrict__ codes,
+                                             uint16_t* __restrict__ scales) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int* ch = c + 4 * h;
+        if (BITS == 4) {
+            const uint16_t packed = static_cast<uint16_t>((ch[0] & 0xF) | ((ch[1] & 0xF) << 4) |
+                                                          ((ch[2] & 0xF) << 8) | ((ch[3] & 0xF) << 12));
+            __stcs(reinterpret_cast<unsigned short*>(codes + gid * 32 + h * 16 + l8 * 2), packed);
+        } else {
+            const uint32_t packed = (ch[0] & 0xFF) | ((ch[1] & 0xFF) << 8) | ((ch[2] & 0xFF) << 16) |
+                                    (static_cast<uint32_t>(ch[3] & 0xFF) << 24);
+            __stcs(reinterpret_cast<unsigned int*>(codes + gid * 64 + h * 32 + l8 * 4), packed);
+        }
     }
-    if (lane16 == 0) scales[gid] = s_bits;
+    if (l8 == 0) scales[gid] = s_bits;
 }
 
 // NONFINITE overrides everything; RANGE only replaces OK.
@@ -91,9 +127,10 @@ __device__ __forceinline__ void raise_status(int* dev_status, int status) {
     else if (status == 6) atomicCAS(dev_status, 0, 6);
 }
 
-// Half-warp h takes groups h + H*(kQU*i + j), j < kQU, for i = 0, 1, ...
-// (H = half-warps in the grid): the kQU groups' loads are issued together.
-constexpr int kQU = 4;
+// Eight lanes per group, four groups per warp.  An 8-lane team takes groups
+// t + T*(kQU*i + j), j < kQU, for i = 0, 1, ... (T = teams in the grid): the
+// kQU groups' loads (two 16-byte loads per lane each) are issued together.
+constexpr int kQU = 2;
 
 template <int BITS>
 __global__ void __launch_bounds__(256) quantize_g64_kernel(const float4* __restrict__ W,
@@ -101,30 +138,32 @@ __global__ void __launch_bounds__(256) quantize_g64_kernel(const float4* __restr
                                                            uint8_t* __restrict__ codes,
                                                            uint16_t* __restrict__ scales,
                                                            int* __restrict__ dev_status) {
-    const int lane16 = threadIdx.x & 15;
-    const unsigned half_mask = 0xFFFFu << (threadIdx.x & 16);
-    const int64_t first = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
-    const int64_t step = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
+    const int l8 = threadIdx.x & 7;
+    const unsigned mask8 = 0xFFu << (threadIdx.x & 24);
+    const int64_t first = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 3;
+    const int64_t step = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 3;
 
     for (int64_t g0 = first; g0 < n_groups; g0 += kQU * step) {
-        float4 v[kQU];
+        float4 v[kQU][2];
 #pragma unroll
         for (int j = 0; j < kQU; ++j) {
             const int64_t gid = g0 + j * step;
-            v[j] = gid < n_groups ? __ldcs(&W[gid * 16 + lane16]) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                v[j][h] = gid < n_groups ? __ldcs(&W[gid * 16 + h * 8 + l8]) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         int status_any = 0;
 #pragma unroll
         for (int j = 0; j < kQU; ++j) {
             const int64_t gid = g0 + j * step;
-            if (gid >= n_groups) break;   // uniform over the half-warp
+            if (gid >= n_groups) break;   // uniform over the team
             uint16_t s_bits;
-            int c[4], status;
-            quantize_group16<BITS>(v[j], half_mask, s_bits, c, status);
-            store_group16<BITS>(gid, lane16, s_bits, c, codes, scales);
+            int c[8], status;
+            quantize_group8<BITS>(v[j], mask8, s_bits, c, status);
+            store_group8<BITS>(gid, l8, s_bits, c, codes, scales);
             if (status == 5 || (status == 6 && status_any == 0)) status_any = status;
         }
-        if (lane16 == 0 && status_any != 0) raise_status(dev_status, status_any);
+        if (l8 == 0 && status_any != 0) raise_status(dev_status, status_any);
     }
 }
 
@@ -138,7 +177,7 @@ static int quantize_grid(int64_t n_groups, const void* kern) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0) != cudaSuccess ||
         per_sm <= 0)
         per_sm = 1;
-    const int64_t need = (n_groups + 15) / 16;
+    const int64_t need = (n_groups + 31) / 32;
     const int64_t full = static_cast<int64_t>(sms) * per_sm;
     return static_cast<int>(need < full ? need : full);
 }
