@@ -54,9 +54,9 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # until a new capture is taken.
 DECODE_SOURCES = ("rq_api.cu", "rq_gemv.cu", "rq_gemv_ck.cu", "rq_gemv_unit.cuh", "rq_ptx.cuh",
                   "rq_internal.h", "rq_gemv_rb.cuh", "rq_gemv_rb.cu", "rq_gemv_rb_g64_4.cu",
-                  "rq_gemv_rb_g64_8.cu")
+                  "rq_gemv_rb_g64_8.cu", "rq_tcs.cu")
 KERNEL_NAMES = {"rowtile": "gemv_wq_kernel (row tiles)", "cluster": "gemv_ck_kernel (cluster split-K)",
-                "rowblock": "gemv_rb_kernel (row blocks)"}
+                "rowblock": "gemv_rb_kernel (row blocks)", "tensor": "tcs_kernel (tcgen05, K split over a cluster)"}
 DECODE_TRAFFIC = {"code_sha256_16": "076aa3b7224c42d8", "bytes_per_launch": 6823383}
 
 
@@ -496,7 +496,7 @@ def main():
     ap.add_argument("--M", type=int, default=1, help="batch of --case")
     ap.add_argument("--bits", type=int, default=4, choices=[4, 8], help="bits of --case")
     ap.add_argument("--repeat", type=int, default=2, help="calls of --case")
-    ap.add_argument("--decode-kernel", default="auto", choices=["auto", "rowtile", "cluster", "rowblock"],
+    ap.add_argument("--decode-kernel", default="auto", choices=sorted(rq.DECODE_KERNELS),
                     help="decode kernel of --case gemv/rkv")
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--skip-extras", action="store_true",

@@ -106,10 +106,12 @@ def test_control_calls(L):
 
 def test_decode_kernel_choice(L):
     """The automatic choice between the decode kernels (host logic, no GPU,
-    so the SM count is taken as 148): the row-block kernel at every M for
-    launches of at least one 16-row m-tile per SM (the fused R/K/V and the
-    channel-mix key of the 1.5B-shaped layer); below that the row-tile kernel
-    for M <= 16 and the cluster kernel for M > 16."""
+    so the SM count is taken as 148).  Launches with at least one 16-row
+    m-tile per SM (the fused R/K/V and the channel-mix key of the 1.5B-shaped
+    layer, every projection of the 13.3B-shaped one): the row-block kernel,
+    except M > 16 on rows of >= 16384 k (the tensor-core kernel).  Fewer
+    m-tiles: row tiles for M <= 8, row blocks for M 9..16 and for M > 16 on
+    rows of <= 4096 k, the cluster kernel for M > 16 on longer rows."""
     D = 2048
     layer = {"rkv": (D, D, 3), "o": (D, D, 1), "key": (4 * D, D, 1), "value": (D, 4 * D, 1)}
     for M in (1, 4, 8, 9, 16, 17, 24, 32):
@@ -117,15 +119,18 @@ def test_decode_kernel_choice(L):
             N, K, nmat = layer[name]
             assert rq.decode_kernel_for(M, K, N, 4, nmat) == "rowblock", (M, name)
             assert rq.decode_kernel_for(M, K, N, 8, nmat) == "rowblock", (M, name)
-        for name in ("o", "value"):
-            N, K, nmat = layer[name]
-            want = "rowtile" if M <= 16 else "cluster"
-            assert rq.decode_kernel_for(M, K, N, 4, nmat) == want, (M, name)
+        small = "rowtile" if M <= 8 else "rowblock"
+        assert rq.decode_kernel_for(M, D, D, 4, 1) == small, M                          # o
+        assert rq.decode_kernel_for(M, 4 * D, D, 4, 1) == (
+            small if M <= 16 else "cluster"), M                                          # value
+    # the 13.3B-shaped layer (D = 4096): row blocks, the value projection at M > 16 on tensor cores
+    for M in (1, 8, 16, 17, 32):
+        for N, K, nmat in ((4096, 4096, 3), (4096, 4096, 1), (16384, 4096, 1)):
+            assert rq.decode_kernel_for(M, K, N, 4, nmat) == "rowblock", (M, N, K)
+        assert rq.decode_kernel_for(M, 16384, 4096, 4, 1) == ("tensor" if M > 16 else "rowblock")
     # the boundary: 148 m-tiles (2368 rows) in the launch
     assert rq.decode_kernel_for(1, D, 2368, 4, 1) == "rowblock"
     assert rq.decode_kernel_for(1, D, 2352, 4, 1) == "rowtile"
-    assert rq.decode_kernel_for(1, 16384, 16384, 4, 1) == "rowblock"
-    assert rq.decode_kernel_for(32, 16384, 16384, 4, 1) == "rowblock"
     # a selection overrides the automatic choice
     for kind in ("rowtile", "cluster"):
         with rq.decode_kernel(kind):

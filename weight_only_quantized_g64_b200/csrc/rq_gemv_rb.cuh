@@ -142,7 +142,14 @@ __device__ __forceinline__ void i8_word_biased(uint32_t w, uint32_t (&Q)[2]) {
 //           group for the tokens nt*8+g; xph[nt] their swizzle phase
 //   grp[c]  the group (for scales read from global memory when !SSC)
 // The group's four MMA steps run as one chain that starts from the bias term
-// (so no additions are needed), and the scale is applied with one fma.
+// (so no additions are needed), and the scale is applied with one fma.  With
+// several token tiles and few m-tiles the bias MMAs (4 per token tile and
+// column, shared by the m-tiles) would cost more tensor-pipe time than they
+// save: there the codes are unbiased exactly in fp16 instead (one
+// subtraction per register) and the chain starts from zero.
+template <int MT, int NT>
+constexpr bool rb_unbias() { return NT >= 4 || (NT == 2 && MT <= 4); }
+
 template <int BITS, int MT, int NT, int NC, bool SSC>
 __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
                                            const uint16_t* const (&sp)[NC], const uint8_t* xbase,
@@ -176,8 +183,9 @@ __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
         }
     // ---- -sum_k bias_k x_k of each column's group, per token tile (the same
     // for every row)
+    constexpr bool kUnbias = rb_unbias<MT, NT>();
     float negc[NC][NT][4];
-    {
+    if constexpr (!kUnbias) {
         uint32_t an[4];
         if constexpr (BITS == 4) {
             an[0] = an[1] = 0xE408E408u;   // -1032 (slots 2t, 2t+1: low-nibble pairs)
@@ -247,10 +255,28 @@ __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
                     }
                 }
             }
+            if constexpr (kUnbias) {
+                // exact: 1032 + c, 72 + c and 1152 + c minus their bias is c
+                const __half2 blo = __halves2half2(__ushort_as_half(BITS == 4 ? 0x6408 : 0x6480),
+                                                   __ushort_as_half(BITS == 4 ? 0x6408 : 0x6480));
+                const __half2 bhi = __halves2half2(__ushort_as_half(BITS == 4 ? 0x5480 : 0x6480),
+                                                   __ushort_as_half(BITS == 4 ? 0x5480 : 0x6480));
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        __half2 v = *reinterpret_cast<const __half2*>(&A[jj][r]);
+                        v = __hsub2(v, r < 2 ? blo : bhi);
+                        A[jj][r] = *reinterpret_cast<const uint32_t*>(&v);
+                    }
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 float part[4];
-                mma16816_c(part, A[0], b[c][nt][0][0], b[c][nt][0][1], negc[c][nt]);
+                if constexpr (kUnbias)
+                    mma16816(part, A[0], b[c][nt][0][0], b[c][nt][0][1], true);
+                else
+                    mma16816_c(part, A[0], b[c][nt][0][0], b[c][nt][0][1], negc[c][nt]);
 #pragma unroll
                 for (int jj = 1; jj < 4; ++jj) mma16816(part, A[jj], b[c][nt][jj][0], b[c][nt][jj][1], false);
 #pragma unroll
@@ -288,9 +314,10 @@ __device__ __forceinline__ void u4_word_biased(uint32_t w, uint32_t (&P)[4]) {
     asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(P[3]) : "r"(w8), "r"(0x00F000F0u), "r"(0x54005400u));
 }
 
-// A small unsigned integer (< 2^23) as an exact fp32 without a conversion.
-__device__ __forceinline__ float small_u_to_f32(uint32_t v) {
-    return __uint_as_float(0x4B000000u | v) - 8388608.0f;
+// Byte k of v as the fp32 2^23 + v.byte[k] (one prmt, no conversion).
+template <int k>
+__device__ __forceinline__ float byte_plus_2p23(uint32_t v) {
+    return __uint_as_float(__byte_perm(v, 0x4B000000u, 0x7540u + k));
 }
 
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
@@ -314,8 +341,9 @@ __device__ __forceinline__ void rb_column_p8(const uint8_t* const (&cwa)[4], con
             b[nt][jj][1] = v.y;
         }
     }
+    constexpr bool kUnbias = rb_unbias<MT, NT>();
     float negc[NT][4][4];   // [nt][step][element]
-    {
+    if constexpr (!kUnbias) {
         uint32_t an[4];
         an[0] = an[1] = an[2] = an[3] = 0xE480E480u;   // -1152
 #pragma unroll
@@ -333,6 +361,15 @@ __device__ __forceinline__ void rb_column_p8(const uint8_t* const (&cwa)[4], con
             for (int jj = 0; jj < 4; ++jj) {
                 uint32_t Q[2];
                 i8_word_biased(lds32(cwa[jj] + (16 * i + 8 * h) * 128), Q);
+                if constexpr (kUnbias) {
+                    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        __half2 v = *reinterpret_cast<const __half2*>(&Q[r]);
+                        v = __hsub2(v, bias);
+                        Q[r] = *reinterpret_cast<const uint32_t*>(&v);
+                    }
+                }
                 A[jj][h] = Q[0];
                 A[jj][h + 2] = Q[1];
                 sv[jj][h] = __half2float(__ushort_as_half(sp[(16 * i + 8 * h) * kRbSrowP8 + jj]));
@@ -343,7 +380,10 @@ __device__ __forceinline__ void rb_column_p8(const uint8_t* const (&cwa)[4], con
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
                 float part[4];
-                mma16816_c(part, A[jj], b[nt][jj][0], b[nt][jj][1], negc[nt][jj]);
+                if constexpr (kUnbias)
+                    mma16816(part, A[jj], b[nt][jj][0], b[nt][jj][1], true);
+                else
+                    mma16816_c(part, A[jj], b[nt][jj][0], b[nt][jj][1], negc[nt][jj]);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[i][nt][e] = fmaf(part[e], sv[jj][e >> 1], acc[i][nt][e]);
             }
@@ -409,10 +449,13 @@ __device__ __forceinline__ void rb_column_p4a(const uint8_t* cwa, const uint8_t*
             const uint32_t dd = n < N ? __ldg(supp + (16 * i + 8 * h) * nsb) : 0u;
             const float ds = __half2float(__ushort_as_half(static_cast<unsigned short>(dd & 0xFFFFu)));
             const float dm = __half2float(__ushort_as_half(static_cast<unsigned short>(dd >> 16)));
-            S[0][h] = ds * small_u_to_f32(ab & 0xFFu);
-            O[0][h] = -(dm * small_u_to_f32((ab >> 8) & 0xFFu));
-            S[1][h] = ds * small_u_to_f32((ab >> 16) & 0xFFu);
-            O[1][h] = -(dm * small_u_to_f32(ab >> 24));
+            // S = ds a = ds (2^23 + a) - ds 2^23 and O = -(dm b) likewise, each
+            // one fused multiply-add: exact (ds a and dm b fit in 17 bits)
+            const float ds23 = ds * 8388608.0f, dm23 = dm * 8388608.0f;
+            S[0][h] = fmaf(ds, byte_plus_2p23<0>(ab), -ds23);
+            O[0][h] = fmaf(-dm, byte_plus_2p23<1>(ab), dm23);
+            S[1][h] = fmaf(ds, byte_plus_2p23<2>(ab), -ds23);
+            O[1][h] = fmaf(-dm, byte_plus_2p23<3>(ab), dm23);
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)

@@ -83,7 +83,7 @@ cudaError_t launch_tcs(const uint16_t* const* xs, int nx, int64_t M, int64_t K, 
                        cudaStream_t s);
 bool tcs_fits(int64_t M, int64_t K, int64_t N, int bits);
 // Its K split (cluster size) for a shape.
-int tcs_ksplit(int64_t K, int64_t N, int nmat);
+int tcs_ksplit(int64_t K, int64_t N, int nmat, int bits);
 
 // Whether the row-block kernel takes a product of this shape and format.
 bool gemv_rowblock_fits(int64_t M, int64_t K, int64_t N, int bits, int nmat, int fmt = FMT_G64);

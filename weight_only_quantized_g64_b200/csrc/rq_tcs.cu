@@ -11,11 +11,12 @@
 // keeping the streaming shape of a decode kernel:
 //
 // Work.  A CTA owns one 256-row block of one matrix and a contiguous range
-// of its 64-k groups: the ks CTAs of a thread-block cluster split the block's
-// K range (ks chosen so that blocks x ks fills the SMs, at most 16).  Their
-// fp32 partial sums meet in shared memory and are added across the cluster
-// through distributed shared memory in rank order -- deterministic, no
-// workspace, no atomics.
+// of its stages (4 k groups of int4, 2 of int8): the ks CTAs of a
+// thread-block cluster split the block's K range (ks chosen from the
+// cluster occupancy so that the blocks run in as few waves as possible).
+// Their fp32 partial sums meet in shared memory and are added across the
+// cluster through distributed shared memory in rank order -- deterministic,
+// no workspace, no atomics.
 //
 // Roles (704 threads):
 //   warp 0      TMA producer: per unit the codes of 256 rows x 64 k (one box)
@@ -73,42 +74,49 @@ struct TcsParams {
 
 constexpr int kTcsRows = 256;          // rows per block (two 128-row MMA tiles)
 constexpr int kTcsG = 4;               // dequantiser groups
-constexpr int kTcsSA = kTcsG;          // TMEM A stages (one per group)
 constexpr int kTcsThreads = 32 * (2 + 4 + 4 * kTcsG);
-constexpr int kTcsSmemBudget = 200 * 1024;
+constexpr int kTcsSmemBudget = 220 * 1024;
 
 template <int BITS, int BNT>
 struct TcsCfg {
-    static constexpr int kCodeBytes = 64 * BITS / 8;              // per row per unit
-    static constexpr int kXStage = BNT * 128;
-    static constexpr int kWStage = kTcsRows * kCodeBytes;
+    // A stage is KS k groups: 128 bytes of codes per row (one box of 256 rows
+    // x 128 B, 128-byte swizzle) and the KS x tiles [BNT tokens x 64 k].
+    static constexpr int KS = BITS == 4 ? 4 : 2;                  // k groups per stage
+    static constexpr int kCodeBytes = 64 * BITS / 8;              // per row per k group
+    static constexpr int kXTile = BNT * 128;                      // x of one k group
+    static constexpr int kXStage = KS * kXTile;
+    static constexpr int kWStage = kTcsRows * 128;
     static constexpr int kStage = kXStage + kWStage;
+    // ring depth: as many stages as fit, a multiple of G / KS so that every
+    // stage is always read by the same dequantiser groups (a group must never
+    // see a stage's barrier two rounds ahead of it)
+    static constexpr int kSSmul = kTcsG / KS;
     static constexpr int kSSraw = kTcsSmemBudget / kStage;
-    static constexpr int kSS = (kSSraw > 32 ? 32 : kSSraw) / kTcsG * kTcsG;
+    static constexpr int kSS = kSSraw / kSSmul * kSSmul;
     static constexpr int kRing = kSS * kStage;
-    // TMEM: the accumulators (2 tiles x BNT columns), then the A stages
-    // (2 tiles x 32 columns each)
+    // TMEM: the accumulators (2 tiles x BNT columns), then as many A stages
+    // (2 tiles x 32 columns each) as fit in the 512 columns.  A group writes
+    // k group i into A stage i % SA once the MMAs of k group i - SA are done;
+    // with SA above the group count that wait is over long before.
     static constexpr int kAccCols = 2 * BNT;
     static constexpr int kACol0 = kAccCols;
-    static constexpr int kColsNeeded = kACol0 + kTcsSA * 64;
-    static constexpr int kTmemCols = kColsNeeded <= 256 ? 256 : 512;
-    static constexpr int kChunks = kCodeBytes / 16;               // 16-byte code chunks per row
-    static constexpr int kBars = 2 * kSS + 2 * kTcsSA + 1;
+    static constexpr int kSA = (512 - kAccCols) / 64;
+    static constexpr int kColsNeeded = kACol0 + kSA * 64;
+    static constexpr int kTmemCols = 512;
+    static constexpr int kChunks = kCodeBytes / 16;               // 16-byte code chunks per group
+    static constexpr int kBars = 2 * kSS + 2 * kSA + 1;
     static constexpr int kSmem = 1024 + kRing + kBars * 8 + 64;
-    static_assert(kSS >= kTcsG, "ring too shallow");
-    static_assert(kColsNeeded <= 512, "TMEM overflow");
-    static_assert(kXStage % 1024 == 0 && kWStage % 1024 == 0, "stage alignment");
+    static_assert(kSS >= 2, "ring too shallow");
+    static_assert(kColsNeeded <= 512 && kSA > kTcsG, "TMEM layout");
+    static_assert(kXTile % 1024 == 0 && kWStage % 1024 == 0, "stage alignment");
+    static_assert(kSmem <= 227 * 1024, "shared memory");
     static_assert(kRing >= 64 * kTcsRows * 4, "the partial sums reuse the ring");
 };
 
-// 16-byte chunk c of row r of a swizzled codes box (32-byte rows with
-// SWIZZLE_32B for int4; 64-byte rows with SWIZZLE_64B for int8).
-template <int BITS>
+// 16-byte chunk c of row r of the codes box (128-byte rows, 128-byte swizzle:
+// chunk index ^= row % 8, so the rows a warp reads hit distinct banks).
 __device__ __forceinline__ uint4 tcs_code_chunk(const uint8_t* tile, int r, int c) {
-    if constexpr (BITS == 4)
-        return *reinterpret_cast<const uint4*>(tile + r * 32 + ((c ^ ((r >> 2) & 1)) << 4));
-    else
-        return *reinterpret_cast<const uint4*>(tile + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+    return *reinterpret_cast<const uint4*>(tile + r * 128 + ((c ^ (r & 7)) << 4));
 }
 
 __device__ __forceinline__ uint32_t tcs_lop3_6a(uint32_t a, uint32_t b, uint32_t c) {
@@ -168,8 +176,9 @@ template <int BITS, int BNT>
 __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_constant__ TcsParams p) {
     using Cfg = TcsCfg<BITS, BNT>;
     constexpr int SS = Cfg::kSS;
-    constexpr int SA = kTcsSA;
+    constexpr int SA = Cfg::kSA;
     constexpr int G = kTcsG;
+    constexpr int KS = Cfg::KS;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t s0 = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
     uint8_t* smem = smem_raw + ((1024u - (s0 & 1023u)) & 1023u);
@@ -191,15 +200,21 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
     const int mat = blk / p.nrb;
     const int rb = blk - mat * p.nrb;
     const int KB = p.kblocks;
-    const int kb0 = static_cast<int>((static_cast<int64_t>(kq) * KB) / ks);
-    const int kb1 = static_cast<int>((static_cast<int64_t>(kq + 1) * KB) / ks);
-    const int n_units = kb1 - kb0;
+    const int nst = (KB + KS - 1) / KS;               // stages of a row
+    const int st0 = static_cast<int>((static_cast<int64_t>(kq) * nst) / ks);
+    const int st1 = static_cast<int>((static_cast<int64_t>(kq + 1) * nst) / ks);
+    const int n_stages = st1 - st0;
+    // k groups of this CTA: units 0 .. n_units-1 are k groups st0*KS + i
+    // (those at or past KB, in the row's last stage, are zero-filled)
+    const int n_units = n_stages * KS;
+    const int kb0 = st0 * KS;
     const CUtensorMap* tmx = &p.tm_x[p.nx > 1 ? mat : 0];
 
+    const int pre = n_stages < SS ? n_stages : SS;
     if (threadIdx.x == 0) {
         for (int s = 0; s < SS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 4 + 1);
+            mbar_init(&empty[s], 4 * KS + 1);
         }
         for (int a = 0; a < SA; ++a) {
             mbar_init(&afull[a], 4);
@@ -208,6 +223,31 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
         mbar_init(accfull, 1);
         *abort_flag = 0;
         fence_mbar_init();
+        // codes never depend on the previous kernel: the first stages' go out
+        // at once, while the rest of the CTA sets up
+        tma_prefetch_desc(&p.tm_w[mat]);
+        tma_prefetch_desc(tmx);
+        const uint64_t pol_w = l2_policy_evict_first();
+        for (int j = 0; j < pre; ++j) {
+            mbar_arrive_expect_tx(&full[j], Cfg::kStage);
+            tma_load_2d(ring + j * Cfg::kStage + Cfg::kXStage, &p.tm_w[mat], &full[j],
+                        (st0 + j) * 128, rb * kTcsRows, pol_w);
+        }
+    }
+    // dequantisers: their rows' scales, and the first unit's, also early
+    const int dw = warp - 6;
+    const int grp = dw >> 2;                        // k groups grp, grp + G, ...
+    const uint16_t* srow[2] = {nullptr, nullptr};
+    bool row_ok[2] = {false, false};
+    uint16_t sc_next[2] = {0, 0};
+    if (warp >= 6) {
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+            const int n = rb * kTcsRows + tt * 128 + (warp & 3) * 32 + lane;
+            row_ok[tt] = n < p.N;
+            srow[tt] = p.scales[mat] + static_cast<int64_t>(row_ok[tt] ? n : 0) * KB;
+            sc_next[tt] = (row_ok[tt] && grp < n_units && kb0 + grp < KB) ? __ldg(srow[tt] + kb0 + grp) : 0;
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, Cfg::kTmemCols);
@@ -221,32 +261,22 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
-        if (elect_one()) {
+        if (threadIdx.x == 0) {
             const uint64_t pol_w = l2_policy_evict_first();   // codes: read once
             const uint64_t pol_x = l2_policy_evict_last();    // x: read by every block
-            tma_prefetch_desc(&p.tm_w[mat]);
-            tma_prefetch_desc(tmx);
-            const int pre = n_units < SS ? n_units : SS;
-            // codes never depend on the previous kernel: the first stages' go
-            // out before waiting for it
-            for (int i = 0; i < pre; ++i) {
-                mbar_arrive_expect_tx(&full[i], Cfg::kStage);
-                tma_load_2d(ring + i * Cfg::kStage + Cfg::kXStage, &p.tm_w[mat], &full[i],
-                            (kb0 + i) * Cfg::kCodeBytes, rb * kTcsRows, pol_w);
-            }
             pdl_wait();
-            for (int i = 0; i < pre; ++i)
-                tma_load_2d(ring + i * Cfg::kStage, tmx, &full[i], (kb0 + i) * 64, 0, pol_x);
+            for (int j = 0; j < pre; ++j)
+                tma_load_3d(ring + j * Cfg::kStage, tmx, &full[j], 0, 0, (st0 + j) * KS, pol_x);
             int issued = pre;
             int s = 0;
             uint32_t ph = 0;            // parity of the round stage s is in
-            for (int i = SS; i < n_units; ++i) {
+            for (int j = SS; j < n_stages; ++j) {
                 if (!mbar_wait(&empty[s], ph, abort_flag, p.timeout_ns, p.status)) break;
                 mbar_arrive_expect_tx(&full[s], Cfg::kStage);
                 tma_load_2d(ring + s * Cfg::kStage + Cfg::kXStage, &p.tm_w[mat], &full[s],
-                            (kb0 + i) * Cfg::kCodeBytes, rb * kTcsRows, pol_w);
-                tma_load_2d(ring + s * Cfg::kStage, tmx, &full[s], (kb0 + i) * 64, 0, pol_x);
-                issued = i + 1;
+                            (st0 + j) * 128, rb * kTcsRows, pol_w);
+                tma_load_3d(ring + s * Cfg::kStage, tmx, &full[s], 0, 0, (st0 + j) * KS, pol_x);
+                issued = j + 1;
                 if (++s == SS) {
                     s = 0;
                     ph ^= 1u;
@@ -256,8 +286,8 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
             // into every stage, so none is in flight when the CTA exits
             int dummy_abort = 0;
             const int first = issued > SS ? issued - SS : 0;
-            for (int i = first; i < issued; ++i)
-                mbar_wait(&full[i % SS], static_cast<uint32_t>(i / SS) & 1u, &dummy_abort,
+            for (int j = first; j < issued; ++j)
+                mbar_wait(&full[j % SS], static_cast<uint32_t>(j / SS) & 1u, &dummy_abort,
                           p.timeout_ns, p.status);
         }
         __syncwarp();
@@ -266,16 +296,17 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
         if (elect_one()) {
             constexpr uint32_t idesc = idesc_f16_f32(128, BNT);
             for (int i = 0; i < n_units; ++i) {
-                const int s = i % SS;
+                const int j = i / KS;                 // stage index within the CTA
+                const int s = j % SS;
                 const int a = i % SA;
-                if (!mbar_wait(&full[s], static_cast<uint32_t>(i / SS) & 1u, abort_flag,
-                               p.timeout_ns, p.status))
+                if (i % KS == 0 && !mbar_wait(&full[s], static_cast<uint32_t>(j / SS) & 1u, abort_flag,
+                                              p.timeout_ns, p.status))
                     break;
                 if (!mbar_wait(&afull[a], static_cast<uint32_t>(i / SA) & 1u, abort_flag,
                                p.timeout_ns, p.status))
                     break;
                 tc_fence_after();
-                const uint32_t xs = smem_u32(ring + s * Cfg::kStage);
+                const uint32_t xs = smem_u32(ring + s * Cfg::kStage + (i % KS) * Cfg::kXTile);
                 const uint32_t acol = tmem_base + Cfg::kACol0 + a * 64;
 #pragma unroll
                 for (int tt = 0; tt < 2; ++tt)
@@ -283,8 +314,8 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
                     for (int t = 0; t < 4; ++t)
                         tc_mma_ts(tmem_base + tt * BNT, acol + tt * 32 + t * 8,
                                   smem_desc_k_sw128(xs + t * 32), idesc, (i == 0 && t == 0) ? 0u : 1u);
-                tc_commit(&empty[s]);
                 tc_commit(&aempty[a]);
+                if (i % KS == KS - 1) tc_commit(&empty[s]);
             }
             tc_commit(accfull);
         }
@@ -333,34 +364,26 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
         }
     } else {
         // ---------------------------------------- dequantise into TMEM --
-        const int dw = warp - 6;
-        const int grp = dw >> 2;                    // units grp, grp + G, ...
         const int q = warp & 3;                     // TMEM lane quarter
         const int r0 = q * 32 + lane;
         const int tg = (dw & 3) * 32 + lane;        // thread within the group
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-        const uint16_t* srow[2];
-        bool row_ok[2];
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-            const int n = rb * kTcsRows + tt * 128 + r0;
-            row_ok[tt] = n < p.N;
-            srow[tt] = p.scales[mat] + static_cast<int64_t>(row_ok[tt] ? n : 0) * KB;
-        }
-        // scales of this thread's rows for unit i (0 outside the matrix)
+        // scales of this thread's rows for unit i (0 outside the matrix and
+        // past the row's last k group)
         auto scales_of = [&](int i, uint16_t (&sc)[2]) {
+            const int kb = kb0 + i;
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt)
-                sc[tt] = (row_ok[tt] && i < n_units) ? __ldg(srow[tt] + kb0 + i) : 0;
+                sc[tt] = (row_ok[tt] && i < n_units && kb < KB) ? __ldg(srow[tt] + kb) : 0;
         };
-        uint16_t sc_next[2];
-        scales_of(grp, sc_next);
         for (int i = grp; i < n_units; i += G) {
-            const int s = i % SS;
+            const int j = i / KS;
+            const int s = j % SS;
             const int a = i % SA;
+            const int kj = i % KS;                      // k group within the stage
             uint16_t sc[2] = {sc_next[0], sc_next[1]};
             scales_of(i + G, sc_next);
-            if (!mbar_wait(&full[s], static_cast<uint32_t>(i / SS) & 1u, abort_flag, p.timeout_ns,
+            if (!mbar_wait(&full[s], static_cast<uint32_t>(j / SS) & 1u, abort_flag, p.timeout_ns,
                            p.status))
                 break;
             uint8_t* st = ring + s * Cfg::kStage;
@@ -369,11 +392,13 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
-                for (int c = 0; c < Cfg::kChunks; ++c) v[tt][c] = tcs_code_chunk<BITS>(wt, tt * 128 + r0, c);
+                for (int c = 0; c < Cfg::kChunks; ++c)
+                    v[tt][c] = tcs_code_chunk(wt, tt * 128 + r0, kj * Cfg::kChunks + c);
             if constexpr (BITS == 4) {
-                // x chunks into the pair order of the unpacking
+                // this k group's x chunks into the pair order of the unpacking
+                uint8_t* xt = st + kj * Cfg::kXTile;
                 for (int ch = tg; ch < BNT * 8; ch += 128) {
-                    uint4* xp = reinterpret_cast<uint4*>(st + ch * 16);
+                    uint4* xp = reinterpret_cast<uint4*>(xt + ch * 16);
                     const uint4 xv = *xp;
                     uint4 o;
                     o.x = __byte_perm(xv.x, xv.z, 0x5410);
@@ -467,11 +492,11 @@ bool tcs_fits(int64_t M, int64_t K, int64_t N, int bits) {
 }
 
 // K split (cluster size): as many CTAs per block as keep blocks x ks within
-// the SMs, at most 16 and at most one per k group.
-int tcs_ksplit(int64_t K, int64_t N, int nmat) {
+// the SMs, at most 16 and at most one per stage of k groups.
+int tcs_ksplit(int64_t K, int64_t N, int nmat, int bits) {
     const int64_t blocks = static_cast<int64_t>(nmat) * ((N + kTcsRows - 1) / kTcsRows);
     int64_t ks = num_sms() / blocks;
-    const int64_t kb = K / kGroup;
+    const int64_t kb = (K / kGroup + (bits == 4 ? 3 : 1)) / (bits == 4 ? 4 : 2);   // stages
     if (ks > 16) ks = 16;
     if (ks > kb) ks = kb;
     if (ks < 1) ks = 1;
@@ -522,16 +547,18 @@ static cudaError_t tcs_launch_cfg(const TcsParams& prm, int ks_want, int blocks,
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    // the cluster size that keeps the most CTAs working at once (clusters must
-    // fit in a GPC: large ones may not all be resident together)
+    // the cluster size with the least time per block: a block's work shrinks
+    // as 1/ks, but clusters must fit in a GPC, so large ones may not all be
+    // resident at once and then run in waves (ks / waves is the figure of merit)
     int ks = 1;
-    int64_t best = -1;
+    double best = -1.0;
     for (int c = ks_want; c >= 1; --c) {
         const int act = tcs_active_clusters<BITS, BNT>(dev, c);
         if (act <= 0) continue;
-        const int64_t busy = static_cast<int64_t>(act < blocks ? act : blocks) * c;
-        if (busy > best) {
-            best = busy;
+        const int waves = (blocks + act - 1) / act;
+        const double merit = static_cast<double>(c) / waves;
+        if (merit > best) {
+            best = merit;
             ks = c;
         }
     }
@@ -575,21 +602,23 @@ cudaError_t launch_tcs(const uint16_t* const* xs, int nx, int64_t M, int64_t K, 
     prm.epi = epilogue;
     prm.status = device_status_ptr();
     prm.timeout_ns = wait_limit_ns();
-    const int ks = tcs_ksplit(K, N, nmat);
+    const int ks = tcs_ksplit(K, N, nmat, bits);
     const int blocks = nmat * prm.nrb;
     const uint64_t row_bytes = static_cast<uint64_t>(K) * bits / 8;
     for (int i = 0; i < nmat; ++i) {
         if (!make_tmap_2d(&prm.tm_w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, w[i].codes, row_bytes,
-                          static_cast<uint64_t>(N), row_bytes, 64 * bits / 8, kTcsRows,
-                          bits == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B))
+                          static_cast<uint64_t>(N), row_bytes, 128, kTcsRows,
+                          CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
         prm.scales[i] = w[i].scales;
         prm.y[i] = w[i].y;
     }
+    // x as {64 k, M tokens, K/64 groups}: one box per stage = KS x tiles
+    const uint32_t kstage = bits == 4 ? 4 : 2;
     for (int i = 0; i < nx; ++i)
-        if (!make_tmap_2d(&prm.tm_x[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs[i],
-                          static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                          static_cast<uint64_t>(K) * 2, 64, static_cast<uint32_t>(bnt),
+        if (!make_tmap_3d(&prm.tm_x[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs[i], 64,
+                          static_cast<uint64_t>(M), static_cast<uint64_t>(K / kGroup),
+                          static_cast<uint64_t>(K) * 2, 128, 64, static_cast<uint32_t>(bnt), kstage,
                           CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     if (bits == 4)
