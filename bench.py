@@ -47,17 +47,20 @@ METRIC = "decode w4g64 GEMV weight GB/s (% of B200 HBM peak); prefill TFLOP/s; 1
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# DRAM traffic of the decode kernels per launch (dram__bytes_read.sum +
-# dram__bytes_write.sum from an ncu capture, see the profile summaries).  It
-# is valid only for the kernel code it was taken on: when the code's hash
-# (comments and whitespace ignored) differs, the bench reports traffic as null
-# until a new capture is taken.
+# DRAM traffic of the decode kernels: dram__bytes_read.sum +
+# dram__bytes_write.sum of a one-launch ncu capture of the row-block kernel on
+# 16384 x 4096 int4 at M = 1, divided by that launch's algorithmic bytes
+# (codes + scales).  Traffic grows in proportion to the weights a launch
+# streams, so the bench reports this ratio times its average algorithmic bytes
+# per launch.  It is valid only for the kernel code it was taken on: when the
+# code's hash (comments and whitespace ignored) differs, the bench reports
+# traffic as null until a new capture is taken.
 DECODE_SOURCES = ("rq_api.cu", "rq_gemv.cu", "rq_gemv_ck.cu", "rq_gemv_unit.cuh", "rq_ptx.cuh",
                   "rq_internal.h", "rq_gemv_rb.cuh", "rq_gemv_rb.cu", "rq_gemv_rb_g64_4.cu",
                   "rq_gemv_rb_g64_8.cu", "rq_tcs.cu")
 KERNEL_NAMES = {"rowtile": "gemv_wq_kernel (row tiles)", "cluster": "gemv_ck_kernel (cluster split-K)",
                 "rowblock": "gemv_rb_kernel (row blocks)", "tensor": "tcs_kernel (tcgen05, K split over a cluster)"}
-DECODE_TRAFFIC = {"code_sha256_16": "076aa3b7224c42d8", "bytes_per_launch": 6823383}
+DECODE_TRAFFIC = {"code_sha256_16": "c2f67e878ff169f2", "dram_per_algorithmic_byte": 35697920 / 35651584}
 
 
 def decode_code_hash():
@@ -72,10 +75,10 @@ def decode_code_hash():
     return h.hexdigest()[:16]
 
 
-def decode_traffic():
+def decode_traffic(algorithmic_bytes_per_launch):
     if decode_code_hash() != DECODE_TRAFFIC["code_sha256_16"]:
         return None
-    return DECODE_TRAFFIC["bytes_per_launch"]
+    return DECODE_TRAFFIC["dram_per_algorithmic_byte"] * algorithmic_bytes_per_launch
 
 
 def peaks():
@@ -629,7 +632,8 @@ def main():
             "hbm_frac": value / world / hbm_peak,
             "per_M": per_m,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "traffic": decode_traffic(),
+                         "frac": achieved / hbm_peak,
+                         "traffic": decode_traffic(bytes_per_step / launches_per_step),
                          "kernel": "decode products (fused RKV + O + key + value, all M): " +
                                    ", ".join(f"{KERNEL_NAMES[k]} x{len(v)}" for k, v in
                                              sorted(stack.kernels().items())),
