@@ -345,18 +345,20 @@ rq_status rq_gemm_wq(const uint16_t *x, int64_t M, int64_t K, const void *codes,
  * allocator.
  *
  * Same arguments, result and rules as rq_gemv_wq (1 <= M <= 32; y fully
- * overwritten).  Limits: N <= 16384 * 32 rows, and the partial sums of one
- * launch must fit the fixed array (true for every M on a 148-SM B200);
- * otherwise RQ_ERR_SHAPE is returned and nothing is launched.
+ * overwritten).  Only the row-tile kernel (see rq_set_decode_kernel) uses
+ * the array: its launch must fit it -- one counter per row tile of 16 to 64
+ * rows, at most 16384, and the partial sums within 5 MiB (true for every M
+ * on a 148-SM B200) -- else RQ_ERR_SHAPE is returned and nothing is
+ * enqueued; such a call clears the counters it uses (an asynchronous memset
+ * on `stream`) and then launches the product.  The row-block, cluster and
+ * tensor-core kernels keep their partial sums on chip: a call that runs on
+ * one of them uses no scratch, launches only the product and has no row
+ * limit of its own.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current) -- make it before any stream capture.
- * A call that runs on the row-tile kernel (see rq_set_decode_kernel) clears
- * the counters it uses (an asynchronous memset on `stream`) and then launches
- * the product; one that runs on the cluster kernel needs no scratch and
- * launches only the product.  Each device has its own copy of the array, and
- * all calls on one device share it: calls that may overlap on the same device
- * (e.g. on two streams with no ordering between them) race on it and give
- * wrong results.
+ * Each device has its own copy of the array; calls that may overlap on the
+ * same device (e.g. on two streams with no ordering between them) race on
+ * it and give wrong results.
  */
 rq_status rq_gemv_wq_noalloc(const uint16_t *x, int64_t M, int64_t K, const void *codes,
                              const uint16_t *scales, int64_t N, int bits, float *y,

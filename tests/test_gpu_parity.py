@@ -129,6 +129,24 @@ def test_gemv_parity(kernel, bits, M, N, K):
     check_close(to_host(y), y_ref, bound, f"gemv {kernel} bits={bits} M={M} N={N} K={K}")
 
 
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M", [1, 3, 8, 16, 32])
+@pytest.mark.parametrize("N,K", [(2400, 512), (5000, 256), (7500, 192), (16400, 128)])
+def test_rowblock_tall_blocks(bits, M, N, K):
+    """Every output of launches whose row blocks hold 2, 3, 4 and 7 m-tiles
+    (the row-block kernel splits them over two halves of 16 warps at M <= 8,
+    an odd count leaving the second half one short), ragged N included."""
+    x, codes, scales = product_case(N, K, bits, M, seed=3000 + M + N)
+    cd, sd = upload(codes, scales)
+    with rq.decode_kernel("rowblock"):
+        y = rq.gemv_wq(x, cd, sd, N, bits)
+        y2 = rq.gemv_wq(x, cd, sd, N, bits)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+    y_ref, bound = oracle.matmul(to_host(x), codes, scales, bits)
+    check_close(to_host(y), y_ref, bound, f"rowblock bits={bits} M={M} N={N} K={K}")
+
+
 @pytest.mark.parametrize("kernel", DECODE_KERNELS)
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("M", [1, 8, 13, 32])

@@ -63,11 +63,40 @@ def test_noalloc_matches_gemv_two_calls(N, K, M, bits, kernel):
     assert rq.read_device_status() == rq.OK
 
 
-def test_noalloc_rejects_beyond_its_scratch():
-    """More rows than the fixed counters cover: refused, nothing launched."""
-    N = 16384 * 32 + 1
-    K = 64
-    fake = 1 << 20     # aligned, never dereferenced: the size check comes first
+def test_noalloc_rejects_bad_batch():
+    """M outside 1..32 is refused before anything is enqueued (the fake
+    pointers are never touched).  The scratch bound itself cannot be reached
+    on a 148-SM B200: the row-tile kernel needs counters only when it splits
+    row tiles across CTAs, which it does only while there are few of them."""
+    fake = 1 << 20
     L = rq.lib()
-    assert L.rq_gemv_wq_noalloc(fake, 1, K, fake, fake, N, 4, fake, None) == rq.ERR_SHAPE
-    assert L.rq_gemv_wq_noalloc(fake, 33, K, fake, fake, 128, 4, fake, None) == rq.ERR_SHAPE
+    assert L.rq_gemv_wq_noalloc(fake, 33, 64, fake, fake, 128, 4, fake, None) == rq.ERR_SHAPE
+    assert L.rq_gemv_wq_noalloc(fake, 0, 64, fake, fake, 128, 4, fake, None) == rq.ERR_SHAPE
+
+
+def test_noalloc_tall_projection_on_chip_kernels():
+    """N = 262144 + 16 rows at M = 32: the automatic choice runs a kernel that
+    keeps its partial sums on chip, so the fixed counters do not limit it;
+    checked against rq_gemv_wq and, on sampled outputs, the oracle."""
+    N, K, M, bits = 262144 + 16, 64, 32, 4
+    W = synth.weights(N, K, seed=91, device="cuda")
+    codes, scales = rq.quantize_g64(W, bits)
+    x = synth.activations(M, K, seed=91, device="cuda")
+    y = torch.full((M, N), float("nan"), device="cuda")
+    L = rq.lib()
+    s = torch.cuda.current_stream().cuda_stream
+    assert rq.decode_kernel_for(M, K, N, bits) != "rowtile"
+    st = L.rq_gemv_wq_noalloc(x.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(), N, bits,
+                              y.data_ptr(), s)
+    assert st == rq.OK, rq.STATUS[st]
+    y_ref = rq.gemv_wq(x, codes, scales, N, bits)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_ref)
+    rng = np.random.default_rng(5)
+    ms = rng.integers(0, M, 512)
+    ns = np.concatenate([[0, N - 1], rng.integers(0, N, 510)])
+    yo, bound = oracle.matmul_sampled(x.cpu().numpy(), codes.cpu().numpy(),
+                                      scales.cpu().numpy().view(np.uint16), bits, ms, ns)
+    d = np.abs(y.cpu().numpy().astype(np.float64)[ms, ns] - yo)
+    assert np.all(d <= TOL * bound)
+    assert rq.read_device_status() == rq.OK

@@ -613,10 +613,16 @@ static cudaError_t gv_launch(GvParams& prm, const uint16_t* x, const void* const
     } else {
         if (ws_bytes > scratch->ws_bytes || n_cnt > scratch->n_cnt) {
             if (scratch->too_large) *scratch->too_large = true;
-            return cudaErrorInvalidValue;
+            return cudaErrorInvalidValue;   // refused before anything is enqueued
         }
         prm.ws = scratch->ws;
         prm.cnt = scratch->cnt;
+        // a completed launch leaves its counters at zero, an aborted one might
+        // not: clear the ones this launch uses
+        if (n_cnt > 0) {
+            e = cudaMemsetAsync(prm.cnt, 0, n_cnt * sizeof(int), s);
+            if (e != cudaSuccess) return e;
+        }
     }
 
     // Codes as {128 B of a stage, row, stage}: a box is ks consecutive stages

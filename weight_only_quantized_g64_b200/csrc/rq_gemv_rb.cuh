@@ -150,12 +150,14 @@ __device__ __forceinline__ void i8_word_biased(uint32_t w, uint32_t (&Q)[2]) {
 template <int MT, int NT>
 constexpr bool rb_unbias() { return NT >= 4 || (NT == 2 && MT <= 4); }
 
-template <int BITS, int MT, int NT, int NC, bool SSC>
+// MT: m-tiles this warp takes (of the block's MTALL, from m-tile mi0 on).
+template <int BITS, int MT, int NT, int NC, bool SSC, int MTALL = MT>
 __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
                                            const uint16_t* const (&sp)[NC], const uint8_t* xbase,
                                            const int (&xrow)[NC][NT], const int (&xph)[NT], int t,
                                            float (&acc)[MT][NT][4], const uint16_t* gscales,
-                                           int64_t grow0, int groups, const int (&grp)[NC], int N) {
+                                           int64_t grow0, int groups, const int (&grp)[NC], int N,
+                                           int mi0 = 0) {
     constexpr int CW = BITS == 4 ? 2 : 4;   // code words per row and group
     // ---- x fragments: token nt*8+g, positions 16t .. 16t+15 of the group
     uint32_t b[NC][NT][4][2];
@@ -183,7 +185,7 @@ __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
         }
     // ---- -sum_k bias_k x_k of each column's group, per token tile (the same
     // for every row)
-    constexpr bool kUnbias = rb_unbias<MT, NT>();
+    constexpr bool kUnbias = rb_unbias<MTALL, NT>();
     float negc[NC][NT][4];
     if constexpr (!kUnbias) {
         uint32_t an[4];
@@ -203,15 +205,17 @@ __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
                     mma16816(negc[c][nt], an, b[c][nt][jj][0], b[c][nt][jj][1], false);
             }
     }
-    // ---- every m-tile
+    // ---- every m-tile of this warp
 #pragma unroll
     for (int i = 0; i < MT; ++i) {
+        const int mi = mi0 + i;                // m-tile within the block
+        if (MT != MTALL && mi >= MTALL) break;   // (odd split: the second half is short)
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
             uint32_t cw[2][CW];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const uint8_t* cp = cw0[c] + (16 * i + 8 * h) * 128;
+                const uint8_t* cp = cw0[c] + (16 * mi + 8 * h) * 128;
                 if constexpr (BITS == 4) {
                     const uint2 v = lds64(cp);
                     cw[h][0] = v.x;
@@ -226,9 +230,9 @@ __device__ __forceinline__ void rb_columns(const uint8_t* const (&cw0)[NC],
             for (int h = 0; h < 2; ++h) {
                 uint16_t s16;
                 if constexpr (SSC) {
-                    s16 = sp[c][(16 * i + 8 * h) * kRbSrow];
+                    s16 = sp[c][(16 * mi + 8 * h) * kRbSrow];
                 } else {
-                    const int64_t n = grow0 + 16 * i + 8 * h;
+                    const int64_t n = grow0 + 16 * mi + 8 * h;
                     s16 = (n < N && grp[c] < groups) ? __ldg(gscales + n * groups + grp[c])
                                                      : static_cast<uint16_t>(0);
                 }
@@ -476,9 +480,15 @@ __device__ __forceinline__ void rb_column_p4a(const uint8_t* cwa, const uint8_t*
     }
 }
 
-template <int FMT, int BITS, int MT, int NT, bool SSC>
-__global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_constant__ RbParams p) {
+// WARPS = 8: every warp takes all MT m-tiles of its columns; WARPS = 16 (the
+// group-64 format at M <= 8 on blocks of >= 2 m-tiles): warps w and w + 8
+// share the columns and split the m-tiles, so twice the warps (with half the
+// accumulators each) hide the shared-memory latency of the loop.
+template <int FMT, int BITS, int MT, int NT, bool SSC, int WARPS = 8>
+__global__ void __launch_bounds__(WARPS * 32, 1) gemv_rb_kernel(const __grid_constant__ RbParams p) {
+    static_assert(WARPS == 8 || (WARPS == 16 && FMT == FMT_G64), "m-tile halves: group-64 only");
     constexpr int GPS = BITS == 4 ? 4 : 2;      // groups per 128-byte stage
+    constexpr int MTH = WARPS == 16 ? (MT + 1) / 2 : MT;   // m-tiles per warp
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned start, reached by an offset from the shared array
     // itself so every access below stays a shared-memory access
@@ -487,7 +497,9 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
     uint8_t* ring = smem;
     RbBars* bars = reinterpret_cast<RbBars*>(smem + p.bar_off);
     volatile int* abort_flag = &bars->abort;
-    const int warp = threadIdx.x >> 5;
+    const int warp_id = threadIdx.x >> 5;
+    const int warp = warp_id & 7;               // column warp: columns warp, warp + 8, ...
+    const int mi0 = (warp_id >> 3) * MTH;       // first m-tile of this warp
     const int lane = threadIdx.x & 31;
     const int SG = p.sg;
     const int RB = 16 * MT;                     // rows of a block (== 16 * p.tc)
@@ -600,9 +612,9 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
                 if (++rq == SG) rq = 0;
             }
         }
-        float acc[MT][NT][4];
+        float acc[MTH][NT][4];
 #pragma unroll
-        for (int i = 0; i < MT; ++i)
+        for (int i = 0; i < MTH; ++i)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -669,8 +681,8 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
                         xr[1][nt] = xrow0[nt] + (c + 1) * x_step;
                     }
                     const int gr[2] = {grp0 + warp + kRbWarps * c, grp0 + warp + kRbWarps * (c + 1)};
-                    rb_columns<BITS, MT, NT, 2, SSC>(cw0, sp, base, xr, xph, t, acc, p.scales[m],
-                                                     row0 + prow, p.groups, gr, p.N);
+                    rb_columns<BITS, MTH, NT, 2, SSC, MT>(cw0, sp, base, xr, xph, t, acc, p.scales[m],
+                                                          row0 + prow, p.groups, gr, p.N, mi0);
                 }
                 for (; warp + kRbWarps * c < jn; ++c) {
                     const uint8_t* cw0[1] = {cbase + c * code_step};
@@ -679,8 +691,8 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) xr[0][nt] = xrow0[nt] + c * x_step;
                     const int gr[1] = {grp0 + warp + kRbWarps * c};
-                    rb_columns<BITS, MT, NT, 1, SSC>(cw0, sp, base, xr, xph, t, acc, p.scales[m],
-                                                     row0 + prow, p.groups, gr, p.N);
+                    rb_columns<BITS, MTH, NT, 1, SSC, MT>(cw0, sp, base, xr, xph, t, acc, p.scales[m],
+                                                          row0 + prow, p.groups, gr, p.N, mi0);
                 }
             }
             // ---- release the slot; the last warp out refills it with the
@@ -689,7 +701,7 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
             if (lane == 0) {
                 __threadfence_block();
                 const int prev = atomicAdd(&bars->done[r], 1);
-                if (prev == kRbWarps - 1) {
+                if (prev == WARPS - 1) {
                     __threadfence_block();
                     bars->done[r] = 0;
                     const int nsl = sl + SG;
@@ -715,11 +727,12 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
         for (int nt0 = 0; nt0 < NT; ++nt0) {
             // round nt0: tokens [8 nt0, 8 nt0 + 8)
 #pragma unroll
-            for (int i = 0; i < MT; ++i)
+            for (int i = 0; i < MTH; ++i)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
+                    if (MTH != MT && mi0 + i >= MT) break;   // (odd split)
                     const int tl = 2 * t + (e & 1);
-                    const int rr = 16 * i + 8 * (e >> 1) + prow;
+                    const int rr = 16 * (mi0 + i) + 8 * (e >> 1) + prow;
                     float v = 0.0f;
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
@@ -728,7 +741,7 @@ __global__ void __launch_bounds__(kRbThreads, 1) gemv_rb_kernel(const __grid_con
                 }
             __syncthreads();
             const int ntok = min(8, p.M - 8 * nt0);
-            for (int o = threadIdx.x; o < ntok * RB; o += kRbThreads) {
+            for (int o = threadIdx.x; o < ntok * RB; o += WARPS * 32) {
                 const int tl = o / RB;
                 const int rr = o - tl * RB;
                 float v = 0.0f;
@@ -773,10 +786,10 @@ struct RbPlan {
     bool three_d;
 };
 
-template <int FMT, int BITS, int MT, int NT, bool SSC>
-inline cudaError_t rb_launch(RbParams& prm, const RbPlan& P, const uint16_t* const* xs,
-                             const void* const* codes, int nmat, cudaStream_t s) {
-    auto kern = gemv_rb_kernel<FMT, BITS, MT, NT, SSC>;
+template <int FMT, int BITS, int MT, int NT, bool SSC, int WARPS>
+inline cudaError_t rb_launch_w(RbParams& prm, const RbPlan& P, const uint16_t* const* xs,
+                               const void* const* codes, int nmat, cudaStream_t s) {
+    auto kern = gemv_rb_kernel<FMT, BITS, MT, NT, SSC, WARPS>;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -823,7 +836,7 @@ inline cudaError_t rb_launch(RbParams& prm, const RbPlan& P, const uint16_t* con
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(P.grid), 1, 1);
-    cfg.blockDim = dim3(kRbThreads, 1, 1);
+    cfg.blockDim = dim3(WARPS * 32, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(P.smem);
     cfg.stream = s;
     cudaLaunchAttribute attrs[1];
@@ -836,6 +849,19 @@ inline cudaError_t rb_launch(RbParams& prm, const RbPlan& P, const uint16_t* con
     cfg.attrs = attrs;
     cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, kern, static_cast<const RbParams&>(prm));
+}
+
+// 16 warps (two halves splitting each block's m-tiles) measured faster only
+// for int4 at M <= 8 on rows of <= 2048 k with blocks of >= 3 m-tiles (fused
+// R/K/V 3 x 2048 x 2048: 4.08 -> 3.68 us; 8192 x 2048: 4.67 -> 4.22 us); with
+// longer rows, fewer m-tiles or int8 the 8-warp form is faster.
+template <int FMT, int BITS, int MT, int NT, bool SSC>
+inline cudaError_t rb_launch(RbParams& prm, const RbPlan& P, const uint16_t* const* xs,
+                             const void* const* codes, int nmat, cudaStream_t s) {
+    if constexpr (FMT == FMT_G64 && BITS == 4 && NT == 1 && MT >= 3) {
+        if (prm.K <= 2048) return rb_launch_w<FMT, BITS, MT, NT, SSC, 16>(prm, P, xs, codes, nmat, s);
+    }
+    return rb_launch_w<FMT, BITS, MT, NT, SSC, 8>(prm, P, xs, codes, nmat, s);
 }
 
 template <int FMT, int BITS, int NT, bool SSC>

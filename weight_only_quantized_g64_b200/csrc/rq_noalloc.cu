@@ -70,10 +70,6 @@ extern "C" rq_status rq_gemv_wq_noalloc(const uint16_t* x, int64_t M, int64_t K,
     const auto mis = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
     if (mis(x) || mis(codes) || mis(scales) || mis(y)) return RQ_ERR_ALIGN;
 
-    // large projections use 32-row tiles: reject shapes whose counters do not fit
-    const int64_t tiles = (N + 31) / 32;
-    if (tiles > static_cast<int64_t>(kMaxTiles)) return RQ_ERR_SHAPE;
-
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     WOperand w = {codes, scales, y};
     const int which = decode_kernel_for(M, K, N, bits, 1);
@@ -99,16 +95,8 @@ extern "C" rq_status rq_gemv_wq_noalloc(const uint16_t* x, int64_t M, int64_t K,
     }
     float* ws = reinterpret_cast<float*>(base);
     int* cnt = reinterpret_cast<int*>(base + kSlotBytes);
-    // The counters must start at zero; a completed launch leaves them at zero,
-    // an aborted one might not, so clear the ones this call uses.
-    // (row tiles are 16 to 64 rows: clear enough counters for the smallest)
-    const int64_t t16 = (N + 15) / 16;
-    const size_t n_clear = static_cast<size_t>(t16 < static_cast<int64_t>(kMaxTiles) ? t16 : kMaxTiles);
-    e = cudaMemsetAsync(cnt, 0, n_clear * sizeof(int), s);
-    if (e != cudaSuccess) {
-        record_cuda_error(e);
-        return RQ_ERR_CUDA;
-    }
+    // the launcher checks the scratch it needs against these sizes before it
+    // enqueues anything (then clears the counters it uses)
     bool too_large = false;
     GemvScratch sc = {ws, kSlotBytes, cnt, kMaxTiles, &too_large};
     e = launch_gemv_product_scratch(x, M, K, N, bits, &w, 1, s, &sc);
