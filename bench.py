@@ -403,8 +403,25 @@ def bench_quantizer(hbm_peak, reps=50):
         times.append(e0.elapsed_time(e1))
     ms = statistics.median(times)
     byts = N * K * 4 + synth.algorithmic_weight_bytes(N, K, 4)
+    # the E[x^2]-weighted scale search on the same shape, 7 candidates
+    # (offline work; also reads E[x^2] and writes the choices)
+    e2 = torch.rand(K, generator=torch.Generator(device="cuda").manual_seed(6), device="cuda") * 4.0
+    factors = torch.tensor([1.0, 0.95, 0.9, 0.85, 0.8, 0.75, 0.7], device="cuda")
+    rq.quantize_g64_ex2(W, e2, 4, factors, codes=codes, scales=scales)
+    t2 = []
+    for _ in range(max(5, reps // 5)):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        rq.quantize_g64_ex2(W, e2, 4, factors, codes=codes, scales=scales)
+        e1.record(s)
+        e1.synchronize()
+        t2.append(e0.elapsed_time(e1))
+    ms2 = statistics.median(t2)
     return {"shape": [N, K], "bits": 4, "ms": ms, "gbs": byts / ms / 1e6,
-            "frac": byts / ms / 1e6 / hbm_peak}
+            "frac": byts / ms / 1e6 / hbm_peak,
+            "e2_search": {"candidates": 7, "ms": ms2, "gbs": byts / ms2 / 1e6,
+                          "frac": byts / ms2 / 1e6 / hbm_peak}}
 
 
 def bench_gptq(reps=3):

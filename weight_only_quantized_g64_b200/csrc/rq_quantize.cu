@@ -55,15 +55,22 @@ __device__ __forceinline__ float max_nan(float a, float b) {
 // separates it from fl(q).  Near ties (weights on the grid) take the IEEE
 // division.  Rounding: t + 1.5 * 2^23 rounds to an integer, ties to even, for
 // |t| <= 2^22; its bit pattern minus that of 1.5 * 2^23 is the integer.
-template <int QMAX>
+//
+// With a normal fp16 scale the clamp never acts: s16 >= (amax / qmax)(1 -
+// 2^-11)(1 - 2^-24), so |t| <= qmax (1 + 5e-4) (1 + 2^-24) < qmax + 0.5, and
+// the same bound holds for the IEEE quotient; only subnormal scales (relative
+// rounding up to 1/2) need it (CLAMP).
+template <int QMAX, bool CLAMP>
 __device__ __forceinline__ int rint_quotient_q(float w, float sf, float r) {
     constexpr float kNear = static_cast<float>(QMAX + 1) * 4.76837158203125e-7f;   // 2^-21
     constexpr float kMagic = 12582912.0f;                                          // 1.5 * 2^23
-    const float t = fminf(fmaxf(__fmul_rn(w, r), static_cast<float>(-QMAX)), static_cast<float>(QMAX));
+    float t = __fmul_rn(w, r);
+    if constexpr (CLAMP) t = fminf(fmaxf(t, static_cast<float>(-QMAX)), static_cast<float>(QMAX));
     const float m = __fadd_rn(t, kMagic);
     const float d = __fsub_rn(t, __fsub_rn(m, kMagic));
     if (fabsf(__fsub_rn(fabsf(d), 0.5f)) > kNear) return __float_as_int(m) - __float_as_int(kMagic);
-    return max(-QMAX, min(QMAX, __float2int_rn(__fdiv_rn(w, sf))));
+    const int q = __float2int_rn(__fdiv_rn(w, sf));
+    return CLAMP ? max(-QMAX, min(QMAX, q)) : q;
 }
 
 // One group held by 8 lanes, 8 weights per lane (positions 4l..4l+3 and
@@ -95,8 +102,31 @@ __device__ __forceinline__ void quantize_group8(const float4 (&v)[2], unsigned m
         status = 6;  // RQ_ERR_RANGE
     } else if (sf != 0.0f) {
         const float r = __frcp_rn(sf);
+        if (sf >= 6.103515625e-05f) {
+            // normal fp16 scale: no clamp needed.  The fast value for every
+            // weight first, the near ties collected in a mask and redone with
+            // the IEEE division afterwards (rare), so the common path has no
+            // branch per weight.
+            constexpr float kNear = static_cast<float>(kQmax + 1) * 4.76837158203125e-7f;
+            constexpr float kMagic = 12582912.0f;
+            uint32_t slow = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) c[i] = rint_quotient_q<kQmax>(w[i], sf, r);
+            for (int i = 0; i < 8; ++i) {
+                const float t = __fmul_rn(w[i], r);
+                const float m = __fadd_rn(t, kMagic);
+                const float d = __fsub_rn(t, __fsub_rn(m, kMagic));
+                c[i] = __float_as_int(m) - __float_as_int(kMagic);
+                slow |= (fabsf(__fsub_rn(fabsf(d), 0.5f)) > kNear ? 0u : 1u) << i;
+            }
+            if (slow) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (slow & (1u << i)) c[i] = __float2int_rn(__fdiv_rn(w[i], sf));
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) c[i] = rint_quotient_q<kQmax, true>(w[i], sf, r);
+        }
     }
 }
 
@@ -214,75 +244,93 @@ cudaError_t launch_quantize(const float* W, int64_t n_groups, int bits, void* co
 // on a tie, and one whose scale overflows is never chosen (if every one
 // does, the group is quantized by RTN).
 //
-// Layout of the work: as the RTN kernel, 16 threads per group, one float4 of
-// weights and one of E[x^2] each.  Thread j evaluates candidate j (nf <= 16)
-// over all 64 weights, fetched by shuffles in k order, so its sum runs in the
-// same order as a scalar loop; lane 0 then scans the candidates in order
-// (the same comparisons as a sequential argmin, NaN included).
-template <int BITS>
+// Layout of the work: a team of TL lanes per group (16, or 8 when there are
+// at most 8 candidates, so a warp takes 2 or 4 groups at once).  Lane j
+// evaluates candidate j over all 64 weights in k order, reading the weights
+// and E[x^2] four at a time (the same address for every lane of the team:
+// one broadcast load), so its sum runs in the same order as a scalar loop;
+// the team's first lane then scans the candidates in order (the same
+// comparisons as a sequential argmin, NaN included).  Each lane also holds
+// 64 / TL weights of the group for the max and for the final codes.
+template <int BITS, int TL>
 __global__ void __launch_bounds__(256) quantize_g64_ex2_kernel(
     const float4* __restrict__ W, int64_t n_groups, int64_t groups_per_row,
     const float4* __restrict__ e2, const float* __restrict__ factors, int nf,
     uint8_t* __restrict__ codes, uint16_t* __restrict__ scales, int32_t* __restrict__ chosen,
     int* __restrict__ dev_status) {
     constexpr int kQmax = BITS == 4 ? 7 : 127;
-    const int lane16 = threadIdx.x & 15;
-    const int base = threadIdx.x & 16;                      // first lane of this half-warp
-    const unsigned half_mask = 0xFFFFu << base;
-    const int64_t first = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
-    const int64_t step = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
-    const float fj = lane16 < nf ? factors[lane16] : 1.0f;
+    constexpr int NV = 16 / TL;                              // float4 of weights per lane
+    const int lt = threadIdx.x & (TL - 1);                   // lane in the team
+    const int base = threadIdx.x & (31 & ~(TL - 1));         // first lane of the team
+    const unsigned tmask = (TL == 32 ? 0xFFFFFFFFu : ((1u << TL) - 1u)) << base;
+    const int64_t first = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / TL;
+    const int64_t step = (static_cast<int64_t>(gridDim.x) * blockDim.x) / TL;
+    const float fj = lt < nf ? factors[lt] : 1.0f;
 
     for (int64_t gid = first; gid < n_groups; gid += step) {
-        const float4 v = __ldcs(&W[gid * 16 + lane16]);
-        const float4 ev = __ldg(&e2[(gid % groups_per_row) * 16 + lane16]);
-        const bool finite = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
-        float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+        const float4* wg = W + gid * 16;
+        const float4* eg = e2 + (gid % groups_per_row) * 16;
+        float4 v[NV];
 #pragma unroll
-        for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(half_mask, a, off));
-        const bool all_finite = __all_sync(half_mask, finite);
+        for (int h = 0; h < NV; ++h) v[h] = __ldg(&wg[h * TL + lt]);
+        // max |w| over the group; NaN-propagating, so it also flags a
+        // non-finite weight (NaN or +inf exactly then)
+        float a = 0.0f;
+#pragma unroll
+        for (int h = 0; h < NV; ++h)
+            a = max_nan(max_nan(a, max_nan(fabsf(v[h].x), fabsf(v[h].y))),
+                        max_nan(fabsf(v[h].z), fabsf(v[h].w)));
+#pragma unroll
+        for (int off = TL / 2; off > 0; off >>= 1) a = max_nan(a, __shfl_xor_sync(tmask, a, off));
+        const bool all_finite = isfinite(a);
 
-        // ---- candidate lane16: scale, then its error over the 64 weights
+        // ---- candidate lt: scale, then its error over the 64 weights in order
         const float a32 = __fmul_rn(a, fj);
         const __half s16j = __float2half_rn(__fdiv_rn(a32, static_cast<float>(kQmax)));
         const float sfj = __half2float(s16j);
-        const bool valid = lane16 < nf && __half_as_ushort(s16j) != 0x7C00u;
+        const bool valid = lt < nf && __half_as_ushort(s16j) != 0x7C00u;
         const float rj = (sfj != 0.0f && valid) ? __frcp_rn(sfj) : 0.0f;
-        const float wv[4] = {v.x, v.y, v.z, v.w};
-        const float evv[4] = {ev.x, ev.y, ev.z, ev.w};
         float err = 0.0f;
-#pragma unroll 4
-        for (int k = 0; k < 64; ++k) {
-            const float wk = __shfl_sync(half_mask, wv[k & 3], base + (k >> 2));
-            const float ek = __shfl_sync(half_mask, evv[k & 3], base + (k >> 2));
-            int c = 0;
-            if (sfj != 0.0f) c = max(-kQmax, min(kQmax, rint_quotient(wk, sfj, rj)));
-            const float t = __fmul_rn(static_cast<float>(c), sfj);
-            const float d = __fsub_rn(wk, t);
-            err = __fadd_rn(err, __fmul_rn(ek, __fmul_rn(d, d)));
+        if (all_finite) {
+#pragma unroll 2
+            for (int k4 = 0; k4 < 16; ++k4) {
+                const float4 wq = __ldg(&wg[k4]);
+                const float4 eq = __ldg(&eg[k4]);
+                const float wk[4] = {wq.x, wq.y, wq.z, wq.w};
+                const float ek[4] = {eq.x, eq.y, eq.z, eq.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int c = sfj != 0.0f ? rint_quotient_q<kQmax, true>(wk[i], sfj, rj) : 0;
+                    const float t = __fmul_rn(static_cast<float>(c), sfj);
+                    const float d = __fsub_rn(wk[i], t);
+                    err = __fadd_rn(err, __fmul_rn(ek[i], __fmul_rn(d, d)));
+                }
+            }
         }
-        // ---- lane 0 scans the candidates in order (a sequential argmin)
+        // ---- the team's first lane scans the candidates in order
         int best = -1;
         float best_err = 0.0f;
         for (int j = 0; j < nf; ++j) {
-            const float ej = __shfl_sync(half_mask, err, base + j);
-            const int vj = __shfl_sync(half_mask, valid ? 1 : 0, base + j);
+            const float ej = __shfl_sync(tmask, err, base + j);
+            const int vj = __shfl_sync(tmask, valid ? 1 : 0, base + j);
             if (vj && (best < 0 || ej < best_err)) {
                 best = j;
                 best_err = ej;
             }
         }
-        best = __shfl_sync(half_mask, best, base);
+        best = __shfl_sync(tmask, best, base);
 
         // ---- the chosen scale (or RTN when no candidate is valid) and codes
-        const float fb = best >= 0 ? __shfl_sync(half_mask, fj, base + best) : 1.0f;
+        const float fb = best >= 0 ? __shfl_sync(tmask, fj, base + best) : 1.0f;
         const float s32 = best >= 0 ? __fdiv_rn(__fmul_rn(a, fb), static_cast<float>(kQmax))
                                     : __fdiv_rn(a, static_cast<float>(kQmax));
         const __half s16 = __float2half_rn(s32);
         uint16_t s_bits = __half_as_ushort(s16);
         const float sf = __half2float(s16);
         int status = 0;
-        int c[4] = {0, 0, 0, 0};
+        int c[4 * NV];
+#pragma unroll
+        for (int i = 0; i < 4 * NV; ++i) c[i] = 0;
         if (!all_finite) {
             s_bits = 0x7E00u;
             status = 5;  // RQ_ERR_NONFINITE
@@ -291,19 +339,27 @@ __global__ void __launch_bounds__(256) quantize_g64_ex2_kernel(
         } else if (sf != 0.0f) {
             const float r = __frcp_rn(sf);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) c[i] = max(-kQmax, min(kQmax, rint_quotient(wv[i], sf, r)));
+            for (int h = 0; h < NV; ++h) {
+                const float wv[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) c[4 * h + i] = rint_quotient_q<kQmax, true>(wv[i], sf, r);
+            }
         }
-        if (BITS == 4) {
-            const uint16_t packed = static_cast<uint16_t>((c[0] & 0xF) | ((c[1] & 0xF) << 4) |
-                                                          ((c[2] & 0xF) << 8) |
-                                                          ((c[3] & 0xF) << 12));
-            __stcs(reinterpret_cast<unsigned short*>(codes + gid * 32 + lane16 * 2), packed);
-        } else {
-            const uint32_t packed = (c[0] & 0xFF) | ((c[1] & 0xFF) << 8) | ((c[2] & 0xFF) << 16) |
-                                    (static_cast<uint32_t>(c[3] & 0xFF) << 24);
-            __stcs(reinterpret_cast<unsigned int*>(codes + gid * 64 + lane16 * 4), packed);
+#pragma unroll
+        for (int h = 0; h < NV; ++h) {
+            const int* ch = c + 4 * h;
+            const int pos = h * TL + lt;                     // float4 index within the group
+            if (BITS == 4) {
+                const uint16_t packed = static_cast<uint16_t>((ch[0] & 0xF) | ((ch[1] & 0xF) << 4) |
+                                                              ((ch[2] & 0xF) << 8) | ((ch[3] & 0xF) << 12));
+                __stcs(reinterpret_cast<unsigned short*>(codes + gid * 32 + pos * 2), packed);
+            } else {
+                const uint32_t packed = (ch[0] & 0xFF) | ((ch[1] & 0xFF) << 8) | ((ch[2] & 0xFF) << 16) |
+                                        (static_cast<uint32_t>(ch[3] & 0xFF) << 24);
+                __stcs(reinterpret_cast<unsigned int*>(codes + gid * 64 + pos * 4), packed);
+            }
         }
-        if (lane16 == 0) {
+        if (lt == 0) {
             scales[gid] = s_bits;
             if (chosen != nullptr) chosen[gid] = (all_finite && best >= 0) ? best : 0;
             if (dev_status != nullptr) {
@@ -314,27 +370,36 @@ __global__ void __launch_bounds__(256) quantize_g64_ex2_kernel(
     }
 }
 
+template <int BITS, int TL>
+static cudaError_t launch_ex2_cfg(const float* W, int64_t n_groups, int64_t groups_per_row,
+                                  const float* e2, const float* factors, int nf, void* codes,
+                                  uint16_t* scales, int32_t* chosen, int* dev_status, cudaStream_t s) {
+    auto kern = quantize_g64_ex2_kernel<BITS, TL>;
+    // (quantize_grid counts 32 groups per block of 256 threads: a block holds
+    // 256 / TL groups here)
+    const int blocks = quantize_grid(n_groups * TL / 8, reinterpret_cast<const void*>(kern));
+    kern<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        reinterpret_cast<const float4*>(W), n_groups, groups_per_row,
+        reinterpret_cast<const float4*>(e2), factors, nf, static_cast<uint8_t*>(codes), scales,
+        chosen, dev_status);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_ex2(const float* W, int64_t N, int64_t K, int bits, const float* e2,
                                 const float* factors, int nf, void* codes, uint16_t* scales,
                                 int32_t* chosen, int* dev_status, cudaStream_t s) {
     const int64_t groups_per_row = K / kGroup;
     const int64_t n_groups = N * groups_per_row;
     if (n_groups <= 0) return cudaSuccess;
-    const int threads = 256;
-    const int blocks = quantize_grid(
-        n_groups, bits == 4 ? reinterpret_cast<const void*>(quantize_g64_ex2_kernel<4>)
-                            : reinterpret_cast<const void*>(quantize_g64_ex2_kernel<8>));
     if (bits == 4)
-        quantize_g64_ex2_kernel<4><<<static_cast<unsigned>(blocks), threads, 0, s>>>(
-            reinterpret_cast<const float4*>(W), n_groups, groups_per_row,
-            reinterpret_cast<const float4*>(e2), factors, nf, static_cast<uint8_t*>(codes), scales,
-            chosen, dev_status);
-    else
-        quantize_g64_ex2_kernel<8><<<static_cast<unsigned>(blocks), threads, 0, s>>>(
-            reinterpret_cast<const float4*>(W), n_groups, groups_per_row,
-            reinterpret_cast<const float4*>(e2), factors, nf, static_cast<uint8_t*>(codes), scales,
-            chosen, dev_status);
-    return cudaGetLastError();
+        return nf <= 8 ? launch_ex2_cfg<4, 8>(W, n_groups, groups_per_row, e2, factors, nf, codes, scales,
+                                              chosen, dev_status, s)
+                       : launch_ex2_cfg<4, 16>(W, n_groups, groups_per_row, e2, factors, nf, codes, scales,
+                                               chosen, dev_status, s);
+    return nf <= 8 ? launch_ex2_cfg<8, 8>(W, n_groups, groups_per_row, e2, factors, nf, codes, scales,
+                                          chosen, dev_status, s)
+                   : launch_ex2_cfg<8, 16>(W, n_groups, groups_per_row, e2, factors, nf, codes, scales,
+                                           chosen, dev_status, s);
 }
 
 }  // namespace rq
