@@ -109,7 +109,8 @@ def test_decode_kernel_choice(L):
     so the SM count is taken as 148).  Launches with at least one 16-row
     m-tile per SM (the fused R/K/V and the channel-mix key of the 1.5B-shaped
     layer, every projection of the 13.3B-shaped one): the row-block kernel,
-    except M > 16 on rows of >= 16384 k (the tensor-core kernel).  Fewer
+    except M > 16 on rows of >= 16384 k or launches of >= 16384 rows (the
+    tensor-core kernel).  Fewer
     m-tiles: row tiles for M <= 8, row blocks for M 9..16 and for M > 16 on
     rows of <= 4096 k, the cluster kernel for M > 16 on longer rows."""
     D = 2048
@@ -123,11 +124,14 @@ def test_decode_kernel_choice(L):
         assert rq.decode_kernel_for(M, D, D, 4, 1) == small, M                          # o
         assert rq.decode_kernel_for(M, 4 * D, D, 4, 1) == (
             small if M <= 16 else "cluster"), M                                          # value
-    # the 13.3B-shaped layer (D = 4096): row blocks, the value projection at M > 16 on tensor cores
+    # the 13.3B-shaped layer (D = 4096): row blocks, the key and value
+    # projections (16384 rows, 16384-long rows) at M > 16 on tensor cores
     for M in (1, 8, 16, 17, 32):
-        for N, K, nmat in ((4096, 4096, 3), (4096, 4096, 1), (16384, 4096, 1)):
+        for N, K, nmat in ((4096, 4096, 3), (4096, 4096, 1)):
             assert rq.decode_kernel_for(M, K, N, 4, nmat) == "rowblock", (M, N, K)
-        assert rq.decode_kernel_for(M, 16384, 4096, 4, 1) == ("tensor" if M > 16 else "rowblock")
+        big = "tensor" if M > 16 else "rowblock"
+        assert rq.decode_kernel_for(M, 16384, 4096, 4, 1) == big
+        assert rq.decode_kernel_for(M, 4096, 16384, 4, 1) == big
     # the boundary: 148 m-tiles (2368 rows) in the launch
     assert rq.decode_kernel_for(1, D, 2368, 4, 1) == "rowblock"
     assert rq.decode_kernel_for(1, D, 2352, 4, 1) == "rowtile"

@@ -48,14 +48,17 @@ int decode_kernel_for(int64_t M, int64_t K, int64_t N, int bits, int nmat) {
     if (g_decode_kernel == RQ_DECODE_TENSOR) return tcs_fits(M, K, N, bits) ? RQ_DECODE_TENSOR : -1;
     // measured on B200 (graph-replayed chains with PDL, int4 and int8):
     // * at least one 16-row m-tile per SM: the row-block kernel, except for
-    //   M > 16 on rows of >= 16384 k, where the MMA work of mma.sync makes the
-    //   tensor-core kernel faster (4096 x 16384 at M = 32: 26.0 vs 29.5 us);
+    //   M > 16 on rows of >= 16384 k or launches of >= 16384 rows, where the
+    //   MMA work of mma.sync makes the tensor-core kernel faster (at M = 32:
+    //   4096 x 16384 23.8 vs 29.5 us, 16384 x 4096 20.4 vs 20.9 us);
     // * fewer m-tiles than SMs: the row-tile kernel (which also splits K) for
     //   M <= 8; the row-block kernel for M 9..16 and for M > 16 on rows of
     //   <= 4096 k; the cluster kernel for M > 16 on longer rows.
     const int64_t mtiles = static_cast<int64_t>(nmat) * ((N + 15) / 16);
     if (mtiles >= num_sms()) {
-        if (M > 16 && K >= 16384 && tcs_fits(M, K, N, bits)) return RQ_DECODE_TENSOR;
+        if (M > 16 && (K >= 16384 || static_cast<int64_t>(nmat) * N >= 16384) &&
+            tcs_fits(M, K, N, bits))
+            return RQ_DECODE_TENSOR;
         if (gemv_rowblock_fits(M, K, N, bits, nmat)) return RQ_DECODE_ROWBLOCK;
     } else if (M > 8 && (M <= 16 || K <= 4096) && gemv_rowblock_fits(M, K, N, bits, nmat)) {
         return RQ_DECODE_ROWBLOCK;

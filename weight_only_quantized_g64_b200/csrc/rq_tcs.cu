@@ -25,7 +25,9 @@
 //   warp 1      TMEM allocator and MMA issuer: per unit two 128-row MMAs
 //               (tcgen05.mma kind::f16, M = 128, N = BNT, 4 steps of K = 16)
 //               accumulating in TMEM.
-//   warps 2-5   epilogue: tcgen05.ld of the accumulators, then y (or the
+//   warps 2-5   (int4) while the accumulators fill, put each stage's x
+//               tiles into the pair order of the unpacking; then the
+//               epilogue: tcgen05.ld of the accumulators, then y (or the
 //               partial sums into shared memory for the cluster sum, which
 //               all threads then share).
 //   warps 6-21  four dequantiser groups of four warps; group g takes units
@@ -38,10 +40,10 @@
 // (p0,p4), (p1,p5), (p2,p6), (p3,p7) with one lop3 each (bit placement of Kim
 // et al., arXiv:2211.10017: low nibbles as 1024 + c + 8, high nibbles as
 // 64 + c + 8), an exact fp16 subtraction and the fp16 scale product.  That
-// pair order is a permutation of k inside each 8-k chunk; the dequantiser
-// group applies the same permutation to the unit's x tile in shared memory
-// (each 16-byte chunk in place, which the swizzle leaves intact) before the
-// MMAs read it, so the sum over k is unchanged.
+// pair order is a permutation of k inside each 8-k chunk; the epilogue warps
+// apply the same permutation to each stage's x tiles in shared memory (each
+// 16-byte chunk in place, which the swizzle leaves intact) before the MMAs
+// read them, so the sum over k is unchanged.
 //
 // Numerics: A = fp16(code * s16) (one rounding), fp32 accumulation in the
 // tensor core, partial sums added in fp32 in k order.
@@ -104,7 +106,7 @@ struct TcsCfg {
     static constexpr int kColsNeeded = kACol0 + kSA * 64;
     static constexpr int kTmemCols = 512;
     static constexpr int kChunks = kCodeBytes / 16;               // 16-byte code chunks per group
-    static constexpr int kBars = 2 * kSS + 2 * kSA + 1;
+    static constexpr int kBars = 3 * kSS + 2 * kSA + 1;
     static constexpr int kSmem = 1024 + kRing + kBars * 8 + 64;
     static_assert(kSS >= 2, "ring too shallow");
     static_assert(kColsNeeded <= 512 && kSA > kTcsG, "TMEM layout");
@@ -189,7 +191,8 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
     uint64_t* afull = bars + 2 * SS;         // [SA] A stage written
     uint64_t* aempty = bars + 2 * SS + SA;   // [SA] MMAs reading the A stage done
     uint64_t* accfull = bars + 2 * SS + 2 * SA;      // accumulators complete
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accfull + 1);
+    uint64_t* xready = accfull + 1;                   // [SS] (int4) x tiles put in pair order
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xready + SS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -221,6 +224,7 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
             mbar_init(&aempty[a], 1);
         }
         mbar_init(accfull, 1);
+        for (int s = 0; s < SS; ++s) mbar_init(&xready[s], 4);
         *abort_flag = 0;
         fence_mbar_init();
         // codes never depend on the previous kernel: the first stages' go out
@@ -302,6 +306,10 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
                 if (i % KS == 0 && !mbar_wait(&full[s], static_cast<uint32_t>(j / SS) & 1u, abort_flag,
                                               p.timeout_ns, p.status))
                     break;
+                if (BITS == 4 && i % KS == 0 &&
+                    !mbar_wait(&xready[s], static_cast<uint32_t>(j / SS) & 1u, abort_flag,
+                               p.timeout_ns, p.status))
+                    break;
                 if (!mbar_wait(&afull[a], static_cast<uint32_t>(i / SA) & 1u, abort_flag,
                                p.timeout_ns, p.status))
                     break;
@@ -326,6 +334,34 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
         const int r0 = q * 32 + lane;               // row of tile 0; tile 1: + 128
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
         pdl_wait();                                 // y: after the previous grid
+        if constexpr (BITS == 4) {
+            // While the accumulators fill, these warps put every stage's x
+            // tiles into the pair order of the int4 unpacking (each 16-byte
+            // chunk in place; the swizzle moves whole chunks), off the
+            // dequantisers' path; the MMAs wait for it per stage.
+            const int et = threadIdx.x - 64;        // 0 .. 127
+            for (int j = 0; j < n_stages; ++j) {
+                const int s = j % SS;
+                if (!mbar_wait(&full[s], static_cast<uint32_t>(j / SS) & 1u, abort_flag, p.timeout_ns,
+                               p.status))
+                    break;
+                uint8_t* xs = ring + s * Cfg::kStage;
+                for (int ch = et; ch < KS * BNT * 8; ch += 128) {
+                    uint4* xp = reinterpret_cast<uint4*>(xs + ch * 16);
+                    const uint4 xv = *xp;
+                    uint4 o;
+                    o.x = __byte_perm(xv.x, xv.z, 0x5410);
+                    o.y = __byte_perm(xv.x, xv.z, 0x7632);
+                    o.z = __byte_perm(xv.y, xv.w, 0x5410);
+                    o.w = __byte_perm(xv.y, xv.w, 0x7632);
+                    *xp = o;
+                }
+                // the MMAs read x through the async proxy
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xready[s]);
+            }
+        }
         // (suspending between checks: these warps wait for most of the kernel)
         const bool ok = mbar_wait_suspend(accfull, 0, abort_flag, p.timeout_ns, p.status);
         tc_fence_after();
@@ -366,7 +402,6 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
         // ---------------------------------------- dequantise into TMEM --
         const int q = warp & 3;                     // TMEM lane quarter
         const int r0 = q * 32 + lane;
-        const int tg = (dw & 3) * 32 + lane;        // thread within the group
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
         // scales of this thread's rows for unit i (0 outside the matrix and
         // past the row's last k group)
@@ -394,22 +429,6 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
 #pragma unroll
                 for (int c = 0; c < Cfg::kChunks; ++c)
                     v[tt][c] = tcs_code_chunk(wt, tt * 128 + r0, kj * Cfg::kChunks + c);
-            if constexpr (BITS == 4) {
-                // this k group's x chunks into the pair order of the unpacking
-                uint8_t* xt = st + kj * Cfg::kXTile;
-                for (int ch = tg; ch < BNT * 8; ch += 128) {
-                    uint4* xp = reinterpret_cast<uint4*>(xt + ch * 16);
-                    const uint4 xv = *xp;
-                    uint4 o;
-                    o.x = __byte_perm(xv.x, xv.z, 0x5410);
-                    o.y = __byte_perm(xv.x, xv.z, 0x7632);
-                    o.z = __byte_perm(xv.y, xv.w, 0x5410);
-                    o.w = __byte_perm(xv.y, xv.w, 0x7632);
-                    *xp = o;
-                }
-                // the MMAs read x through the async proxy
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
             if (i >= SA && !mbar_wait(&aempty[a], static_cast<uint32_t>(i / SA - 1) & 1u, abort_flag,
