@@ -112,7 +112,11 @@ struct TcsCfg {
     static_assert(kColsNeeded <= 512 && kSA > kTcsG, "TMEM layout");
     static_assert(kXTile % 1024 == 0 && kWStage % 1024 == 0, "stage alignment");
     static_assert(kSmem <= 227 * 1024, "shared memory");
-    static_assert(kRing >= 64 * kTcsRows * 4, "the partial sums reuse the ring");
+    // partial sums of a split K: [256 rows][kRedStride] fp32 in the ring, a
+    // row's tokens contiguous (16-byte stores and loads); the 4-float pad
+    // spreads consecutive rows over the banks
+    static constexpr int kRedStride = BNT + 4;
+    static_assert(kRing >= kTcsRows * kRedStride * 4, "the partial sums reuse the ring");
 };
 
 // 16-byte chunk c of row r of the codes box (128-byte rows, 128-byte swizzle:
@@ -366,7 +370,7 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
         const bool ok = mbar_wait_suspend(accfull, 0, abort_flag, p.timeout_ns, p.status);
         tc_fence_after();
         if (ok && !*abort_flag) {
-            float* red = reinterpret_cast<float*>(ring);     // [M][256] when ks > 1
+            float* red = reinterpret_cast<float*>(ring);     // [256][kRedStride] when ks > 1
 #pragma unroll 1
             for (int tt = 0; tt < 2; ++tt) {
                 const int r = tt * 128 + r0;
@@ -376,14 +380,21 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
                     uint32_t v[16];
                     tmem_ld_32x32b_x16(lane_base + tt * BNT + j0, v);
                     tc_wait_ld();
+                    if (ks > 1) {
+                        // the row's 16 token sums (those past M are never read)
+                        float4* dst = reinterpret_cast<float4*>(red + r * Cfg::kRedStride + j0);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            dst[u] = make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
+                                                 __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
+                        continue;
+                    }
 #pragma unroll
                     for (int jj = 0; jj < 16; ++jj) {
                         const int m = j0 + jj;
                         if (m >= p.M) break;
                         float val = __uint_as_float(v[jj]);
-                        if (ks > 1) {
-                            red[m * kTcsRows + r] = val;
-                        } else if (n < p.N) {
+                        if (n < p.N) {
                             if (p.epi == 1) {
                                 val = fmaxf(val, 0.0f);
                                 val = val * val;
@@ -458,26 +469,40 @@ __global__ void __launch_bounds__(kTcsThreads, 1) tcs_kernel(const __grid_consta
         // cluster barriers on every path.
         cluster_sync();
         if (!*abort_flag) {
-            const int E4 = p.M * (kTcsRows / 4);                 // float4 groups of the block
+            // element e: rows fastest (so a warp's y stores are 32
+            // consecutive n), then groups of 4 tokens
+            const int MQ = (p.M + 3) / 4;
+            const int E4 = MQ * kTcsRows;
             const int e0 = static_cast<int>((static_cast<int64_t>(kq) * E4) / ks);
             const int e1 = static_cast<int>((static_cast<int64_t>(kq + 1) * E4) / ks);
             const uint32_t red_local = smem_u32(ring);
             for (int e = e0 + static_cast<int>(threadIdx.x); e < e1; e += kTcsThreads) {
+                const int m4 = e / kTcsRows;
+                const int r = e - m4 * kTcsRows;
+                const uint32_t off = static_cast<uint32_t>(r * Cfg::kRedStride + 4 * m4) * 4u;
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int src = 0; src < ks; ++src) {
-                    const float4 v = ld_dsmem_f32x4(map_to_rank(red_local + e * 16, src));
-                    acc.x += v.x;
-                    acc.y += v.y;
-                    acc.z += v.z;
-                    acc.w += v.w;
+                for (int src0 = 0; src0 < ks; src0 += 4) {
+                    // four ranks' loads in flight at once, added in rank order
+                    float4 v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (src0 + u < ks) v[u] = ld_dsmem_f32x4(map_to_rank(red_local + off, src0 + u));
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (src0 + u < ks) {
+                            acc.x += v[u].x;
+                            acc.y += v[u].y;
+                            acc.z += v[u].z;
+                            acc.w += v[u].w;
+                        }
                 }
-                const int m = (e * 4) / kTcsRows;
-                const int r = (e * 4) - m * kTcsRows;
-                float out[4] = {acc.x, acc.y, acc.z, acc.w};
+                const int n = rb * kTcsRows + r;
+                if (n >= p.N) continue;
+                const float out[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int n = rb * kTcsRows + r + u;
-                    if (n >= p.N) continue;
+                    const int m = 4 * m4 + u;
+                    if (m >= p.M) break;
                     float val = out[u];
                     if (p.epi == 1) {
                         val = fmaxf(val, 0.0f);
