@@ -60,7 +60,7 @@ DECODE_SOURCES = ("rq_api.cu", "rq_gemv.cu", "rq_gemv_ck.cu", "rq_gemv_unit.cuh"
                   "rq_gemv_rb_g64_8.cu", "rq_tcs.cu")
 KERNEL_NAMES = {"rowtile": "gemv_wq_kernel (row tiles)", "cluster": "gemv_ck_kernel (cluster split-K)",
                 "rowblock": "gemv_rb_kernel (row blocks)", "tensor": "tcs_kernel (tcgen05, K split over a cluster)"}
-DECODE_TRAFFIC = {"code_sha256_16": "c2f67e878ff169f2", "dram_per_algorithmic_byte": 35697920 / 35651584}
+DECODE_TRAFFIC = {"code_sha256_16": "9bba2ce732bb77a5", "dram_per_algorithmic_byte": 35697920 / 35651584}
 
 
 def decode_code_hash():
