@@ -74,7 +74,8 @@ __device__ __forceinline__ int rint_quotient_q(float w, float sf, float r) {
 }
 
 // One group held by 8 lanes, 8 weights per lane (positions 4l..4l+3 and
-// 32+4l..32+4l+3 of the group): scale bits, codes, status (0, 5 = NONFINITE,
+// 32+4l..32+4l+3 of the group): scale bits, codes (only their low 4 / 8 bits
+// are meaningful: the packing keeps just those), status (0, 5 = NONFINITE,
 // 6 = RANGE).
 template <int BITS>
 __device__ __forceinline__ void quantize_group8(const float4 (&v)[2], unsigned mask8,
@@ -104,24 +105,31 @@ __device__ __forceinline__ void quantize_group8(const float4 (&v)[2], unsigned m
         const float r = __frcp_rn(sf);
         if (sf >= 6.103515625e-05f) {
             // normal fp16 scale: no clamp needed.  The fast value for every
-            // weight first, the near ties collected in a mask and redone with
-            // the IEEE division afterwards (rare), so the common path has no
-            // branch per weight.
-            constexpr float kNear = static_cast<float>(kQmax + 1) * 4.76837158203125e-7f;
+            // weight first; if any of the lane's weights is a near tie, those
+            // are redone with the IEEE division afterwards (rare), so the
+            // common path has no branch per weight.  d = t - rint(t) is exact
+            // and |d| <= 1/2, so "more than kNear away from a half-integer"
+            // is |d| < 1/2 - kNear (exact in fp32).  The code is taken from
+            // the low bits of m: m's bit pattern is that of 1.5 * 2^23 plus
+            // the integer, and 1.5 * 2^23 has zero low bytes.
+            constexpr float kTie = 0.5f - static_cast<float>(kQmax + 1) * 4.76837158203125e-7f;
             constexpr float kMagic = 12582912.0f;
-            uint32_t slow = 0;
+            bool any_slow = false;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float t = __fmul_rn(w[i], r);
                 const float m = __fadd_rn(t, kMagic);
                 const float d = __fsub_rn(t, __fsub_rn(m, kMagic));
-                c[i] = __float_as_int(m) - __float_as_int(kMagic);
-                slow |= (fabsf(__fsub_rn(fabsf(d), 0.5f)) > kNear ? 0u : 1u) << i;
+                c[i] = __float_as_int(m);
+                any_slow |= fabsf(d) >= kTie;
             }
-            if (slow) {
+            if (any_slow) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    if (slow & (1u << i)) c[i] = __float2int_rn(__fdiv_rn(w[i], sf));
+                for (int i = 0; i < 8; ++i) {
+                    const float t = __fmul_rn(w[i], r);
+                    const float d = __fsub_rn(t, __fsub_rn(__fadd_rn(t, kMagic), kMagic));
+                    if (fabsf(d) >= kTie) c[i] = __float2int_rn(__fdiv_rn(w[i], sf));
+                }
             }
         } else {
 #pragma unroll
