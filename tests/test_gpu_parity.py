@@ -96,6 +96,40 @@ def test_quantizer_special_values(bits):
     assert np.array_equal(to_host(codes2), c2)
 
 
+@pytest.mark.parametrize("bits", [4, 8])
+def test_quantizer_near_ties(bits):
+    """Weights at and a few ulps around half-integer multiples of the scale,
+    where w * (1/s) and the IEEE quotient w / s can round to different
+    integers: exact scales (powers of two) and inexact ones, on both sides of
+    every half-integer of the code range."""
+    qmax = 7 if bits == 4 else 127
+    rng = np.random.default_rng(91)
+    groups = []
+    for gi in range(512):
+        # group max q_max * s sets the scale; exact for the first half
+        s = np.float32(2.0 ** -rng.integers(2, 9)) if gi < 256 else np.float32(rng.uniform(1e-3, 0.2))
+        g = np.empty(64, np.float32)
+        g[0] = np.float32(qmax) * s * (1 if gi % 2 else -1)
+        k = rng.integers(-qmax, qmax, size=63).astype(np.float32) + np.float32(0.5)
+        base = (k * s).astype(np.float32)
+        ulps = rng.integers(-6, 7, size=63)
+        v = base.copy()
+        for u in range(1, 7):       # move |ulps| steps towards +inf or -inf
+            up = ulps >= u
+            dn = ulps <= -u
+            v[up] = np.nextafter(v[up], np.float32(np.inf))
+            v[dn] = np.nextafter(v[dn], np.float32(-np.inf))
+        g[1:] = v
+        groups.append(g)
+    W = np.stack(groups).reshape(16, 32 * 64)
+    codes, scales = rq.quantize_g64(torch.from_numpy(W).cuda(), bits)
+    c_ref, s_ref, st = oracle.quantize_g64(W, bits)
+    torch.cuda.synchronize()
+    assert st == 0
+    assert np.array_equal(to_host(scales).view(np.uint16), s_ref)
+    assert np.array_equal(to_host(codes), c_ref)
+
+
 # -------------------------------------------------------------- products ---
 
 def product_case(N, K, bits, M, seed, massive=None):
