@@ -73,6 +73,23 @@ __device__ __forceinline__ int rint_quotient_q(float w, float sf, float r) {
     return CLAMP ? max(-QMAX, min(QMAX, q)) : q;
 }
 
+// rint_quotient_q<QMAX, true> returned as the float value of the code (for
+// the error sums of the scale search): q = (t + 1.5 * 2^23) - 1.5 * 2^23 is
+// rint(t) exactly, with no integer conversion on the common path; the
+// near-tie test is the one comparison |t - q| >= 1/2 - (QMAX + 1) 2^-21 (t - q
+// is exact and at most 1/2 in magnitude), the same decision as above.
+template <int QMAX>
+__device__ __forceinline__ float rint_quotient_qf(float w, float sf, float r) {
+    constexpr float kTie = 0.5f - static_cast<float>(QMAX + 1) * 4.76837158203125e-7f;
+    constexpr float kMagic = 12582912.0f;                                          // 1.5 * 2^23
+    float t = __fmul_rn(w, r);
+    t = fminf(fmaxf(t, static_cast<float>(-QMAX)), static_cast<float>(QMAX));
+    const float q = __fsub_rn(__fadd_rn(t, kMagic), kMagic);
+    if (fabsf(__fsub_rn(t, q)) < kTie) return q;
+    const int qi = __float2int_rn(__fdiv_rn(w, sf));
+    return static_cast<float>(max(-QMAX, min(QMAX, qi)));
+}
+
 // One group held by 8 lanes, 8 weights per lane (positions 4l..4l+3 and
 // 32+4l..32+4l+3 of the group): scale bits, codes (only their low 4 / 8 bits
 // are meaningful: the packing keeps just those), status (0, 5 = NONFINITE,
@@ -308,8 +325,8 @@ __global__ void __launch_bounds__(256) quantize_g64_ex2_kernel(
                 const float ek[4] = {eq.x, eq.y, eq.z, eq.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int c = sfj != 0.0f ? rint_quotient_q<kQmax, true>(wk[i], sfj, rj) : 0;
-                    const float t = __fmul_rn(static_cast<float>(c), sfj);
+                    const float cf = sfj != 0.0f ? rint_quotient_qf<kQmax>(wk[i], sfj, rj) : 0.0f;
+                    const float t = __fmul_rn(cf, sfj);
                     const float d = __fsub_rn(wk[i], t);
                     err = __fadd_rn(err, __fmul_rn(ek[i], __fmul_rn(d, d)));
                 }
